@@ -1,0 +1,364 @@
+#!/usr/bin/env python
+"""Throughput of the SchNet energy + force + integrate path on B200.
+
+One step = one BAOAB Langevin step of every replica (B-A-O-A, forward over all
+interactions, backward for forces, closing B), with the neighbour list rebuilt
+every n_rebuild steps (its cost amortised inside the timed steps).  Workload
+(default): 64 replicas x 269-bead compact chains, F=128, 50 Gaussians on
+0-15 A, cutoff 15 A, 3 interactions, skin 2 A, rebuild every 20 steps, dt 4 fs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+With N > 1 (torchrun) every rank simulates its own replica batch (weak
+scaling, no data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "atom-steps/s & ns/day (SchNet E+F+integrate, 1 B200); HBM GB/s % of peak"
+KB = 0.0019872041            # kcal/mol/K
+ACC = 4.184e-4               # (kcal/mol/A)/amu -> A/fs^2
+FWD_FLOP_PER_EDGE = None     # set from the workload: 2 (K F + F^2)
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    def __init__(self, index=0):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(index), f"--query-gpu={q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        self.p.wait(timeout=10)
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            t = [x.strip() for x in line.split(",")]
+            if len(t) < 8:
+                continue
+            try:
+                sm.append(float(t[0])); mx.append(float(t[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, t[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _workload(name):
+    from schnet_gnn_molecular_b200 import workloads
+    if name in workloads.ALL:
+        return workloads.ALL[name]
+    if name.startswith("cg_protein_") and name.endswith("x269"):
+        return workloads.sweep(int(name[len("cg_protein_"):-len("x269")]))
+    if name.startswith("cg_globule_"):
+        return workloads.globule(int(name[len("cg_globule_"):]))
+    raise SystemExit(f"unknown workload {name}")
+
+
+def _inputs(w, rank):
+    from schnet_gnn_molecular_b200 import workloads
+    wr = w.with_(seed=w.seed + 100000 * rank) if rank else w
+    pos = workloads.positions(wr)
+    types = workloads.types(wr)
+    weights = workloads.weights(w)            # same model on every rank
+    mass = workloads.masses(wr)
+    vel = (workloads.velocity_normals(wr) * np.sqrt(KB * w.temperature * ACC / w.mass)).astype(np.float32)
+    return pos, types, weights, mass, vel
+
+
+def cpu_baseline(w, seconds: float):
+    """The float64 oracle timed on this host on whole replicas (one MD step each)."""
+    import oracle
+    from schnet_gnn_molecular_b200 import workloads
+    pos, types, weights, mass, vel = _inputs(w, 0)
+    om = oracle.Model(n_types=w.n_types, F=w.F, K=w.K, L=w.L, rbf_min=w.rbf_min, rbf_max=w.rbf_max,
+                      rbf_sigma=w.rbf_sigma, cutoff=w.cutoff, weights=weights, periodic=w.periodic,
+                      box=(w.box,) * 3 if w.periodic else (0.0, 0.0, 0.0))
+    oracle.lib()
+    cores = len(os.sched_getaffinity(0))
+    atoms, t0, reps = 0, time.perf_counter(), 0
+    if w.periodic:
+        raise SystemExit("cpu baseline sample for periodic workloads is not defined here")
+    dt = 0.0
+    while True:
+        r = reps % w.n_replicas
+        sl = slice(r * w.beads, (r + 1) * w.beads)
+        x = pos[sl].astype(np.float64)
+        _, _, F = oracle.energy_forces(om, x, types[sl])          # forces at the start (not timed)
+        t1 = time.perf_counter()
+        oracle.md_step(om, x, vel[sl].astype(np.float64), types[sl], mass[sl].astype(np.float64), F, w.dt_fs,
+                       w.gamma_per_ps, w.temperature, 1, reps)
+        dt += time.perf_counter() - t1
+        atoms += w.beads
+        reps += 1
+        if dt >= seconds:
+            break
+    return {"value": atoms / dt, "unit": "atom-steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} BAOAB steps, each of one whole {w.beads}-bead replica of this workload, "
+                      f"{dt:.1f} s timed"}
+
+
+def _edge_stats(model, pos, w):
+    """Listed and within-cutoff directed edges of the current list (host-side count)."""
+    rp, col, _ = model.neighbors()
+    rows = np.repeat(np.arange(w.n_atoms), np.diff(rp))
+    p = pos.astype(np.float64)
+    v = p[col] - p[rows]
+    if w.periodic:
+        v -= w.box * np.rint(v / w.box)
+    d = np.sqrt((v * v).sum(1))
+    return int(len(col)), int((d < w.cutoff).sum())
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+    from schnet_gnn_molecular_b200 import api
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    w = _workload(args.workload)
+    pos, types, weights, mass, vel = _inputs(w, rank)
+    n_rb = w.n_rebuild
+    steps = int(args.steps)
+    model = api.from_workload(w, weights, device=f"cuda:{local}", edge_capacity=args.edge_capacity)
+    dev = torch.device(f"cuda:{local}")
+    p = torch.tensor(pos, device=dev)
+    v = torch.tensor(vel, device=dev)
+    t = torch.tensor(types, device=dev)
+    m = torch.tensor(mass, device=dev)
+    kw = dict(dt=w.dt_fs, gamma=w.gamma_per_ps, temperature=w.temperature, n_rebuild=n_rb, seed=1234)
+    # warm-up: initial build + forces, graph capture, W steps
+    model.step(p, v, t, m, args.warmup, step0=0, **kw)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local) if rank == 0 else None
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    l0 = model.kernel_launches()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    model.step(p, v, t, m, steps, step0=args.warmup, resume=True, **kw)
+    ev1.record()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    launches = model.kernel_launches() - l0
+    clk = clocks.stop() if clocks else None
+    t_max = ms
+    if ws > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    atoms_total = w.n_atoms * ws
+    value = atoms_total * steps / (t_max * 1e-3)
+    step_s = t_max * 1e-3 / steps
+    ns_day_rep = (1.0 / step_s) * w.dt_fs * 86400 * 1e-6
+
+    out = None
+    if rank == 0:
+        # per-kernel device times on the library stream (eager profiling pass, same trajectory)
+        prof = model.profile_steps(p, v, t, m, n_rb, step0=args.warmup + steps, **kw)
+        E_list, E_cut = _edge_stats(model, p.cpu().numpy(), w)
+        peaks, src = _peaks()
+        flop_fwd = 2.0 * (w.K * w.F + w.F * w.F) * E_cut
+        flop_bwd = 2.0 * flop_fwd
+        fwd_ms = prof["cfconv_fwd"][0] / max(prof["cfconv_fwd"][1], 1)
+        bwd_ms = prof["cfconv_bwd"][0] / max(prof["cfconv_bwd"][1], 1)
+        tot_ms = sum(x[0] for x in prof.values())
+        dominant = "cfconv_bwd" if prof["cfconv_bwd"][0] >= prof["cfconv_fwd"][0] else "cfconv_fwd"
+        flops, kms = (flop_bwd, bwd_ms) if dominant == "cfconv_bwd" else (flop_fwd, fwd_ms)
+        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        achieved = flops / (kms * 1e-3) / 1e12
+        traffic = None
+        tf = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(tf):
+            try:
+                traffic = json.load(open(tf)).get(dominant)
+            except Exception:
+                traffic = None
+        roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 2),
+                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                    "peak_source": f"{src} dense bf16/fp16 sustained",
+                    "flop_per_launch": flops, "ms_per_launch": round(kms, 4),
+                    "per_kernel_ms_per_step": {k: round(x[0] / n_rb, 4) for k, x in prof.items()},
+                    "kernel_share": {k: round(x[0] / tot_ms, 4) for k, x in prof.items()}}
+        cfg = {"workload": w.name, "replicas": w.n_replicas, "beads_per_replica": w.beads, "atoms": w.n_atoms,
+               "F": w.F, "K": w.K, "L": w.L, "cutoff_A": w.cutoff, "skin_A": w.skin, "n_rebuild": n_rb,
+               "dt_fs": w.dt_fs, "integrator": "BAOAB" if w.gamma_per_ps > 0 else "velocity Verlet",
+               "weight_dtype": w.weight_dtype, "edges_listed": E_list, "edges_within_cutoff": E_cut,
+               "l2": "no flush: state carried step to step; per-step working set "
+                     f"{(E_list * 20 + w.n_atoms * 128 * 4 * (2 * w.L + 4)) / 1e6:.0f} MB > 126 MB L2",
+               "parallelism": f"replicas x{ws} ranks (independent)"}
+        out = {"metric": METRIC, "value": round(value, 1), "unit": "atom-steps/s", "n_gpus": ws, "steps": steps,
+               "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 4), "higher_is_better": True,
+               "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+               "mma": "fp16 hi/lo split operands, fp32 accumulate (tcgen05 kind::f16)", "data": "synthetic",
+               "ns_per_day_per_replica": round(ns_day_rep, 2),
+               "ns_per_day_aggregate": round(ns_day_rep * w.n_replicas * ws, 1),
+               "config": cfg, "gpu_launches": int(launches), "clocks": clk, "roofline": roofline}
+        if not args.no_e2e:
+            out["e2e"] = e2e(model, w, pos, vel, types, mass, kw, args)
+        if not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    model.close()
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+def e2e(model, w, pos, vel, types, mass, kw, args):
+    """Same metric through the host-buffer entry point: every step copies the step's inputs
+    from pinned host memory and reads the step's results back (schnet_step_host, one step per call)."""
+    import torch
+    hp = torch.from_numpy(pos.copy()).pin_memory().numpy()
+    hv = torch.from_numpy(vel.copy()).pin_memory().numpy()
+    ht = torch.from_numpy(types.copy()).pin_memory().numpy()
+    hm = torch.from_numpy(mass.copy()).pin_memory().numpy()
+    ep = torch.empty(w.n_replicas, dtype=torch.float64).pin_memory().numpy()
+    ek = torch.empty(w.n_replicas, dtype=torch.float64).pin_memory().numpy()
+    model.step_host(hp, hv, ht, hm, 0, step0=0, resume=False, epot=ep, ekin=ek, **kw)  # initial forces
+    n = max(w.n_rebuild, int(args.e2e_steps))
+    for s in range(3):
+        model.step_host(hp, hv, ht, hm, 1, step0=s, resume=True, epot=ep, ekin=ek, **kw)
+    t0 = time.perf_counter()
+    for s in range(n):
+        model.step_host(hp, hv, ht, hm, 1, step0=3 + s, resume=True, epot=ep, ekin=ek, **kw)
+    dt = time.perf_counter() - t0
+    h2d = hp.nbytes + hv.nbytes + ht.nbytes + hm.nbytes
+    d2h = hp.nbytes + hv.nbytes + ep.nbytes + ek.nbytes
+    return {"value": round(w.n_atoms * n / dt, 1), "unit": "atom-steps/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": n,
+            "how": "schnet_step_host, one step per call, pinned host buffers, wall clock"}
+
+
+def run_reference(args):
+    """The float64 oracle as the reference arm (rank 0 only).  One step = one BAOAB
+    step of a replica-shaped sample: a whole replica when the run fits the time
+    budget, else the first n beads of replica 0 (a contiguous chain segment)."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    w = _workload(args.workload)
+    import oracle
+    pos, types, weights, mass, vel = _inputs(w, 0)
+    om = oracle.Model(n_types=w.n_types, F=w.F, K=w.K, L=w.L, rbf_min=w.rbf_min, rbf_max=w.rbf_max,
+                      rbf_sigma=w.rbf_sigma, cutoff=w.cutoff, weights=weights)
+    oracle.lib()
+    cores = len(os.sched_getaffinity(0))
+
+    def sample(nb):
+        sl = slice(0, nb)
+        x = pos[sl].astype(np.float64); vv = vel[sl].astype(np.float64); ms = mass[sl].astype(np.float64)
+        _, _, F = oracle.energy_forces(om, x, types[sl])
+        return sl, x, vv, ms, F
+
+    # calibrate one whole-replica step (not counted), then size the per-step sample
+    sl, x, vv, ms, F = sample(w.beads)
+    t0 = time.perf_counter()
+    oracle.md_step(om, x, vv, types[sl], ms, F, w.dt_fs, w.gamma_per_ps, w.temperature, 1, 0)
+    t_unit = time.perf_counter() - t0
+    nb = w.beads
+    total = (args.steps + args.warmup) * t_unit
+    if total > args.ref_budget:
+        nb = max(16, int(w.beads * (args.ref_budget / total) ** 0.5))
+    sl, x, vv, ms, F = sample(nb)
+    for s in range(args.warmup):
+        x, vv, F, _, _ = oracle.md_step(om, x, vv, types[sl], ms, F, w.dt_fs, w.gamma_per_ps, w.temperature, 1, s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        x, vv, F, _, _ = oracle.md_step(om, x, vv, types[sl], ms, F, w.dt_fs, w.gamma_per_ps, w.temperature, 1,
+                                        args.warmup + s)
+    dt = time.perf_counter() - t0
+    value = nb * args.steps / dt
+    what = (f"replica 0 of {w.n_replicas} ({w.beads} beads)" if nb == w.beads else
+            f"first {nb} of the {w.beads} beads of replica 0 (chain segment; time budget)")
+    out = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "atom-steps/s", "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "sample": what},
+           "cpu_baseline": {"value": round(value, 2), "unit": "atom-steps/s", "cores": cores, "kind": "oracle",
+                            "sample": f"{args.steps} BAOAB steps of {what}"},
+           "e2e": {"value": round(value, 2), "unit": "atom-steps/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=40)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="cg_protein_64x269")
+    ap.add_argument("--edge-capacity", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=40)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=150.0, help="seconds for the reference arm's timed steps")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,247 @@
+// Device-side helpers shared by the SchNet B200 kernels: padded sizes, the
+// status word, activation functions, and thin inline-PTX wrappers for the
+// sm_100a tensor-core path (tcgen05 MMA with TMEM accumulators, mbarriers).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "../../include/schnet.h"
+
+namespace schnet {
+
+// Feature, Gaussian and readout widths are padded to these on the device.
+constexpr int FP = 128;   // features (tensor-core M)
+constexpr int KP = 64;    // Gaussians (GEMM1 K)
+constexpr int HP = 64;    // readout hidden width
+constexpr int TILE_E = 128;  // edges per tensor-core tile (GEMM N)
+
+// Accumulators and status shared by all kernels of one context.
+struct DevMeta {
+    long long n_edges;            // listed edges of the current neighbour list
+    unsigned int status;          // SCHNET_FLAG_* bits, sticky until read
+    unsigned int pad0;
+    unsigned long long step;      // MD step counter (noise stream)
+    long long timeout_where;      // diagnostic for bounded waits
+};
+
+__device__ __forceinline__ void set_flag(DevMeta* meta, unsigned int bit)
+{
+    atomicOr(&meta->status, bit);
+}
+
+// ---------------------------------------------------------------------------
+// activations: shifted softplus and its derivative (the logistic function)
+// ---------------------------------------------------------------------------
+constexpr float LN2F = 0.69314718055994530942f;
+
+__device__ __forceinline__ float ssp(float x)
+{
+    float t = __expf(-fabsf(x));
+    return fmaxf(x, 0.0f) + __logf(1.0f + t) - LN2F;
+}
+
+__device__ __forceinline__ float sigmoidf(float x)
+{
+    float t = __expf(-fabsf(x));
+    float r = __fdividef(1.0f, 1.0f + t);
+    return x >= 0.0f ? r : t * r;
+}
+
+// ssp(x) and ssp'(x) sharing one exponential
+__device__ __forceinline__ void ssp_and_grad(float x, float& s, float& g)
+{
+    float t = __expf(-fabsf(x));
+    float r = __fdividef(1.0f, 1.0f + t);
+    s = fmaxf(x, 0.0f) + __logf(1.0f + t) - LN2F;
+    g = x >= 0.0f ? r : t * r;
+}
+
+// ---------------------------------------------------------------------------
+// minimum image (single precision, used for distances in the filters)
+// ---------------------------------------------------------------------------
+struct Box {
+    float L[3];
+    float invL[3];
+    int periodic;
+};
+
+__device__ __forceinline__ float3 min_image(float3 v, const Box& b)
+{
+    if (b.periodic) {
+        v.x -= b.L[0] * rintf(v.x * b.invL[0]);
+        v.y -= b.L[1] * rintf(v.y * b.invL[1]);
+        v.z -= b.L[2] * rintf(v.z * b.invL[2]);
+    }
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory / mbarrier / tcgen05 wrappers (sm_100a)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after max_iter polls (each poll may itself suspend
+// for a hardware-defined slice), returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t max_iter)
+{
+    for (uint32_t it = 0; it < max_iter; ++it)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// TMEM allocation by one full warp; the base address lands in *dst (smem).
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (f16 or bf16 inputs, f32 accumulate)
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on an mbarrier once all previously issued tcgen05 ops of this thread complete.
+__device__ __forceinline__ void mma_commit(uint64_t* bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+// 32 lanes x 32 columns of 32-bit TMEM -> 32 registers per thread
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32])
+{
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]),
+          "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]), "=r"(u[20]), "=r"(u[21]),
+          "=r"(u[22]), "=r"(u[23]), "=r"(u[24]), "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]),
+          "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, no swizzle ("interleaved" core matrices of
+// 8 rows x 16 bytes stored as 128 contiguous bytes).  lbo: byte distance
+// between core matrices adjacent in K; sbo: adjacent in M/N.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+    // base offset 0, absolute LBO mode 0, layout type 0 (no swizzle)
+    return d;
+}
+
+// Instruction descriptor for kind::f16, dense, f32 accumulate.
+// ab_fmt: 0 = f16, 1 = bf16.  b_mn_major: 1 when B is stored MN-major.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_fmt, int b_mn_major)
+{
+    return (1u << 4)                          // D format f32
+           | ((uint32_t)ab_fmt << 7)          // A format
+           | ((uint32_t)ab_fmt << 10)         // B format
+           | (0u << 15)                       // A K-major
+           | ((uint32_t)b_mn_major << 16)     // B major
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// Byte offset of element (mn, k) of a 16-bit operand tile with MN rows,
+// no-swizzle core matrices, SBO = 128 B, LBO = MN * 16 B.
+__host__ __device__ constexpr uint32_t kmajor_off(int mn, int k, int MN)
+{
+    return (uint32_t)((k >> 3) * (MN * 16) + mn * 16 + (k & 7) * 2);
+}
+__host__ __device__ constexpr uint32_t mnmajor_off(int mn, int k, int MN)
+{
+    return (uint32_t)((k >> 3) * (MN * 16) + (mn >> 3) * 128 + (k & 7) * 16 + (mn & 7) * 2);
+}
+
+// 16-bit hi/lo split of an fp32 value (hi = RN(x), lo = RN(x - hi)).
+template <int FMT>
+struct Split;
+template <>
+struct Split<0> {
+    __device__ __forceinline__ static void run(float x, uint16_t& hi, uint16_t& lo)
+    {
+        __half h = __float2half_rn(x);
+        __half l = __float2half_rn(x - __half2float(h));
+        hi = __half_as_ushort(h);
+        lo = __half_as_ushort(l);
+    }
+};
+template <>
+struct Split<1> {
+    __device__ __forceinline__ static void run(float x, uint16_t& hi, uint16_t& lo)
+    {
+        __nv_bfloat16 h = __float2bfloat16_rn(x);
+        __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
+        hi = __bfloat16_as_ushort(h);
+        lo = __bfloat16_as_ushort(l);
+    }
+};
+
+}  // namespace schnet

@@ -1,0 +1,141 @@
+// Host-side context and launcher declarations shared by the library's .cu files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+#include <utility>
+#include <vector>
+#include <cuda_runtime.h>
+
+#include "../../include/schnet.h"
+#include "common.cuh"
+
+namespace schnet {
+
+constexpr int MAX_L = 8;
+constexpr int GMAX_NONPERIODIC = 8;   // max cells per dimension of one replica's grid
+constexpr int GMAX_PERIODIC = 256;
+constexpr int SCAN_BLOCK = 1024;      // threads per scan block
+constexpr int SCAN_ITEMS = 4;         // items per thread
+constexpr int SCAN_TILE = SCAN_BLOCK * SCAN_ITEMS;
+constexpr int REDUCE_CHUNK = 4096;    // atoms per partial sum of a per-replica reduction
+
+// Per-layer packed tensor-core operand images (bytes) for the filter network.
+constexpr size_t W1_IMG = (size_t)FP * KP * 2;   // one 16-bit term of W1^T (M=128 x K=64)
+constexpr size_t W2_IMG = (size_t)FP * FP * 2;   // one 16-bit term of W2^T (M=128 x K=128)
+constexpr size_t LAYER_IMG = 2 * W1_IMG + 2 * W2_IMG;  // hi + lo of both
+
+struct Workspace {
+    DevMeta* meta;
+    // packed weights
+    uint8_t* img;                 // [L][LAYER_IMG]
+    float *s1, *s2, *b1, *b2;     // [L][FP]
+    float *emb;                   // [T][FP]
+    float *Win, *Wo1, *Wo2;       // [L][FP][FP]  (row-major [in][out])
+    float *WinT, *Wo1T, *Wo2T;    // [L][FP][FP]  (transposed: [out][in])
+    float *bo1, *bo2;             // [L][FP]
+    float *R1, *R1T;              // [FP][HP], [HP][FP]
+    float *c1, *R2;               // [HP]
+    float *c2;                    // [1]
+    // atoms
+    int32_t* atom_rep;            // [N]
+    float4 *pos4, *ref4, *frc4;   // [N]
+    // neighbour list
+    int32_t *row_ptr, *rowcnt;    // [N+1]
+    int32_t *col, *coltmp, *rev, *erow;  // [cap]
+    float* s_edge;                // [cap]
+    int32_t* part;                // [ncta+1]
+    // cell list
+    int32_t *cell_of, *cell_atoms;       // [N]
+    int32_t *cell_cnt, *cell_start, *cell_fill;  // [ncell+1]
+    int32_t* rep_off;             // [R+1] replica offsets
+    int4* rgrid_dims;             // [R]   (gx, gy, gz, first cell)
+    float4* rgrid_org;            // [R]   grid origin
+    float4* rgrid_inv;            // [R]   inverse cell sizes
+    long long* scan_tmp;          // [SCAN_TILE] tile sums
+    // activations
+    float *x, *h, *q, *m, *g, *dh, *pr, *eps, *ke;
+    // reductions
+    double* partial;              // [nchunk]
+    int32_t *chunk_rep, *chunk_lo, *chunk_hi;  // [nchunk]
+    double *epot, *ekin;          // [R] scratch when caller passes NULL
+    // host-step staging
+    float *st_pos, *st_vel, *st_mass;  // [N*3], [N*3], [N]
+    int32_t* st_types;                 // [N]
+    double *st_epot, *st_ekin;         // [R]
+};
+
+struct GraphKey {
+    const void *pos, *vel, *types, *mass, *epot, *ekin, *noise;
+    float dt, gamma, temp;
+    int n_rebuild;
+    unsigned long long seed;
+    bool operator==(const GraphKey& o) const
+    {
+        return pos == o.pos && vel == o.vel && types == o.types && mass == o.mass && epot == o.epot &&
+               ekin == o.ekin && noise == o.noise && dt == o.dt && gamma == o.gamma && temp == o.temp &&
+               n_rebuild == o.n_rebuild && seed == o.seed;
+    }
+};
+
+}  // namespace schnet
+
+struct schnet_ctx {
+    schnet_config cfg;
+    std::vector<int32_t> rep_off;   // host copy [R+1]
+    int N, R, T, F, K, L, H;
+    int weight_fmt;                 // 0 fp16 operands, 1 bf16 operands
+    int n_wterms;                   // 2 (fp32 storage: hi+lo) or 1
+    int64_t cap;
+    int nsm, ncta;                  // SMs; CTAs of the tensor-core kernels
+    int ncell;                      // total cells reserved
+    int nchunk;                     // per-replica reduction chunks
+    int gdim[3];                    // periodic grid dims
+    double rl2;                     // (cutoff + skin)^2 in float64
+    float mu0, dmu;                 // Gaussian centres mu_k = mu0 + k dmu
+    schnet::Box box;
+    cudaStream_t user_stream;
+    cudaStream_t s;                 // internal stream
+    cudaEvent_t ev_in, ev_out;
+    schnet::Workspace ws;
+    bool have_list = false;
+    bool forces_valid = false;
+    // MD phase: steps taken since the last neighbour build
+    int since_build = 0;
+    // graph cache: 0 = build + n_rebuild steps, 1 = build + one step, 2 = one step
+    struct GraphSlot {
+        bool ok = false;
+        schnet::GraphKey key{};
+        cudaGraphExec_t exec = nullptr;
+        int64_t kernels = 0;
+    } graphs[3];
+    int64_t launches = 0;
+    // profiling (schnet_profile_steps): event pairs per kernel class
+    bool prof = false;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> prof_pairs[SCHNET_KERNEL_NCLASS];
+    std::string err;
+};
+
+namespace schnet {
+
+// launchers (each enqueues on ctx->s and counts its kernels in ctx->launches)
+cudaError_t launch_pack_positions(schnet_ctx* c, const float* d_pos);
+cudaError_t launch_build_neighbors(schnet_ctx* c);
+cudaError_t launch_energy_forces(schnet_ctx* c, const int32_t* d_types, double* d_energy, float* d_forces);
+cudaError_t launch_baoa(schnet_ctx* c, float* d_pos, float* d_vel, const float* d_mass, float dt, float gamma,
+                        float temp, unsigned long long seed, const float* d_noise, bool check_skin);
+cudaError_t launch_b_kick(schnet_ctx* c, float* d_vel, const float* d_mass, float dt, double* d_ekin);
+cudaError_t launch_set_step(schnet_ctx* c, unsigned long long step);
+cudaError_t launch_forces(schnet_ctx* c, float* d_forces);
+cudaError_t launch_replica_sum(schnet_ctx* c, const float* v, double* out);
+cudaError_t launch_aw_first(schnet_ctx* c, const int32_t* types);
+cudaError_t launch_aw_fwd(schnet_ctx* c, int layer);
+cudaError_t launch_aw_bwd_top(schnet_ctx* c);
+cudaError_t launch_aw_bwd(schnet_ctx* c, int layer);
+cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer);
+cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s);
+cudaError_t cfconv_init_attributes();
+cudaError_t atomwise_init_attributes();
+
+}  // namespace schnet

@@ -1,0 +1,461 @@
+// Neighbour build: cell list -> destination-sorted CSR with skin, its
+// transpose map rev[], and the per-CTA row partition of the tensor-core kernels.
+//
+// Follows "Ab Initio Accuracy Beyond the Cutoff" (Tessera), abstract: a
+// conservative neighbour skin (list radius r_c + skin) keeps the graph valid
+// between rebuilds; and FlashSchNet (paper-curation summary), How / flash
+// aggregation: a CSR layout that lets every reduction run per row without
+// atomics.  The pair test is done in float64 with every operation rounded on
+// its own, so the list is a bit-exact function of the float32 coordinates.
+#include "internal.h"
+
+namespace schnet {
+
+// ---------------------------------------------------------------------------
+// exclusive scan (int32 in, int32 out, int64 total) -- three passes
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ long long warp_incl_scan(long long v)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        long long t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+
+// block-wide exclusive scan of one value per thread; returns the block total
+__device__ __forceinline__ long long block_excl_scan(long long v, long long& excl)
+{
+    __shared__ long long wsum[32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    long long inc = warp_incl_scan(v);
+    if (lane == 31) wsum[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        const int nw = blockDim.x >> 5;
+        long long w = lane < nw ? wsum[lane] : 0;
+        long long wi = warp_incl_scan(w);
+        if (lane < nw) wsum[lane] = wi - w;
+        if (lane == nw - 1) wsum[31] = wi;   // total (nw <= 32)
+    }
+    __syncthreads();
+    excl = inc - v + wsum[wid];
+    long long total = wsum[31];
+    __syncthreads();
+    return total;
+}
+
+__global__ void k_scan_tiles(const int32_t* __restrict__ in, int n, long long* __restrict__ tile_sums)
+{
+    const int base = blockIdx.x * SCAN_TILE;
+    long long s = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) {
+        int i = base + threadIdx.x * SCAN_ITEMS + k;
+        if (i < n) s += in[i];
+    }
+    long long ex;
+    long long tot = block_excl_scan(s, ex);
+    if (threadIdx.x == 0) tile_sums[blockIdx.x] = tot;
+}
+
+__global__ void k_scan_sums(long long* __restrict__ tile_sums, int ntiles)
+{
+    // one block of SCAN_BLOCK threads, ntiles <= SCAN_TILE
+    long long v[SCAN_ITEMS];
+    long long s = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) {
+        int i = threadIdx.x * SCAN_ITEMS + k;
+        v[k] = i < ntiles ? tile_sums[i] : 0;
+        s += v[k];
+    }
+    long long ex;
+    block_excl_scan(s, ex);
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) {
+        int i = threadIdx.x * SCAN_ITEMS + k;
+        if (i < ntiles) tile_sums[i] = ex;
+        ex += v[k];
+    }
+}
+
+// out[i] = exclusive prefix, out[n] = total (clamped to int32); *total64 = total
+__global__ void k_scan_apply(const int32_t* __restrict__ in, int n, const long long* __restrict__ tile_sums,
+                             int32_t* __restrict__ out, long long* total64, int ntiles)
+{
+    const int base = blockIdx.x * SCAN_TILE;
+    long long v[SCAN_ITEMS];
+    long long s = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) {
+        int i = base + threadIdx.x * SCAN_ITEMS + k;
+        v[k] = i < n ? in[i] : 0;
+        s += v[k];
+    }
+    long long ex;
+    block_excl_scan(s, ex);
+    ex += tile_sums[blockIdx.x];
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) {
+        int i = base + threadIdx.x * SCAN_ITEMS + k;
+        if (i < n) out[i] = (int32_t)(ex < 0x7fffffffLL ? ex : 0x7fffffffLL);
+        ex += v[k];
+    }
+    if (blockIdx.x == ntiles - 1 && threadIdx.x == blockDim.x - 1) {
+        out[n] = (int32_t)(ex < 0x7fffffffLL ? ex : 0x7fffffffLL);
+        if (total64) *total64 = ex;
+    }
+}
+
+static cudaError_t scan_exclusive(schnet_ctx* c, const int32_t* in, int n, int32_t* out, long long* total64)
+{
+    int ntiles = (n + SCAN_TILE - 1) / SCAN_TILE;
+    if (ntiles < 1) ntiles = 1;
+    if (ntiles > SCAN_TILE) return cudaErrorInvalidValue;
+    k_scan_tiles<<<ntiles, SCAN_BLOCK, 0, c->s>>>(in, n, c->ws.scan_tmp);
+    k_scan_sums<<<1, SCAN_BLOCK, 0, c->s>>>(c->ws.scan_tmp, ntiles);
+    k_scan_apply<<<ntiles, SCAN_BLOCK, 0, c->s>>>(in, n, c->ws.scan_tmp, out, total64, ntiles);
+    c->launches += 3;
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// positions
+// ---------------------------------------------------------------------------
+__global__ void k_pack_positions(int n, const float* __restrict__ pos, float4* __restrict__ pos4,
+                                 const float4* __restrict__ ref4, int check_skin, float half_skin2,
+                                 DevMeta* meta)
+{
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float x = pos[3 * i], y = pos[3 * i + 1], z = pos[3 * i + 2];
+    pos4[i] = make_float4(x, y, z, 0.0f);
+    if (!(isfinite(x) && isfinite(y) && isfinite(z))) set_flag(meta, SCHNET_FLAG_NONFINITE);
+    if (check_skin) {
+        float4 r = ref4[i];
+        float dx = x - r.x, dy = y - r.y, dz = z - r.z;
+        if (dx * dx + dy * dy + dz * dz > half_skin2) set_flag(meta, SCHNET_FLAG_SKIN);
+    }
+}
+
+cudaError_t launch_pack_positions(schnet_ctx* c, const float* d_pos)
+{
+    float hs = 0.5f * c->cfg.skin;
+    k_pack_positions<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, d_pos, c->ws.pos4, c->ws.ref4,
+                                                            c->have_list ? 1 : 0, hs * hs, c->ws.meta);
+    c->launches += 1;
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// cell grid per replica
+// ---------------------------------------------------------------------------
+struct GridParams {
+    int periodic;
+    int gp[3];          // periodic grid dims
+    float rl;           // list radius
+    int gmax;           // non-periodic max dims
+    int cells_per_rep;  // stride between replicas' cell ranges
+};
+
+// one block per replica: bounding box (non-periodic) and grid dims
+__global__ void k_replica_grid(int R, const int32_t* __restrict__ rep_off, const float4* __restrict__ pos4,
+                               GridParams gp, const Box box, int4* __restrict__ dims, float4* __restrict__ org,
+                               float4* __restrict__ inv)
+{
+    int r = blockIdx.x;
+    if (r >= R) return;
+    int a = rep_off[r], b = rep_off[r + 1];
+    if (gp.periodic) {
+        if (threadIdx.x == 0) {
+            dims[r] = make_int4(gp.gp[0], gp.gp[1], gp.gp[2], r * gp.cells_per_rep);
+            org[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+            inv[r] = make_float4(gp.gp[0] * box.invL[0], gp.gp[1] * box.invL[1], gp.gp[2] * box.invL[2], 0.f);
+        }
+        return;
+    }
+    float lo[3] = {3.4e38f, 3.4e38f, 3.4e38f}, hi[3] = {-3.4e38f, -3.4e38f, -3.4e38f};
+    for (int i = a + threadIdx.x; i < b; i += blockDim.x) {
+        float4 p = pos4[i];
+        lo[0] = fminf(lo[0], p.x); lo[1] = fminf(lo[1], p.y); lo[2] = fminf(lo[2], p.z);
+        hi[0] = fmaxf(hi[0], p.x); hi[1] = fmaxf(hi[1], p.y); hi[2] = fmaxf(hi[2], p.z);
+    }
+    __shared__ float slo[3][32], shi[3][32];
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+        for (int o = 16; o > 0; o >>= 1) {
+            lo[d] = fminf(lo[d], __shfl_xor_sync(0xffffffffu, lo[d], o));
+            hi[d] = fmaxf(hi[d], __shfl_xor_sync(0xffffffffu, hi[d], o));
+        }
+    }
+    int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (lane == 0)
+        for (int d = 0; d < 3; ++d) { slo[d][wid] = lo[d]; shi[d][wid] = hi[d]; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int nw = blockDim.x >> 5;
+        int g[3];
+        float o3[3], iv[3];
+        for (int d = 0; d < 3; ++d) {
+            float l = 3.4e38f, h = -3.4e38f;
+            for (int w = 0; w < nw; ++w) { l = fminf(l, slo[d][w]); h = fmaxf(h, shi[d][w]); }
+            if (!(h >= l)) { l = 0.f; h = 0.f; }   // empty replica or non-finite
+            float ext = h - l;
+            int gd = (int)floorf(ext / gp.rl);
+            gd = gd < 1 ? 1 : (gd > gp.gmax ? gp.gmax : gd);
+            g[d] = gd;
+            o3[d] = l;
+            iv[d] = ext > 0.f ? (float)gd / ext : 0.f;
+        }
+        dims[r] = make_int4(g[0], g[1], g[2], r * gp.cells_per_rep);
+        org[r] = make_float4(o3[0], o3[1], o3[2], 0.f);
+        inv[r] = make_float4(iv[0], iv[1], iv[2], 0.f);
+    }
+}
+
+__device__ __forceinline__ int cell_coord(float x, float o, float iv, int g, int periodic)
+{
+    int c = (int)floorf((x - o) * iv);
+    if (periodic) {
+        c %= g;
+        if (c < 0) c += g;
+    }
+    return c < 0 ? 0 : (c >= g ? g - 1 : c);
+}
+
+__global__ void k_cell_assign(int n, const float4* __restrict__ pos4, const int32_t* __restrict__ atom_rep,
+                              const int4* __restrict__ dims, const float4* __restrict__ org,
+                              const float4* __restrict__ inv, int periodic, int32_t* __restrict__ cell_of,
+                              int32_t* __restrict__ cell_cnt)
+{
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    int r = atom_rep[i];
+    float4 p = pos4[i];
+    int4 g = dims[r];
+    float4 o = org[r], v = inv[r];
+    int cx = cell_coord(p.x, o.x, v.x, g.x, periodic);
+    int cy = cell_coord(p.y, o.y, v.y, g.y, periodic);
+    int cz = cell_coord(p.z, o.z, v.z, g.z, periodic);
+    int cell = g.w + cx + g.x * (cy + g.y * cz);
+    cell_of[i] = cell;
+    atomicAdd(&cell_cnt[cell], 1);
+}
+
+__global__ void k_cell_fill(int n, const int32_t* __restrict__ cell_of, const int32_t* __restrict__ cell_start,
+                            int32_t* __restrict__ cell_fill, int32_t* __restrict__ cell_atoms)
+{
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    int cell = cell_of[i];
+    int slot = atomicAdd(&cell_fill[cell], 1);
+    cell_atoms[cell_start[cell] + slot] = i;
+}
+
+// float64 pair test, each operation rounded separately (no contraction)
+__device__ __forceinline__ bool pair_in_list(float4 pi, float4 pj, double rl2, const Box& box)
+{
+    double dx = __dsub_rn((double)pj.x, (double)pi.x);
+    double dy = __dsub_rn((double)pj.y, (double)pi.y);
+    double dz = __dsub_rn((double)pj.z, (double)pi.z);
+    if (box.periodic) {
+        double Lx = (double)box.L[0], Ly = (double)box.L[1], Lz = (double)box.L[2];
+        dx = __dsub_rn(dx, __dmul_rn(Lx, rint(__ddiv_rn(dx, Lx))));
+        dy = __dsub_rn(dy, __dmul_rn(Ly, rint(__ddiv_rn(dy, Ly))));
+        dz = __dsub_rn(dz, __dmul_rn(Lz, rint(__ddiv_rn(dz, Lz))));
+    }
+    double d2 = __dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy));
+    d2 = __dadd_rn(d2, __dmul_rn(dz, dz));
+    return d2 < rl2;
+}
+
+// Visit every candidate j (cells around atom i's cell) passing the list test.
+template <class Fn>
+__device__ __forceinline__ void for_each_neighbor(int i, const float4* __restrict__ pos4,
+                                                  const int32_t* __restrict__ atom_rep,
+                                                  const int32_t* __restrict__ cell_of,
+                                                  const int4* __restrict__ dims,
+                                                  const int32_t* __restrict__ cell_start,
+                                                  const int32_t* __restrict__ cell_atoms, double rl2,
+                                                  const Box& box, Fn&& fn)
+{
+    int r = atom_rep[i];
+    int4 g = dims[r];
+    int local = cell_of[i] - g.w;
+    int cx = local % g.x, cy = (local / g.x) % g.y, cz = local / (g.x * g.y);
+    float4 pi = pos4[i];
+    // stencil offsets per dimension: periodic grids with < 3 cells visit each cell once
+    int lox = -1, hix = 1, loy = -1, hiy = 1, loz = -1, hiz = 1;
+    if (box.periodic) {
+        if (g.x < 3) { lox = 0; hix = g.x - 1; }
+        if (g.y < 3) { loy = 0; hiy = g.y - 1; }
+        if (g.z < 3) { loz = 0; hiz = g.z - 1; }
+    }
+    for (int oz = loz; oz <= hiz; ++oz) {
+        int z = cz + oz;
+        if (box.periodic) { if (g.z >= 3) z = (z + g.z) % g.z; }
+        else if (z < 0 || z >= g.z) continue;
+        for (int oy = loy; oy <= hiy; ++oy) {
+            int y = cy + oy;
+            if (box.periodic) { if (g.y >= 3) y = (y + g.y) % g.y; }
+            else if (y < 0 || y >= g.y) continue;
+            for (int ox = lox; ox <= hix; ++ox) {
+                int x = cx + ox;
+                if (box.periodic) { if (g.x >= 3) x = (x + g.x) % g.x; }
+                else if (x < 0 || x >= g.x) continue;
+                int cell = g.w + x + g.x * (y + g.y * z);
+                int a = cell_start[cell], b = cell_start[cell + 1];
+                for (int k = a; k < b; ++k) {
+                    int j = cell_atoms[k];
+                    if (j == i) continue;
+                    if (pair_in_list(pi, pos4[j], rl2, box)) fn(j);
+                }
+            }
+        }
+    }
+}
+
+__global__ void k_count(int n, const float4* __restrict__ pos4, const int32_t* __restrict__ atom_rep,
+                        const int32_t* __restrict__ cell_of, const int4* __restrict__ dims,
+                        const int32_t* __restrict__ cell_start, const int32_t* __restrict__ cell_atoms,
+                        double rl2, const Box box, int32_t* __restrict__ rowcnt)
+{
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    int cnt = 0;
+    for_each_neighbor(i, pos4, atom_rep, cell_of, dims, cell_start, cell_atoms, rl2, box, [&](int) { ++cnt; });
+    rowcnt[i] = cnt;
+}
+
+__global__ void k_fill(int n, const float4* __restrict__ pos4, const int32_t* __restrict__ atom_rep,
+                       const int32_t* __restrict__ cell_of, const int4* __restrict__ dims,
+                       const int32_t* __restrict__ cell_start, const int32_t* __restrict__ cell_atoms, double rl2,
+                       const Box box, const int32_t* __restrict__ row_ptr, long long cap, DevMeta* meta,
+                       int32_t* __restrict__ coltmp, int32_t* __restrict__ erow)
+{
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    if (meta->n_edges > cap) return;
+    int e = row_ptr[i];
+    for_each_neighbor(i, pos4, atom_rep, cell_of, dims, cell_start, cell_atoms, rl2, box, [&](int j) {
+        coltmp[e] = j;
+        erow[e] = i;
+        ++e;
+    });
+}
+
+// one warp per row: stable placement by rank (entries of a row are distinct)
+__global__ void k_sort_rows(int n, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ coltmp,
+                            long long cap, const DevMeta* meta, int32_t* __restrict__ col)
+{
+    if (meta->n_edges > cap) return;
+    int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int lane = threadIdx.x & 31;
+    int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int i = warp; i < n; i += nwarps) {
+        int a = row_ptr[i], b = row_ptr[i + 1];
+        for (int k = a + lane; k < b; k += 32) {
+            int v = coltmp[k];
+            int rank = 0;
+            for (int t = a; t < b; ++t) rank += coltmp[t] < v;
+            col[a + rank] = v;
+        }
+    }
+}
+
+// rev[e] = position of the reverse edge (binary search of i in row j)
+__global__ void k_rev(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
+                      const int32_t* __restrict__ erow, long long cap, const DevMeta* meta,
+                      int32_t* __restrict__ rev)
+{
+    long long E = meta->n_edges;
+    if (E > cap) return;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < E;
+         e += (long long)gridDim.x * blockDim.x) {
+        int i = erow[e], j = col[e];
+        int lo = row_ptr[j], hi = row_ptr[j + 1] - 1, found = -1;
+        while (lo <= hi) {
+            int mid = (lo + hi) >> 1;
+            int v = col[mid];
+            if (v == i) { found = mid; break; }
+            if (v < i) lo = mid + 1; else hi = mid - 1;
+        }
+        rev[e] = found;
+    }
+}
+
+// erow must describe the sorted list too: rows are unchanged by sorting
+// within a row, so the unsorted erow is already correct.
+
+// Row partition of the tensor-core kernels: CTA c takes whole rows holding
+// about one share of the edges (at least a few tiles).
+__global__ void k_partition(int n, int ncta, const int32_t* __restrict__ row_ptr, long long cap,
+                            const DevMeta* meta, int32_t* __restrict__ part)
+{
+    int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c > ncta) return;
+    long long E = meta->n_edges;
+    if (E > cap) E = 0;
+    long long share = (E + ncta - 1) / ncta;
+    if (share < 2 * TILE_E) share = 2 * TILE_E;
+    share = (share + TILE_E - 1) / TILE_E * TILE_E;
+    if (c == 0) { part[0] = 0; return; }
+    if (c == ncta) { part[c] = n; return; }
+    long long target = (long long)c * share;
+    if (target >= E) { part[c] = n; return; }
+    // first row whose start is >= target
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if ((long long)row_ptr[mid] < target) lo = mid + 1; else hi = mid;
+    }
+    part[c] = lo;
+}
+
+__global__ void k_check_capacity(long long cap, DevMeta* meta)
+{
+    if (meta->n_edges > cap) set_flag(meta, SCHNET_FLAG_CAPACITY);
+}
+
+cudaError_t launch_build_neighbors(schnet_ctx* c)
+{
+    Workspace& w = c->ws;
+    const int N = c->N, R = c->R;
+    GridParams gp;
+    gp.periodic = c->cfg.periodic;
+    gp.gp[0] = c->gdim[0]; gp.gp[1] = c->gdim[1]; gp.gp[2] = c->gdim[2];
+    gp.rl = c->cfg.cutoff + c->cfg.skin;
+    gp.gmax = GMAX_NONPERIODIC;
+    gp.cells_per_rep = c->ncell / R;
+    cudaError_t err;
+
+    k_replica_grid<<<R, 256, 0, c->s>>>(R, w.rep_off, w.pos4, gp, c->box, w.rgrid_dims, w.rgrid_org, w.rgrid_inv);
+    cudaMemsetAsync(w.cell_cnt, 0, sizeof(int32_t) * (c->ncell + 1), c->s);
+    cudaMemsetAsync(w.cell_fill, 0, sizeof(int32_t) * (c->ncell + 1), c->s);
+    int nb = (N + 255) / 256;
+    k_cell_assign<<<nb, 256, 0, c->s>>>(N, w.pos4, w.atom_rep, w.rgrid_dims, w.rgrid_org, w.rgrid_inv,
+                                        gp.periodic, w.cell_of, w.cell_cnt);
+    c->launches += 2;
+    if ((err = scan_exclusive(c, w.cell_cnt, c->ncell, w.cell_start, nullptr)) != cudaSuccess) return err;
+    k_cell_fill<<<nb, 256, 0, c->s>>>(N, w.cell_of, w.cell_start, w.cell_fill, w.cell_atoms);
+    const int nb128 = (N + 127) / 128;
+    k_count<<<nb128, 128, 0, c->s>>>(N, w.pos4, w.atom_rep, w.cell_of, w.rgrid_dims, w.cell_start, w.cell_atoms,
+                                  c->rl2, c->box, w.rowcnt);
+    c->launches += 2;
+    if ((err = scan_exclusive(c, w.rowcnt, N, w.row_ptr, &w.meta->n_edges)) != cudaSuccess) return err;
+    k_check_capacity<<<1, 1, 0, c->s>>>(c->cap, w.meta);
+    k_fill<<<nb128, 128, 0, c->s>>>(N, w.pos4, w.atom_rep, w.cell_of, w.rgrid_dims, w.cell_start, w.cell_atoms,
+                                 c->rl2, c->box, w.row_ptr, c->cap, w.meta, w.coltmp, w.erow);
+    int nsort = c->nsm * 8;
+    k_sort_rows<<<nsort, 256, 0, c->s>>>(N, w.row_ptr, w.coltmp, c->cap, w.meta, w.col);
+    k_rev<<<c->nsm * 8, 256, 0, c->s>>>(w.row_ptr, w.col, w.erow, c->cap, w.meta, w.rev);
+    k_partition<<<(c->ncta + 1 + 127) / 128, 128, 0, c->s>>>(N, c->ncta, w.row_ptr, c->cap, w.meta, w.part);
+    cudaMemcpyAsync(w.ref4, w.pos4, sizeof(float4) * N, cudaMemcpyDeviceToDevice, c->s);
+    c->launches += 5;
+    return cudaGetLastError();
+}
+
+}  // namespace schnet

@@ -1,0 +1,183 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on the
+same seeded inputs.  Tolerances: neighbour lists bit-exact; energies relative
+1e-5 per replica; forces relative Frobenius 1e-4 (16-bit filter weights: 2e-3
+against the fp32 oracle, 1e-4 against the oracle on the dequantized weights)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from _helpers import (ENERGY_RTOL, FORCE_RTOL, FORCE_RTOL_16BIT, FORCE_RTOL_DEQUANT, energy_rel, oracle_model,
+                      rel_frobenius)
+from schnet_gnn_molecular_b200 import api, inputs, workloads
+
+pytestmark = pytest.mark.gpu
+
+SMALL_PROTEIN = workloads.PROTEIN64.with_(name="cg_protein_6x269", n_replicas=6, seed=1000)
+PERIODIC_SMALL = workloads.BOX1M.with_(name="periodic_box_3000", beads=3000, box=(3000 / 0.01) ** (1 / 3),
+                                       seed=4000)
+
+
+def _dev(a, dtype=None):
+    return torch.as_tensor(np.ascontiguousarray(a), dtype=dtype).cuda()
+
+
+def _setup(w, bias_scale=0.0, weight_dtype=None, seed_offset=0):
+    pos = workloads.positions(w)
+    types = workloads.types(w)
+    weights = workloads.weights(w, bias_scale=bias_scale, seed_offset=seed_offset)
+    model = api.from_workload(w, weights, weight_dtype=weight_dtype)
+    return pos, types, weights, model
+
+
+def _gpu_eval(model, pos, types):
+    p = _dev(pos, torch.float32)
+    t = _dev(types, torch.int32)
+    model.build_neighbors(p)
+    E, F = model.energy_forces(p, t)
+    torch.cuda.synchronize()
+    assert model.status() == 0
+    return E.cpu().numpy(), F.cpu().numpy()
+
+
+# ---------------------------------------------------------------------------
+# neighbour lists: bit-exact against the brute-force float64 definition
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [workloads.TINY, SMALL_PROTEIN, PERIODIC_SMALL], ids=lambda w: w.name)
+def test_neighbor_list_bit_exact(w):
+    pos, types, weights, model = _setup(w)
+    model.build_neighbors(_dev(pos, torch.float32))
+    rp, col, rev = model.neighbors()
+    rp_o, col_o = oracle.neighbors(pos, w.cutoff, w.skin, w.replica_offsets(), w.periodic, (w.box,) * 3)
+    assert np.array_equal(rp, rp_o)
+    assert np.array_equal(col, col_o)
+    rows = np.repeat(np.arange(w.n_atoms), np.diff(rp))
+    assert np.all(rev >= 0)
+    assert np.array_equal(col[rev], rows) and np.array_equal(rows[rev], col)
+    assert np.array_equal(rev[rev], np.arange(len(col)))
+
+
+# ---------------------------------------------------------------------------
+# energies and forces
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("bias_scale", [0.0, 0.2])
+def test_energy_forces_tiny_chain(bias_scale):
+    w = workloads.TINY
+    pos, types, weights, model = _setup(w, bias_scale=bias_scale)
+    E, F = _gpu_eval(model, pos, types)
+    Eo, eps_o, Fo = oracle.energy_forces(oracle_model(w, weights), pos.astype(np.float64), types)
+    assert energy_rel(E, Eo, eps_o) <= ENERGY_RTOL, (E, Eo)
+    assert rel_frobenius(F, Fo) <= FORCE_RTOL
+    eps = model.atom_energies().cpu().numpy()
+    assert np.max(np.abs(eps - eps_o)) <= 1e-5 * np.max(np.abs(eps_o))
+
+
+def test_energy_forces_multi_replica():
+    w = SMALL_PROTEIN
+    pos, types, weights, model = _setup(w, bias_scale=0.1)
+    E, F = _gpu_eval(model, pos, types)
+    ro = w.replica_offsets()
+    Eo, eps_o, Fo = oracle.energy_forces(oracle_model(w, weights), pos.astype(np.float64), types, ro)
+    assert energy_rel(E, Eo, eps_o, ro) <= ENERGY_RTOL
+    assert rel_frobenius(F, Fo) <= FORCE_RTOL
+    # no net force inside any (isolated) replica
+    for r in range(w.n_replicas):
+        Fr = F[r * w.beads:(r + 1) * w.beads]
+        assert np.abs(Fr.sum(0)).max() <= 1e-4 * np.abs(Fr).max() * np.sqrt(w.beads)
+
+
+def test_energy_forces_periodic():
+    w = PERIODIC_SMALL
+    pos, types, weights, model = _setup(w)
+    E, F = _gpu_eval(model, pos, types)
+    Eo, eps_o, Fo = oracle.energy_forces(oracle_model(w, weights), pos.astype(np.float64), types)
+    assert energy_rel(E, Eo, eps_o) <= ENERGY_RTOL
+    assert rel_frobenius(F, Fo) <= FORCE_RTOL
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_sixteen_bit_filter_weights(dtype):
+    w = SMALL_PROTEIN.with_(weight_dtype=dtype)
+    pos, types, weights, model = _setup(w)
+    E, F = _gpu_eval(model, pos, types)
+    x64 = pos.astype(np.float64)
+    ro = w.replica_offsets()
+    Eq, eps_q, Fq = oracle.energy_forces(oracle_model(w, weights, dequant=dtype), x64, types, ro)
+    assert energy_rel(E, Eq, eps_q, ro) <= ENERGY_RTOL
+    assert rel_frobenius(F, Fq) <= FORCE_RTOL_DEQUANT
+    E32, _, F32 = oracle.energy_forces(oracle_model(w, weights), x64, types, w.replica_offsets())
+    assert rel_frobenius(F, F32) <= FORCE_RTOL_16BIT
+
+
+def test_isolated_atoms_and_empty_rows():
+    # three replicas: a lone bead, two far-apart beads, and a short chain
+    w = workloads.TINY.with_(n_replicas=3, beads=1)
+    rng = np.random.default_rng(5)
+    chain = inputs.chain(10, rng)
+    pos = np.concatenate([[[0.0, 0, 0]], [[0.0, 0, 0], [50.0, 0, 0]], chain]).astype(np.float32)
+    ro = [0, 1, 3, 13]
+    types = inputs.bead_types(13, w.n_types, rng)
+    weights = workloads.weights(workloads.TINY, bias_scale=0.3)
+    model = api.SchNet(n_types=w.n_types, F=w.F, K=w.K, L=w.L, rbf_min=w.rbf_min, rbf_max=w.rbf_max,
+                       rbf_sigma=w.rbf_sigma, cutoff=w.cutoff, skin=w.skin, replica_offsets=ro, weights=weights)
+    E, F = _gpu_eval(model, pos, types)
+    m = oracle_model(workloads.TINY, weights)
+    Eo, eps_o, Fo = oracle.energy_forces(m, pos.astype(np.float64), types, ro)
+    assert energy_rel(E, Eo, eps_o, ro) <= ENERGY_RTOL
+    assert np.all(F[:3] == 0.0)
+    assert rel_frobenius(F, Fo) <= FORCE_RTOL
+
+
+# ---------------------------------------------------------------------------
+# integrator
+# ---------------------------------------------------------------------------
+def test_one_langevin_step_matches_oracle():
+    w = workloads.TINY
+    pos, types, weights, model = _setup(w)
+    mass = workloads.masses(w)
+    vel = (workloads.velocity_normals(w) * np.sqrt(0.0019872041 * 300 * 4.184e-4 / 12.0)).astype(np.float32)
+    p, v = _dev(pos, torch.float32), _dev(vel, torch.float32)
+    epot, ekin, st = model.step(p, v, _dev(types, torch.int32), _dev(mass, torch.float32), 1, dt=w.dt_fs,
+                                gamma=w.gamma_per_ps, temperature=w.temperature, n_rebuild=w.n_rebuild, seed=77,
+                                step0=5)
+    torch.cuda.synchronize()
+    m = oracle_model(w, weights)
+    x64 = pos.astype(np.float64)
+    _, _, F0 = oracle.energy_forces(m, x64, types)
+    po, vo, Fo, epo, eko = oracle.md_step(m, x64, vel.astype(np.float64), types, mass.astype(np.float64), F0,
+                                          w.dt_fs, w.gamma_per_ps, w.temperature, 77, 5)
+    assert np.max(np.abs(p.cpu().numpy() - po)) < 1e-4
+    assert rel_frobenius(v.cpu().numpy(), vo) < 1e-4
+    assert energy_rel(epot.cpu().numpy(), epo) <= ENERGY_RTOL
+    assert abs(ekin.cpu().numpy()[0] / eko[0] - 1) < 1e-4
+
+
+def test_graph_replay_equals_eager():
+    w = SMALL_PROTEIN
+    pos, types, weights, model = _setup(w)
+    mass = _dev(workloads.masses(w), torch.float32)
+    vel0 = (workloads.velocity_normals(w) * 0.005).astype(np.float32)
+    t = _dev(types, torch.int32)
+    outs = []
+    for use_graph in (False, True):
+        p, v = _dev(pos, torch.float32), _dev(vel0, torch.float32)
+        ep, ek, st = model.step(p, v, t, mass, 40, n_rebuild=10, seed=3, use_graph=use_graph)
+        outs.append((p.cpu().numpy(), v.cpu().numpy(), ep.cpu().numpy()))
+    assert np.array_equal(outs[0][0], outs[1][0])
+    assert np.array_equal(outs[0][1], outs[1][1])
+    assert np.array_equal(outs[0][2], outs[1][2])
+
+
+# ---------------------------------------------------------------------------
+# full-size workload, sampled: 64 x 269 replicas on the GPU, whole replicas in the oracle
+# ---------------------------------------------------------------------------
+def test_protein64_sampled_replicas():
+    w = workloads.PROTEIN64
+    pos, types, weights, model = _setup(w)
+    E, F = _gpu_eval(model, pos, types)
+    m = oracle_model(w, weights)
+    for r in (0, 37, 63):
+        sl = slice(r * w.beads, (r + 1) * w.beads)
+        Eo, eps_o, Fo = oracle.energy_forces(m, pos[sl].astype(np.float64), types[sl])
+        assert energy_rel(E[r:r + 1], Eo, eps_o) <= ENERGY_RTOL
+        assert rel_frobenius(F[sl], Fo) <= FORCE_RTOL

@@ -158,6 +158,11 @@ def _edge_stats(model, pos, w):
     return int(len(col)), int((d < w.cutoff).sum())
 
 
+def nat_status(st):
+    from schnet_gnn_molecular_b200 import _native
+    return _native.STATUS_NAMES.get(int(st), str(st))
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -179,7 +184,9 @@ def run_native(args):
     m = torch.tensor(mass, device=dev)
     kw = dict(dt=w.dt_fs, gamma=w.gamma_per_ps, temperature=w.temperature, n_rebuild=n_rb, seed=1234)
     # warm-up: initial build + forces, graph capture, W steps
-    model.step(p, v, t, m, args.warmup, step0=0, **kw)
+    flagged = []
+    _, _, st = model.step(p, v, t, m, args.warmup, step0=0, raise_on_flag=False, **kw)
+    flagged.append(st)
     torch.cuda.synchronize()
 
     clocks = ClockSampler(local) if rank == 0 else None
@@ -189,8 +196,9 @@ def run_native(args):
     l0 = model.kernel_launches()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
-    model.step(p, v, t, m, steps, step0=args.warmup, resume=True, **kw)
+    _, _, st = model.step(p, v, t, m, steps, step0=args.warmup, resume=True, raise_on_flag=False, **kw)
     ev1.record()
+    flagged.append(st)
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
@@ -248,7 +256,8 @@ def run_native(args):
                "mma": "fp16 hi/lo split operands, fp32 accumulate (tcgen05 kind::f16)", "data": "synthetic",
                "ns_per_day_per_replica": round(ns_day_rep, 2),
                "ns_per_day_aggregate": round(ns_day_rep * w.n_replicas * ws, 1),
-               "config": cfg, "gpu_launches": int(launches), "clocks": clk, "roofline": roofline}
+               "config": cfg, "gpu_launches": int(launches), "clocks": clk, "roofline": roofline,
+               "status": {"warmup": nat_status(flagged[0]), "timed": nat_status(flagged[1])}}
         if not args.no_e2e:
             out["e2e"] = e2e(model, w, pos, vel, types, mass, kw, args)
         if not args.no_cpu_baseline:

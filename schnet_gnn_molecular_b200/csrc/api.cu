@@ -423,6 +423,7 @@ schnet_status step_impl(schnet_ctx* c, float* pos, float* vel, const int32_t* ty
     double* ep = epot ? epot : c->ws.epot;
     double* ek = ekin ? ekin : c->ws.ekin;
     if (!p->resume || !c->forces_valid) {
+        c->have_list = false;            // fresh start: the build below replaces the list (no skin check)
         CK(launch_pack_positions(c, pos));
         CK(launch_build_neighbors(c));
         c->have_list = true;

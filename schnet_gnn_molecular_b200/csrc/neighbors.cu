@@ -29,6 +29,7 @@ __device__ __forceinline__ long long warp_incl_scan(long long v)
 __device__ __forceinline__ long long block_excl_scan(long long v, long long& excl)
 {
     __shared__ long long wsum[32];
+    __shared__ long long wtotal;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     long long inc = warp_incl_scan(v);
     if (lane == 31) wsum[wid] = inc;
@@ -37,12 +38,12 @@ __device__ __forceinline__ long long block_excl_scan(long long v, long long& exc
         const int nw = blockDim.x >> 5;
         long long w = lane < nw ? wsum[lane] : 0;
         long long wi = warp_incl_scan(w);
-        if (lane < nw) wsum[lane] = wi - w;
-        if (lane == nw - 1) wsum[31] = wi;   // total (nw <= 32)
+        if (lane < nw) wsum[lane] = wi - w;   // exclusive prefix of each warp
+        if (lane == nw - 1) wtotal = wi;      // block total
     }
     __syncthreads();
     excl = inc - v + wsum[wid];
-    long long total = wsum[31];
+    long long total = wtotal;
     __syncthreads();
     return total;
 }

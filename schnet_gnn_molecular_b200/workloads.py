@@ -45,7 +45,7 @@ class Workload:
     seed: int = 0
     radius: float | None = None  # confinement radius for compact chains
     rg_target: float = 12.0
-    mass: float = 12.0
+    mass: float = 72.0         # amu per bead (MARTINI-style bead, see the mass reading)
 
     @property
     def n_atoms(self) -> int:

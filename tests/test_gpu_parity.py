@@ -16,6 +16,8 @@ pytestmark = pytest.mark.gpu
 SMALL_PROTEIN = workloads.PROTEIN64.with_(name="cg_protein_6x269", n_replicas=6, seed=1000)
 PERIODIC_SMALL = workloads.BOX1M.with_(name="periodic_box_3000", beads=3000, box=(3000 / 0.01) ** (1 / 3),
                                        seed=4000)
+PERIODIC_20K = workloads.BOX1M.with_(name="periodic_box_20000", beads=20000, box=(20000 / 0.01) ** (1 / 3),
+                                     seed=4000)
 
 
 def _dev(a, dtype=None):
@@ -43,7 +45,8 @@ def _gpu_eval(model, pos, types):
 # ---------------------------------------------------------------------------
 # neighbour lists: bit-exact against the brute-force float64 definition
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("w", [workloads.TINY, SMALL_PROTEIN, PERIODIC_SMALL], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", [workloads.TINY, SMALL_PROTEIN, PERIODIC_SMALL, workloads.PROTEIN64, PERIODIC_20K],
+                         ids=lambda w: w.name)
 def test_neighbor_list_bit_exact(w):
     pos, types, weights, model = _setup(w)
     model.build_neighbors(_dev(pos, torch.float32))
@@ -135,7 +138,7 @@ def test_one_langevin_step_matches_oracle():
     w = workloads.TINY
     pos, types, weights, model = _setup(w)
     mass = workloads.masses(w)
-    vel = (workloads.velocity_normals(w) * np.sqrt(0.0019872041 * 300 * 4.184e-4 / 12.0)).astype(np.float32)
+    vel = (workloads.velocity_normals(w) * np.sqrt(0.0019872041 * 300 * 4.184e-4 / w.mass)).astype(np.float32)
     p, v = _dev(pos, torch.float32), _dev(vel, torch.float32)
     epot, ekin, st = model.step(p, v, _dev(types, torch.int32), _dev(mass, torch.float32), 1, dt=w.dt_fs,
                                 gamma=w.gamma_per_ps, temperature=w.temperature, n_rebuild=w.n_rebuild, seed=77,

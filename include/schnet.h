@@ -229,6 +229,35 @@ SCHNET_API schnet_status schnet_profile_steps(schnet_ctx *ctx, float *d_pos, flo
                                               const float *d_mass, int64_t n_steps, const schnet_step_params *p,
                                               double *ms_total, int64_t *launches);
 
+/* Neighbour list without any device allocation and without a context.
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device memory where they call the library (a host
+ * program that only hands over buffers it already owns, or a runtime that
+ * forbids cudaMalloc while it runs).  It builds the same list as
+ * schnet_build_neighbors (same pair test, rows sorted, rev = transpose map),
+ * with all scratch in one fixed array of about 3.6 MB that every device
+ * loading this library keeps until the process exits.
+ *   d_pos: device float32 [n_atoms][3]; d_replica_offsets: device int32
+ *   [n_replicas+1] (0 .. n_atoms, non-decreasing); box: host float[3]
+ *   (periodic only).  Outputs (caller-owned device buffers): d_row_ptr int32
+ *   [n_atoms+1], d_col and d_rev int32 [edge_capacity], d_n_edges int64 [1]
+ *   = edges found; if that exceeds edge_capacity, col and rev are left
+ *   unspecified and the caller should retry with more room.
+ * Limits: n_atoms <= 65536, n_replicas <= 1024, cells <= 131072 (open
+ * boundaries use 512 cells per replica, so n_replicas <= 256 there),
+ * edge_capacity < 2^31; larger inputs return SCHNET_ERR_UNSUPPORTED, bad
+ * pointers or sizes SCHNET_ERR_INVALID_ARG.  Asynchronous on cuda_stream.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call reuses the same array and zeroes what must start at zero, so
+ * calls that overlap on the GPU (other streams or other host threads)
+ * race and must be serialized by the caller.  No call allocates memory. */
+SCHNET_API schnet_status schnet_build_neighbors_noalloc(const float *d_pos, int32_t n_atoms, int32_t n_replicas,
+                                                        const int32_t *d_replica_offsets, float cutoff, float skin,
+                                                        int32_t periodic, const float *box, int32_t *d_row_ptr,
+                                                        int32_t *d_col, int32_t *d_rev, int64_t edge_capacity,
+                                                        int64_t *d_n_edges, void *cuda_stream);
+
 /* Number of device kernels the library has launched on this context so far
  * (graph replays count each kernel node). */
 SCHNET_API int64_t schnet_kernel_launches(const schnet_ctx *ctx);

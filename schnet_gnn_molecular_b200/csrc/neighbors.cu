@@ -7,6 +7,9 @@
 // aggregation: a CSR layout that lets every reduction run per row without
 // atomics.  The pair test is done in float64 with every operation rounded on
 // its own, so the list is a bit-exact function of the float32 coordinates.
+#include <cmath>
+#include <mutex>
+
 #include "internal.h"
 
 namespace schnet {
@@ -460,3 +463,191 @@ cudaError_t launch_build_neighbors(schnet_ctx* c)
 }
 
 }  // namespace schnet
+
+// ===========================================================================
+// Allocation-free neighbour build (schnet_build_neighbors_noalloc)
+//
+// For callers that cannot allocate device memory at the point of the call --
+// for example a host application that hands this library only the buffers it
+// already owns, or a runtime that forbids allocation while it is running --
+// the build's scratch (packed positions, cell grid, cell counts and starts,
+// row counts, scan partial sums, status) lives in one fixed-size device array
+// defined in this file.  Every device that loads the library keeps that array
+// until the process exits.  The caller supplies positions and the output
+// buffers; the row-sorted columns are staged in the caller's `rev` buffer
+// before the transpose map overwrites it, so no per-edge scratch is needed.
+// ===========================================================================
+namespace schnet {
+
+constexpr int NA_MAX_ATOMS = 65536;
+constexpr int NA_MAX_REPLICAS = 1024;
+constexpr int NA_MAX_CELLS = 131072;
+
+// carve offsets (bytes) inside the static array
+constexpr size_t na_align(size_t x) { return (x + 255) / 256 * 256; }
+constexpr size_t NA_OFF_META = 0;
+constexpr size_t NA_OFF_POS4 = na_align(NA_OFF_META + sizeof(DevMeta));
+constexpr size_t NA_OFF_AREP = na_align(NA_OFF_POS4 + sizeof(float4) * NA_MAX_ATOMS);
+constexpr size_t NA_OFF_CELLOF = na_align(NA_OFF_AREP + sizeof(int32_t) * NA_MAX_ATOMS);
+constexpr size_t NA_OFF_CATOMS = na_align(NA_OFF_CELLOF + sizeof(int32_t) * NA_MAX_ATOMS);
+constexpr size_t NA_OFF_ROWCNT = na_align(NA_OFF_CATOMS + sizeof(int32_t) * NA_MAX_ATOMS);
+constexpr size_t NA_OFF_CCNT = na_align(NA_OFF_ROWCNT + sizeof(int32_t) * (NA_MAX_ATOMS + 1));
+constexpr size_t NA_OFF_CSTART = na_align(NA_OFF_CCNT + sizeof(int32_t) * (NA_MAX_CELLS + 1));
+constexpr size_t NA_OFF_CFILL = na_align(NA_OFF_CSTART + sizeof(int32_t) * (NA_MAX_CELLS + 1));
+constexpr size_t NA_OFF_DIMS = na_align(NA_OFF_CFILL + sizeof(int32_t) * (NA_MAX_CELLS + 1));
+constexpr size_t NA_OFF_ORG = na_align(NA_OFF_DIMS + sizeof(int4) * NA_MAX_REPLICAS);
+constexpr size_t NA_OFF_INV = na_align(NA_OFF_ORG + sizeof(float4) * NA_MAX_REPLICAS);
+constexpr size_t NA_OFF_SCAN = na_align(NA_OFF_INV + sizeof(float4) * NA_MAX_REPLICAS);
+constexpr size_t NA_BYTES = na_align(NA_OFF_SCAN + sizeof(long long) * SCAN_TILE);   // about 3.6 MB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NA_BYTES];
+
+// Per-device address of g_noalloc_scratch, looked up once with the device current.
+static void* g_noalloc_ptr[64] = {};
+static std::mutex g_noalloc_mu;
+
+static cudaError_t noalloc_scratch(void** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+// atom -> replica map from the offsets (binary search)
+__global__ void k_atom_replica(int n, int R, const int32_t* __restrict__ rep_off, int32_t* __restrict__ atom_rep)
+{
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    int lo = 0, hi = R - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (rep_off[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    atom_rep[i] = lo;
+}
+
+// rev[e] by a warp per row (the row of an edge is known from the loop)
+__global__ void k_rev_rows(int n, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
+                           long long cap, const DevMeta* meta, int32_t* __restrict__ rev)
+{
+    if (meta->n_edges > cap) return;
+    int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int lane = threadIdx.x & 31;
+    int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int i = warp; i < n; i += nwarps) {
+        for (int e = row_ptr[i] + lane; e < row_ptr[i + 1]; e += 32) {
+            int j = col[e];
+            int lo = row_ptr[j], hi = row_ptr[j + 1] - 1, found = -1;
+            while (lo <= hi) {
+                int mid = (lo + hi) >> 1;
+                int v = col[mid];
+                if (v == i) { found = mid; break; }
+                if (v < i) lo = mid + 1; else hi = mid - 1;
+            }
+            rev[e] = found;
+        }
+    }
+}
+
+__global__ void k_copy_edge_count(const DevMeta* meta, int64_t* out) { *out = meta->n_edges; }
+
+static cudaError_t scan_exclusive_raw(cudaStream_t s, const int32_t* in, int n, int32_t* out, long long* total64,
+                                      long long* tmp)
+{
+    int ntiles = (n + SCAN_TILE - 1) / SCAN_TILE;
+    if (ntiles < 1) ntiles = 1;
+    if (ntiles > SCAN_TILE) return cudaErrorInvalidValue;
+    k_scan_tiles<<<ntiles, SCAN_BLOCK, 0, s>>>(in, n, tmp);
+    k_scan_sums<<<1, SCAN_BLOCK, 0, s>>>(tmp, ntiles);
+    k_scan_apply<<<ntiles, SCAN_BLOCK, 0, s>>>(in, n, tmp, out, total64, ntiles);
+    return cudaGetLastError();
+}
+
+}  // namespace schnet
+
+extern "C" schnet_status schnet_build_neighbors_noalloc(const float* d_pos, int32_t n_atoms, int32_t n_replicas,
+                                                        const int32_t* d_replica_offsets, float cutoff, float skin,
+                                                        int32_t periodic, const float* box, int32_t* d_row_ptr,
+                                                        int32_t* d_col, int32_t* d_rev, int64_t edge_capacity,
+                                                        int64_t* d_n_edges, void* cuda_stream)
+{
+    using namespace schnet;
+    if (!d_pos || !d_replica_offsets || !d_row_ptr || !d_col || !d_rev || !d_n_edges || n_atoms < 1 ||
+        n_replicas < 1 || edge_capacity < 1 || !(cutoff > 0.f) || !(skin >= 0.f) || (periodic && !box))
+        return SCHNET_ERR_INVALID_ARG;
+    const double rl = (double)cutoff + (double)skin;
+    int gdim[3] = {GMAX_NONPERIODIC, GMAX_NONPERIODIC, GMAX_NONPERIODIC};
+    Box bx;
+    bx.periodic = periodic ? 1 : 0;
+    for (int d = 0; d < 3; ++d) {
+        bx.L[d] = periodic ? box[d] : 0.f;
+        bx.invL[d] = periodic ? 1.0f / box[d] : 0.f;
+        if (periodic) {
+            if (!(box[d] >= 2.0f * (cutoff + skin))) return SCHNET_ERR_UNSUPPORTED;
+            int g = (int)std::floor((double)box[d] / rl);
+            gdim[d] = g < 1 ? 1 : (g > GMAX_PERIODIC ? GMAX_PERIODIC : g);
+        }
+    }
+    const long long cells_per_rep = (long long)gdim[0] * gdim[1] * gdim[2];
+    const long long ncell = cells_per_rep * n_replicas;
+    if (n_atoms > NA_MAX_ATOMS || n_replicas > NA_MAX_REPLICAS || ncell > NA_MAX_CELLS ||
+        edge_capacity > 0x7fffffffLL)
+        return SCHNET_ERR_UNSUPPORTED;
+
+    uint8_t* base = nullptr;
+    if (noalloc_scratch(reinterpret_cast<void**>(&base)) != cudaSuccess) return SCHNET_ERR_CUDA;
+    DevMeta* meta = reinterpret_cast<DevMeta*>(base + NA_OFF_META);
+    float4* pos4 = reinterpret_cast<float4*>(base + NA_OFF_POS4);
+    int32_t* arep = reinterpret_cast<int32_t*>(base + NA_OFF_AREP);
+    int32_t* cell_of = reinterpret_cast<int32_t*>(base + NA_OFF_CELLOF);
+    int32_t* catoms = reinterpret_cast<int32_t*>(base + NA_OFF_CATOMS);
+    int32_t* rowcnt = reinterpret_cast<int32_t*>(base + NA_OFF_ROWCNT);
+    int32_t* ccnt = reinterpret_cast<int32_t*>(base + NA_OFF_CCNT);
+    int32_t* cstart = reinterpret_cast<int32_t*>(base + NA_OFF_CSTART);
+    int32_t* cfill = reinterpret_cast<int32_t*>(base + NA_OFF_CFILL);
+    int4* dims = reinterpret_cast<int4*>(base + NA_OFF_DIMS);
+    float4* org = reinterpret_cast<float4*>(base + NA_OFF_ORG);
+    float4* inv = reinterpret_cast<float4*>(base + NA_OFF_INV);
+    long long* scan_tmp = reinterpret_cast<long long*>(base + NA_OFF_SCAN);
+
+    cudaStream_t s = (cudaStream_t)cuda_stream;
+    const int N = n_atoms, R = n_replicas;
+    const int nb = (N + 255) / 256, nb128 = (N + 127) / 128;
+    GridParams gp;
+    gp.periodic = bx.periodic;
+    gp.gp[0] = gdim[0]; gp.gp[1] = gdim[1]; gp.gp[2] = gdim[2];
+    gp.rl = cutoff + skin;
+    gp.gmax = GMAX_NONPERIODIC;
+    gp.cells_per_rep = (int)cells_per_rep;
+    const double rl2 = rl * rl;
+    // scratch that must start at zero: status and edge count, cell counts and fill cursors
+    if (cudaMemsetAsync(meta, 0, sizeof(DevMeta), s) != cudaSuccess) return SCHNET_ERR_CUDA;
+    if (cudaMemsetAsync(ccnt, 0, sizeof(int32_t) * (ncell + 1), s) != cudaSuccess) return SCHNET_ERR_CUDA;
+    if (cudaMemsetAsync(cfill, 0, sizeof(int32_t) * (ncell + 1), s) != cudaSuccess) return SCHNET_ERR_CUDA;
+    k_pack_positions<<<nb, 256, 0, s>>>(N, d_pos, pos4, nullptr, 0, 0.f, meta);
+    k_atom_replica<<<nb, 256, 0, s>>>(N, R, d_replica_offsets, arep);
+    k_replica_grid<<<R, 256, 0, s>>>(R, d_replica_offsets, pos4, gp, bx, dims, org, inv);
+    k_cell_assign<<<nb, 256, 0, s>>>(N, pos4, arep, dims, org, inv, gp.periodic, cell_of, ccnt);
+    if (scan_exclusive_raw(s, ccnt, (int)ncell, cstart, nullptr, scan_tmp) != cudaSuccess) return SCHNET_ERR_CUDA;
+    k_cell_fill<<<nb, 256, 0, s>>>(N, cell_of, cstart, cfill, catoms);
+    k_count<<<nb128, 128, 0, s>>>(N, pos4, arep, cell_of, dims, cstart, catoms, rl2, bx, rowcnt);
+    if (scan_exclusive_raw(s, rowcnt, N, d_row_ptr, &meta->n_edges, scan_tmp) != cudaSuccess)
+        return SCHNET_ERR_CUDA;
+    // unsorted columns staged in the caller's rev buffer; col doubles as the edge-row scratch
+    k_fill<<<nb128, 128, 0, s>>>(N, pos4, arep, cell_of, dims, cstart, catoms, rl2, bx, d_row_ptr, edge_capacity,
+                                 meta, d_rev, d_col);
+    k_sort_rows<<<256, 256, 0, s>>>(N, d_row_ptr, d_rev, edge_capacity, meta, d_col);
+    k_rev_rows<<<256, 256, 0, s>>>(N, d_row_ptr, d_col, edge_capacity, meta, d_rev);
+    k_copy_edge_count<<<1, 1, 0, s>>>(meta, d_n_edges);
+    return cudaGetLastError() == cudaSuccess ? SCHNET_OK : SCHNET_ERR_CUDA;
+}

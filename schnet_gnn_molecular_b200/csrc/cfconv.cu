@@ -45,17 +45,20 @@ struct MPArgs {
     int accumulate_s;
 };
 
+constexpr int NT = 512;   // threads per CTA: 16 warps, four per TMEM lane quadrant
+
 // shared-memory map (bytes)
 constexpr uint32_t SM_W1 = 0;                          // W1^T hi, lo   2 x 16 KB
 constexpr uint32_t SM_W2 = 32768;                      // W2^T hi, lo   2 x 32 KB
 constexpr uint32_t SM_X = 98304;                       // fwd: rbf hi/lo (32 KB) ; bwd: rbf, rbf' then a (64 KB)
 constexpr uint32_t SM_FWD_A = 131072;                  // fwd: a hi/lo (64 KB)
-constexpr uint32_t SM_BWD_Y = 163840;                  // bwd: ssp'(p) p' hi/lo (64 KB)
+constexpr uint32_t SM_BWD_Y = 163840;                  // bwd: ssp'(p) p' hi/lo (64 KB); partial sums after GEMM2
 constexpr uint32_t SM_META_FWD = 196608;
 constexpr uint32_t SM_META_BWD = 229376;
-constexpr uint32_t META_BYTES = 2048 + 16;
-constexpr uint32_t SMEM_FWD = SM_META_FWD + META_BYTES;
-constexpr uint32_t SMEM_BWD = SM_META_BWD + META_BYTES;
+constexpr uint32_t TILEMETA_BYTES = 2048;
+constexpr uint32_t PART_BYTES = 2 * 4 * 128 * 4;       // first/last-row partial per chunk and feature
+constexpr uint32_t SMEM_FWD = SM_META_FWD + TILEMETA_BYTES + PART_BYTES + 16;
+constexpr uint32_t SMEM_BWD = SM_META_BWD + TILEMETA_BYTES + 16;
 
 constexpr uint32_t RBF_TERM = TILE_E * KP * 2;   // 16 KB: one 16-bit term of a [128 x 64] tile
 constexpr uint32_t ACT_TERM = TILE_E * FP * 2;   // 32 KB: one 16-bit term of a [128 x 128] tile
@@ -75,69 +78,121 @@ __device__ __forceinline__ void copy_weights(uint8_t* smem, const uint8_t* __res
     for (int i = threadIdx.x; i < (int)(LAYER_IMG / 16); i += blockDim.x) dst[i] = __ldg(src + i);
 }
 
-__device__ __forceinline__ uint4 pack8(const uint16_t (&v)[8])
+// two fp32 values -> packed 16-bit hi pair and lo (residual) pair
+template <int FMT>
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo);
+template <>
+__device__ __forceinline__ void split2<0>(float x0, float x1, uint32_t& hi, uint32_t& lo)
 {
-    return make_uint4((uint32_t)v[0] | ((uint32_t)v[1] << 16), (uint32_t)v[2] | ((uint32_t)v[3] << 16),
-                      (uint32_t)v[4] | ((uint32_t)v[5] << 16), (uint32_t)v[6] | ((uint32_t)v[7] << 16));
+    __half2 h = __floats2half2_rn(x0, x1);
+    float2 hf = __half22float2(h);
+    __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<uint32_t*>(&h);
+    lo = *reinterpret_cast<uint32_t*>(&l);
+}
+template <>
+__device__ __forceinline__ void split2<1>(float x0, float x1, uint32_t& hi, uint32_t& lo)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    float2 hf = __bfloat1622float2(h);
+    __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<uint32_t*>(&h);
+    lo = *reinterpret_cast<uint32_t*>(&l);
 }
 
-// Stage R: thread t handles edge t of the tile: distance (minimum image),
-// cutoff mask, Gaussian expansion (and its d-derivative when BWD) written as
-// hi/lo 16-bit K-major B operands.
-template <int FMT, bool BWD>
-__device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMeta* tm, long long e0, int ne)
+// 8 consecutive fp32 values -> one 16-byte hi store and one 16-byte lo store
+template <int FMT>
+__device__ __forceinline__ void store8(uint8_t* hi_base, uint8_t* lo_base, uint32_t off, const float* v)
 {
-    const int t = threadIdx.x;
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) split2<FMT>(v[2 * q], v[2 * q + 1], h[q], l[q]);
+    *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(lo_base + off) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// 32 lanes x 16 columns of TMEM -> 16 registers per thread
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
+{
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+
+// Endpoints of edge (threadIdx.x mod 128) of a tile, loaded one tile ahead so the
+// dependent loads (edge -> atom -> position) overlap the previous tile's work.
+struct EdgePre {
+    int i, j;
+    float4 pi, pj;
+};
+
+__device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, int ne)
+{
+    EdgePre p;
+    p.i = 0;
+    p.j = -1;
+    p.pi = p.pj = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int t = threadIdx.x & (TILE_E - 1);
+    if (t < ne) {
+        p.i = __ldg(a.erow + e0 + t);
+        p.j = __ldg(a.col + e0 + t);
+        p.pi = __ldg(a.pos4 + p.i);
+        p.pj = __ldg(a.pos4 + p.j);
+    }
+    return p;
+}
+
+// Stage R: four threads per edge (one per 16 Gaussians): distance (minimum
+// image), cutoff mask, Gaussian expansion (and its d-derivative when BWD)
+// written as hi/lo 16-bit K-major B operands.
+template <int FMT, bool BWD>
+__device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMeta* tm, const EdgePre& ep, int ne)
+{
+    const int e = threadIdx.x & (TILE_E - 1);
+    const int kq = threadIdx.x >> 7;
     float d = 0.f;
     bool valid = false;
-    int i = 0, j = -1;
-    if (t < ne) {
-        long long e = e0 + t;
-        i = a.erow[e];
-        j = a.col[e];
-        float4 pi = a.pos4[i], pj = a.pos4[j];
-        float3 v = min_image(make_float3(pj.x - pi.x, pj.y - pi.y, pj.z - pi.z), a.box);
+    if (e < ne) {
+        float3 v = min_image(make_float3(ep.pj.x - ep.pi.x, ep.pj.y - ep.pi.y, ep.pj.z - ep.pi.z), a.box);
         d = sqrtf(v.x * v.x + v.y * v.y + v.z * v.z);
         valid = d < a.rc && d > 0.f;
     }
-    float fc = 0.f, dfc = 0.f;
-    if (valid) {
-        float s, c;
-        sincospif(d * a.inv_rc, &s, &c);
-        fc = 0.5f * (c + 1.0f);
-        dfc = -0.5f * 3.14159265358979f * a.inv_rc * s;
+    if (kq == 0) {
+        float fc = 0.f, dfc = 0.f;
+        if (valid) {
+            float sn, cs;
+            sincospif(d * a.inv_rc, &sn, &cs);
+            fc = 0.5f * (cs + 1.0f);
+            dfc = -0.5f * 3.14159265358979f * a.inv_rc * sn;
+        }
+        tm->row[e] = e < ne ? ep.i : 0x7fffffff;
+        tm->col[e] = valid ? ep.j : -1;
+        tm->fc[e] = fc;
+        tm->dfc[e] = dfc;
     }
-    tm->row[t] = t < ne ? i : 0x7fffffff;
-    tm->col[t] = valid ? j : -1;
-    tm->fc[t] = fc;
-    tm->dfc[t] = dfc;
-
     uint8_t* b_hi = smem + SM_X;
     uint8_t* b_lo = b_hi + RBF_TERM;
     uint8_t* p_hi = smem + SM_X + 2 * RBF_TERM;   // derivative tile (backward)
     uint8_t* p_lo = p_hi + RBF_TERM;
 #pragma unroll
-    for (int kg = 0; kg < KP / 8; ++kg) {
-        uint16_t hi[8], lo[8], dhi[8], dlo[8];
+    for (int g = 0; g < 2; ++g) {
+        const int kg = kq * 2 + g;
+        float gv[8], dv[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            int k = kg * 8 + q;
-            float g = 0.f, dg = 0.f;
-            if (valid && k < a.K) {
-                float x = d - (a.mu0 + (float)k * a.dmu);
-                g = __expf(-x * x * a.inv2s2);
-                dg = -x * a.invs2 * g;
-            }
-            Split<FMT>::run(g, hi[q], lo[q]);
-            if (BWD) Split<FMT>::run(dg, dhi[q], dlo[q]);
+            const int k = kg * 8 + q;
+            float x = d - (a.mu0 + (float)k * a.dmu);
+            float gg = (valid && k < a.K) ? __expf(-x * x * a.inv2s2) : 0.f;
+            gv[q] = gg;
+            dv[q] = -x * a.invs2 * gg;
         }
-        uint32_t off = kmajor_off(t, kg * 8, TILE_E);
-        *reinterpret_cast<uint4*>(b_hi + off) = pack8(hi);
-        *reinterpret_cast<uint4*>(b_lo + off) = pack8(lo);
-        if (BWD) {
-            *reinterpret_cast<uint4*>(p_hi + off) = pack8(dhi);
-            *reinterpret_cast<uint4*>(p_lo + off) = pack8(dlo);
-        }
+        const uint32_t off = kmajor_off(e, kg * 8, TILE_E);
+        store8<FMT>(b_hi, b_lo, off, gv);
+        if (BWD) store8<FMT>(p_hi, p_lo, off, dv);
     }
 }
 
@@ -172,35 +227,93 @@ __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, DevMeta
     return true;
 }
 
-// Write a 128-edge activation row (thread = feature f = K index) into an
-// MN-major B operand: 8 consecutive edges per 16-byte store.
-template <int FMT>
-__device__ __forceinline__ void store_act_group(uint8_t* base, int f, int e8, const float* v)
+// x_j,f (one feature per thread) for n consecutive edges starting at e; masked edges read nothing
+template <int N>
+__device__ __forceinline__ void gather(const float* __restrict__ src, const TileMeta* tm, int e, int f,
+                                       float (&dst)[N])
 {
-    uint16_t hi[8], lo[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) Split<FMT>::run(v[q], hi[q], lo[q]);
-    uint32_t off = mnmajor_off(e8, f, TILE_E);
-    *reinterpret_cast<uint4*>(base + off) = pack8(hi);
-    *reinterpret_cast<uint4*>(base + ACT_TERM + off) = pack8(lo);
+    for (int q = 0; q < N; ++q) {
+        const int j = tm->col[e + q];
+        dst[q] = j >= 0 ? __ldg(src + (size_t)j * FP + f) : 0.f;
+    }
+}
+
+// Segmented sum over the edges of one 32-edge chunk (one feature per thread):
+// rows that start and end inside the chunk are written out directly (with
+// zeros for edge-less rows between them); the chunk's first row and, when
+// different, its last row leave partial sums (pf, pl) for the in-order merge.
+struct ChunkSeg {
+    int rfirst, lrow;
+    float acc, pf;
+};
+
+__device__ __forceinline__ void seg_begin(ChunkSeg& c, const TileMeta* tm, int eb)
+{
+    c.rfirst = tm->row[eb];
+    c.lrow = c.rfirst;
+    c.acc = 0.f;
+    c.pf = 0.f;
+}
+
+__device__ __forceinline__ void seg_row(ChunkSeg& c, int row, float* __restrict__ out, int f)
+{
+    if (row != c.lrow) {
+        if (c.lrow == c.rfirst) c.pf = c.acc;
+        else out[(size_t)c.lrow * FP + f] = c.acc;
+        for (int rr = c.lrow + 1; rr < row; ++rr) out[(size_t)rr * FP + f] = 0.f;
+        c.lrow = row;
+        c.acc = 0.f;
+    }
+}
+
+// In-order merge of the four chunks' partials (threads 0..127, feature f).
+__device__ __forceinline__ void merge_chunks(const TileMeta* tm, const float* pf, const float* pl, int ne, int f,
+                                             float* __restrict__ out, int& cur, float& acc)
+{
+#pragma unroll 1
+    for (int c = 0; c < TILE_E / 32; ++c) {
+        const int eb = c * 32;
+        if (eb >= ne) break;
+        const int last = min(eb + 31, ne - 1);
+        const int rfirst = tm->row[eb], rlast = tm->row[last];
+        const float v = pf[c * 128 + f];
+        if (rfirst == cur) {
+            acc += v;
+        } else {
+            out[(size_t)cur * FP + f] = acc;
+            for (int rr = cur + 1; rr < rfirst; ++rr) out[(size_t)rr * FP + f] = 0.f;
+            cur = rfirst;
+            acc = v;
+        }
+        if (rlast != rfirst) {
+            out[(size_t)cur * FP + f] = acc;
+            cur = rlast;
+            acc = pl[c * 128 + f];
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
 // forward: m_i = sum_j h_j (.) W(d_ij)
 // ---------------------------------------------------------------------------
 template <int FMT, int NW>
-__global__ void __launch_bounds__(128, 1) k_cfconv_fwd(MPArgs a)
+__global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     TileMeta* tm = reinterpret_cast<TileMeta*>(smem + SM_META_FWD);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_FWD + 2048);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_FWD + 2056);
+    float* pf_s = reinterpret_cast<float*>(smem + SM_META_FWD + TILEMETA_BYTES);
+    float* pl_s = pf_s + 4 * 128;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_FWD + TILEMETA_BYTES + PART_BYTES);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_FWD + TILEMETA_BYTES + PART_BYTES + 8);
 
     if (a.meta->n_edges > a.cap) return;
     const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
     if (r0 >= r1) return;
     const long long e0 = a.row_ptr[r0], e1 = a.row_ptr[r1];
-    const int f = threadIdx.x, warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qd = warp & 3, cg = warp >> 2;        // TMEM lane quadrant, 32-edge column chunk
+    const int f = qd * 32 + lane;                   // this thread's output feature
 
     if (warp == 0) {
         tmem_alloc(tslot, 256);
@@ -216,84 +329,93 @@ __global__ void __launch_bounds__(128, 1) k_cfconv_fwd(MPArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t tP = tmem, tQ = tmem + 128;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const uint32_t tP = tmem + lane_off + cg * 32, tQ = tmem + 128 + lane_off + cg * 32;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t id = idesc_f16(128, TILE_E, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, TILE_E, FMT, 1);
 
     const float s1 = a.s1[f], b1 = a.b1[f], s2 = a.s2[f], b2 = a.b2[f];
-    int cur = r0;
+    int cur = r0;          // carried row and partial sum (threads 0..127, feature = threadIdx.x)
     float acc = 0.f;
     uint32_t phase = 0;
     bool ok = true;
 
+    EdgePre ep = prefetch_edge(a, e0, (int)min((long long)TILE_E, e1 - e0));
     for (long long t0 = e0; t0 < e1 && ok; t0 += TILE_E) {
         const int ne = (int)min((long long)TILE_E, e1 - t0);
-        stage_rbf<FMT, false>(a, smem, tm, t0, ne);
+        stage_rbf<FMT, false>(a, smem, tm, ep, ne);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         if (threadIdx.x == 0) {
             tc_fence_after();
-            issue_gemm<NW>(tP, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
+            issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
             mma_commit(bar);
         }
         if (!(ok = wait_mma(bar, phase, a.meta))) break;
 
-        // epilogue 1: a = ssp(s1 P + b1) -> MN-major B operand of GEMM2
-#pragma unroll 1
-        for (int c = 0; c < TILE_E / 32; ++c) {
+        // epilogue 1: a = ssp(s1 P + b1) for this warp's 32 edges -> MN-major B operand
+        {
             float r[32];
-            tmem_ld32(tP + lane_off + c * 32, r);
+            tmem_ld32(tP, r);
             tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 32; ++q) r[q] = ssp(fmaf(s1, r[q], b1));
 #pragma unroll
-            for (int g = 0; g < 4; ++g) store_act_group<FMT>(smem + SM_FWD_A, f, c * 32 + g * 8, r + g * 8);
+            for (int g = 0; g < 4; ++g) {
+                const uint32_t off = mnmajor_off(cg * 32 + g * 8, f, TILE_E);
+                store8<FMT>(smem + SM_FWD_A, smem + SM_FWD_A + ACT_TERM, off, r + g * 8);
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         if (threadIdx.x == 0) {
             tc_fence_after();
-            issue_gemm<NW>(tQ, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_FWD_A, ACT_TERM, FP / 16, id_mn);
+            issue_gemm<NW>(tmem + 128, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_FWD_A, ACT_TERM, FP / 16,
+                           id_mn);
             mma_commit(bar);
         }
+        // this chunk's h_j rows are fetched while GEMM2 runs
+        const int eb = cg * 32;
+        float hv[32];
+        gather<32>(a.h, tm, eb, f, hv);
         if (!(ok = wait_mma(bar, phase, a.meta))) break;
+        if (t0 + TILE_E < e1) ep = prefetch_edge(a, t0 + TILE_E, (int)min((long long)TILE_E, e1 - t0 - TILE_E));
 
-        // epilogue 2: W = f_c (s2 Q + b2); segment sum of h_j (.) W per row
-#pragma unroll 1
-        for (int c = 0; c < TILE_E / 32; ++c) {
-            if (c * 32 >= ne) break;
+        // epilogue 2: W = f_c (s2 Q + b2); segmented sum of h_j (.) W over this chunk
+        {
             float r[32];
-            tmem_ld32(tQ + lane_off + c * 32, r);
+            tmem_ld32(tQ, r);
             tmem_ld_wait();
+            float pf = 0.f, pl = 0.f;
+            if (eb < ne) {
+                ChunkSeg c{0, 0, 0.f, 0.f};
+                seg_begin(c, tm, eb);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int e = c * 32 + q;
-                if (e >= ne) break;
-                const int row = tm->row[e];
-                if (row != cur) {
-                    a.out[(size_t)cur * FP + f] = acc;
-                    for (int rr = cur + 1; rr < row; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
-                    cur = row;
-                    acc = 0.f;
+                for (int q = 0; q < 32; ++q) {
+                    const int e = eb + q;
+                    if (e >= ne) break;
+                    seg_row(c, tm->row[e], a.out, f);
+                    if (tm->col[e] >= 0) c.acc = fmaf(tm->fc[e] * fmaf(s2, r[q], b2), hv[q], c.acc);
                 }
-                const int j = tm->col[e];
-                if (j >= 0) {
-                    float w = tm->fc[e] * fmaf(s2, r[q], b2);
-                    acc = fmaf(w, __ldg(a.h + (size_t)j * FP + f), acc);
-                }
+                if (c.lrow == c.rfirst) pf = c.acc; else { pf = c.pf; pl = c.acc; }
             }
+            pf_s[cg * 128 + f] = pf;
+            pl_s[cg * 128 + f] = pl;
         }
+        __syncthreads();
+        if (threadIdx.x < 128) merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
         tc_fence_before();
-        __syncthreads();   // tile metadata and operand tiles are rewritten next
+        __syncthreads();   // tile metadata, partials and operand tiles are rewritten next
     }
 
     if (ok) {
-        a.out[(size_t)cur * FP + f] = acc;
-        for (int rr = cur + 1; rr < r1; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
+        if (threadIdx.x < 128) {
+            a.out[(size_t)cur * FP + threadIdx.x] = acc;
+            for (int rr = cur + 1; rr < r1; ++rr) a.out[(size_t)rr * FP + threadIdx.x] = 0.f;
+        }
     } else {
         // drain: give in-flight MMAs a bounded chance to retire before freeing TMEM
         mbar_wait_bounded(bar, phase, WAIT_POLLS);
@@ -310,19 +432,24 @@ __global__ void __launch_bounds__(128, 1) k_cfconv_fwd(MPArgs a)
 // backward: dh_i = sum_j u_j (.) W_ij ;  s_e = sum_f W'_e,f u_i,f h_j,f
 // ---------------------------------------------------------------------------
 template <int FMT, int NW>
-__global__ void __launch_bounds__(128, 1) k_cfconv_bwd(MPArgs a)
+__global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     TileMeta* tm = reinterpret_cast<TileMeta*>(smem + SM_META_BWD);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_BWD + 2048);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_BWD + 2056);
-    float* partial = reinterpret_cast<float*>(smem + SM_BWD_Y);   // [4][128] after GEMM2
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_BWD + TILEMETA_BYTES);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_BWD + TILEMETA_BYTES + 8);
+    // after GEMM2 the ssp'(p)p' tile is dead: its space holds the partial sums
+    float* pf_s = reinterpret_cast<float*>(smem + SM_BWD_Y);
+    float* pl_s = pf_s + 4 * 128;
+    float* ps_s = pl_s + 4 * 128;   // [quadrant][edge] per-edge partial of s_e
 
     if (a.meta->n_edges > a.cap) return;
     const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
     if (r0 >= r1) return;
     const long long e0 = a.row_ptr[r0], e1 = a.row_ptr[r1];
-    const int f = threadIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qd = warp & 3, cg = warp >> 2;
+    const int f = qd * 32 + lane;
 
     if (warp == 0) {
         tmem_alloc(tslot, 512);
@@ -338,8 +465,10 @@ __global__ void __launch_bounds__(128, 1) k_cfconv_bwd(MPArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    const uint32_t tP = tmem, tPd = tmem + 128, tQ = tmem + 256, tQd = tmem + 384;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    const uint32_t col0 = cg * 32;
+    const uint32_t tP = tmem + lane_off + col0, tPd = tmem + 128 + lane_off + col0;
+    const uint32_t tQ = tmem + 256 + lane_off + col0, tQd = tmem + 384 + lane_off + col0;
     const uint32_t sbase = smem_u32(smem);
     const uint32_t id = idesc_f16(128, TILE_E, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, TILE_E, FMT, 1);
@@ -347,43 +476,44 @@ __global__ void __launch_bounds__(128, 1) k_cfconv_bwd(MPArgs a)
     const float s1 = a.s1[f], b1 = a.b1[f], s2 = a.s2[f], b2 = a.b2[f];
     int cur = r0;
     float acc = 0.f;
-    float u_row = a.u[(size_t)r0 * FP + f];
     uint32_t phase = 0;
     bool ok = true;
 
+    EdgePre ep = prefetch_edge(a, e0, (int)min((long long)TILE_E, e1 - e0));
     for (long long t0 = e0; t0 < e1 && ok; t0 += TILE_E) {
         const int ne = (int)min((long long)TILE_E, e1 - t0);
-        stage_rbf<FMT, true>(a, smem, tm, t0, ne);
+        stage_rbf<FMT, true>(a, smem, tm, ep, ne);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         if (threadIdx.x == 0) {
             tc_fence_after();
-            issue_gemm<NW>(tP, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
-            issue_gemm<NW>(tPd, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X + 2 * RBF_TERM, RBF_TERM, KP / 16,
-                           id);
+            issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
+            issue_gemm<NW>(tmem + 128, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X + 2 * RBF_TERM, RBF_TERM,
+                           KP / 16, id);
             mma_commit(bar);
         }
         if (!(ok = wait_mma(bar, phase, a.meta))) break;
 
-        // epilogue 1: a = ssp(p), b = ssp'(p) p'   (p = s1 P + b1, p' = s1 P')
-#pragma unroll 1
-        for (int c = 0; c < TILE_E / 32; ++c) {
-            float r[32], rd[32];
-            tmem_ld32(tP + lane_off + c * 32, r);
-            tmem_ld32(tPd + lane_off + c * 32, rd);
+        // epilogue 1: a = ssp(p), b = ssp'(p) p'   (p = s1 P + b1, p' = s1 P'), 16 edges at a time
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float r[16], rd[16];
+            tmem_ld16(tP + hh * 16, r);
+            tmem_ld16(tPd + hh * 16, rd);
             tmem_ld_wait();
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
+            for (int q = 0; q < 16; ++q) {
                 float sv, gv;
                 ssp_and_grad(fmaf(s1, r[q], b1), sv, gv);
                 r[q] = sv;
                 rd[q] = gv * s1 * rd[q];
             }
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                store_act_group<FMT>(smem + SM_X, f, c * 32 + g * 8, r + g * 8);
-                store_act_group<FMT>(smem + SM_BWD_Y, f, c * 32 + g * 8, rd + g * 8);
+            for (int g = 0; g < 2; ++g) {
+                const uint32_t off = mnmajor_off(col0 + hh * 16 + g * 8, f, TILE_E);
+                store8<FMT>(smem + SM_X, smem + SM_X + ACT_TERM, off, r + g * 8);
+                store8<FMT>(smem + SM_BWD_Y, smem + SM_BWD_Y + ACT_TERM, off, rd + g * 8);
             }
         }
         fence_proxy_async_smem();
@@ -391,73 +521,95 @@ __global__ void __launch_bounds__(128, 1) k_cfconv_bwd(MPArgs a)
         __syncthreads();
         if (threadIdx.x == 0) {
             tc_fence_after();
-            issue_gemm<NW>(tQ, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_X, ACT_TERM, FP / 16, id_mn);
-            issue_gemm<NW>(tQd, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_BWD_Y, ACT_TERM, FP / 16, id_mn);
+            issue_gemm<NW>(tmem + 256, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_X, ACT_TERM, FP / 16, id_mn);
+            issue_gemm<NW>(tmem + 384, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_BWD_Y, ACT_TERM, FP / 16,
+                           id_mn);
             mma_commit(bar);
         }
+        const int eb = (int)col0;
+        float uv[16], hv[16];
+        gather<16>(a.u, tm, eb, f, uv);
+        gather<16>(a.h, tm, eb, f, hv);
         if (!(ok = wait_mma(bar, phase, a.meta))) break;
+        if (t0 + TILE_E < e1) ep = prefetch_edge(a, t0 + TILE_E, (int)min((long long)TILE_E, e1 - t0 - TILE_E));
 
         // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 Q + b2, z' = s2 Q')
-#pragma unroll 1
-        for (int c = 0; c < TILE_E / 32; ++c) {
-            float r[32], rd[32];
-            tmem_ld32(tQ + lane_off + c * 32, r);
-            tmem_ld32(tQd + lane_off + c * 32, rd);
-            tmem_ld_wait();
+        {
+            ChunkSeg c{0, 0, 0.f, 0.f};
+            const bool active = eb < ne;
+            if (active) seg_begin(c, tm, eb);
+            float u_row = active ? __ldg(a.u + (size_t)c.rfirst * FP + f) : 0.f;
 #pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int e = c * 32 + q;
-                float tval = 0.f;
-                if (e < ne) {
-                    const int row = tm->row[e];
-                    if (row != cur) {
-                        a.out[(size_t)cur * FP + f] = acc;
-                        for (int rr = cur + 1; rr < row; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
-                        cur = row;
-                        acc = 0.f;
-                        u_row = a.u[(size_t)row * FP + f];
+            for (int hh = 0; hh < 2; ++hh) {
+                if (hh == 1) {
+                    gather<16>(a.u, tm, eb + 16, f, uv);
+                    gather<16>(a.h, tm, eb + 16, f, hv);
+                }
+                float r[16], rd[16];
+                tmem_ld16(tQ + hh * 16, r);
+                tmem_ld16(tQd + hh * 16, rd);
+                tmem_ld_wait();
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const int e = eb + hh * 16 + q;
+                    float tval = 0.f;
+                    if (e < ne) {
+                        const int row = tm->row[e];
+                        if (row != c.lrow) {
+                            seg_row(c, row, a.out, f);
+                            u_row = __ldg(a.u + (size_t)row * FP + f);
+                        }
+                        if (tm->col[e] >= 0) {
+                            const float z = fmaf(s2, r[q], b2);
+                            const float fcv = tm->fc[e];
+                            const float wd = fmaf(tm->dfc[e], z, fcv * s2 * rd[q]);
+                            c.acc = fmaf(fcv * z, uv[q], c.acc);
+                            tval = wd * u_row * hv[q];
+                        }
                     }
-                    const int j = tm->col[e];
-                    if (j >= 0) {
-                        const float z = fmaf(s2, r[q], b2);
-                        const float fcv = tm->fc[e];
-                        const float w = fcv * z;
-                        const float wd = fmaf(tm->dfc[e], z, fcv * s2 * rd[q]);
-                        const float uj = __ldg(a.u + (size_t)j * FP + f);
-                        const float hj = __ldg(a.h + (size_t)j * FP + f);
-                        acc = fmaf(w, uj, acc);
-                        tval = wd * u_row * hj;
+                    rd[q] = tval;
+                }
+                // transpose-reduce the 16 per-edge values over the warp's 32 features:
+                // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
+#pragma unroll
+                for (int sh = 16; sh >= 2; sh >>= 1) {
+                    const bool upper = (lane & sh) != 0;
+#pragma unroll
+                    for (int k = 0; k < sh / 2; ++k) {
+                        float send = upper ? rd[k] : rd[k + sh / 2];
+                        float keep = upper ? rd[k + sh / 2] : rd[k];
+                        rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
                     }
                 }
-                rd[q] = tval;
+                rd[0] += __shfl_xor_sync(0xffffffffu, rd[0], 1);
+                if ((lane & 1) == 0) ps_s[qd * TILE_E + eb + hh * 16 + (lane >> 1)] = rd[0];
             }
-            // transpose-reduce the 32 per-edge values over the warp's 32 features:
-            // afterwards lane l holds the warp's sum for edge c*32 + l.
-#pragma unroll
-            for (int sh = 16; sh >= 1; sh >>= 1) {
-                const bool upper = (lane & sh) != 0;
-#pragma unroll
-                for (int k = 0; k < sh; ++k) {
-                    float send = upper ? rd[k] : rd[k + sh];
-                    float keep = upper ? rd[k + sh] : rd[k];
-                    rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
-                }
+            float pf = 0.f, pl = 0.f;
+            if (active) {
+                if (c.lrow == c.rfirst) pf = c.acc; else { pf = c.pf; pl = c.acc; }
             }
-            partial[warp * TILE_E + c * 32 + lane] = rd[0];
+            pf_s[cg * 128 + f] = pf;
+            pl_s[cg * 128 + f] = pl;
         }
         __syncthreads();
-        if (f < ne) {
-            float s = partial[f] + partial[TILE_E + f] + partial[2 * TILE_E + f] + partial[3 * TILE_E + f];
-            float* dst = a.s_edge + (t0 + f);
-            *dst = a.accumulate_s ? *dst + s : s;
+        if (threadIdx.x < 128) {
+            merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
+            const int t = threadIdx.x;
+            if (t < ne) {
+                const float sv = ps_s[t] + ps_s[TILE_E + t] + ps_s[2 * TILE_E + t] + ps_s[3 * TILE_E + t];
+                float* dst = a.s_edge + (t0 + t);
+                *dst = a.accumulate_s ? *dst + sv : sv;
+            }
         }
         tc_fence_before();
         __syncthreads();
     }
 
     if (ok) {
-        a.out[(size_t)cur * FP + f] = acc;
-        for (int rr = cur + 1; rr < r1; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
+        if (threadIdx.x < 128) {
+            a.out[(size_t)cur * FP + threadIdx.x] = acc;
+            for (int rr = cur + 1; rr < r1; ++rr) a.out[(size_t)rr * FP + threadIdx.x] = 0.f;
+        }
     } else {
         mbar_wait_bounded(bar, phase, WAIT_POLLS);
     }
@@ -526,11 +678,11 @@ cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
     MPArgs a = make_args(c, layer);
     a.out = c->ws.m;
     if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_fwd<0, 2><<<c->ncta, 128, SMEM_FWD, c->s>>>(a);
+        k_cfconv_fwd<0, 2><<<c->ncta, NT, SMEM_FWD, c->s>>>(a);
     else if (c->weight_fmt == 0)
-        k_cfconv_fwd<0, 1><<<c->ncta, 128, SMEM_FWD, c->s>>>(a);
+        k_cfconv_fwd<0, 1><<<c->ncta, NT, SMEM_FWD, c->s>>>(a);
     else
-        k_cfconv_fwd<1, 1><<<c->ncta, 128, SMEM_FWD, c->s>>>(a);
+        k_cfconv_fwd<1, 1><<<c->ncta, NT, SMEM_FWD, c->s>>>(a);
     c->launches += 1;
     return cudaGetLastError();
 }
@@ -541,11 +693,11 @@ cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s)
     a.out = c->ws.dh;
     a.accumulate_s = accumulate_s;
     if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_bwd<0, 2><<<c->ncta, 128, SMEM_BWD, c->s>>>(a);
+        k_cfconv_bwd<0, 2><<<c->ncta, NT, SMEM_BWD, c->s>>>(a);
     else if (c->weight_fmt == 0)
-        k_cfconv_bwd<0, 1><<<c->ncta, 128, SMEM_BWD, c->s>>>(a);
+        k_cfconv_bwd<0, 1><<<c->ncta, NT, SMEM_BWD, c->s>>>(a);
     else
-        k_cfconv_bwd<1, 1><<<c->ncta, 128, SMEM_BWD, c->s>>>(a);
+        k_cfconv_bwd<1, 1><<<c->ncta, NT, SMEM_BWD, c->s>>>(a);
     c->launches += 1;
     return cudaGetLastError();
 }

@@ -216,7 +216,8 @@ enum {
     SCHNET_KERNEL_FORCES = 4,      /* force assembly from the per-edge scalars                 */
     SCHNET_KERNEL_INTEGRATE = 5,   /* B-A-O-A and closing B kicks                              */
     SCHNET_KERNEL_REDUCE = 6,      /* per-replica energy sums                                  */
-    SCHNET_KERNEL_NCLASS = 7
+    SCHNET_KERNEL_MASK = 7,        /* per-step cutoff masking: listed edges with d < r_c       */
+    SCHNET_KERNEL_NCLASS = 8
 };
 
 /* Profiling pass: continue the trajectory for n_steps steps exactly as

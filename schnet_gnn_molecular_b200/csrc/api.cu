@@ -152,6 +152,8 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.col = cv.take<int32_t>(d.cap); w.coltmp = cv.take<int32_t>(d.cap);
     w.rev = cv.take<int32_t>(d.cap); w.erow = cv.take<int32_t>(d.cap);
     w.s_edge = cv.take<float>(d.cap);
+    w.crow = cv.take<int32_t>(d.cap); w.ccol = cv.take<int32_t>(d.cap); w.cidx = cv.take<int32_t>(d.cap);
+    w.ccount = cv.take<int32_t>(MAX_CTA);
     w.part = cv.take<int32_t>(MAX_CTA + 1);
     w.cell_of = cv.take<int32_t>(N); w.cell_atoms = cv.take<int32_t>(N);
     w.cell_cnt = cv.take<int32_t>((size_t)d.ncell + 1); w.cell_start = cv.take<int32_t>((size_t)d.ncell + 1);
@@ -468,6 +470,7 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
         Timed t_(c, kind);                              \
         if ((e = (expr)) != cudaSuccess) return e;      \
     } while (0)
+    SCHNET_TIMED(SCHNET_KERNEL_MASK, launch_compact(c));
     SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_first(c, types));
     for (int l = 0; l < c->L; ++l) {
         SCHNET_TIMED(SCHNET_KERNEL_CFCONV_FWD, launch_cfconv_fwd(c, l));

@@ -26,8 +26,10 @@ namespace schnet {
 
 struct MPArgs {
     const float4* pos4;
-    const int32_t* erow;
-    const int32_t* col;
+    const int32_t* crow;     // compacted edges (d < r_c) of each CTA's rows: row, column,
+    const int32_t* ccol;     //   and index in the full list; CTA c's run starts at
+    const int32_t* cidx;     //   row_ptr[part[c]] and holds ccount[c] edges
+    const int32_t* ccount;
     const int32_t* row_ptr;
     const int32_t* part;
     DevMeta* meta;
@@ -64,12 +66,13 @@ constexpr uint32_t RBF_TERM = TILE_E * KP * 2;   // 16 KB: one 16-bit term of a 
 constexpr uint32_t ACT_TERM = TILE_E * FP * 2;   // 32 KB: one 16-bit term of a [128 x 128] tile
 constexpr uint32_t WAIT_POLLS = 1u << 22;
 
-struct TileMeta {
-    int32_t row[TILE_E];
-    int32_t col[TILE_E];   // -1: padding or d >= r_c (masked)
-    float fc[TILE_E];
-    float dfc[TILE_E];
+struct EdgeMeta {          // one 16-byte record per edge of the tile
+    int32_t row;
+    int32_t col;           // -1: padding or d >= r_c (masked)
+    float fc;
+    float dfc;
 };
+typedef EdgeMeta TileMeta;
 
 __device__ __forceinline__ void copy_weights(uint8_t* smem, const uint8_t* __restrict__ img)
 {
@@ -138,8 +141,8 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
     p.pi = p.pj = make_float4(0.f, 0.f, 0.f, 0.f);
     const int t = threadIdx.x & (TILE_E - 1);
     if (t < ne) {
-        p.i = __ldg(a.erow + e0 + t);
-        p.j = __ldg(a.col + e0 + t);
+        p.i = __ldg(a.crow + e0 + t);
+        p.j = __ldg(a.ccol + e0 + t);
         p.pi = __ldg(a.pos4 + p.i);
         p.pj = __ldg(a.pos4 + p.j);
     }
@@ -157,8 +160,8 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMe
     float d = 0.f;
     bool valid = false;
     if (e < ne) {
-        float3 v = min_image(make_float3(ep.pj.x - ep.pi.x, ep.pj.y - ep.pi.y, ep.pj.z - ep.pi.z), a.box);
-        d = sqrtf(v.x * v.x + v.y * v.y + v.z * v.z);
+        float3 v;
+        d = edge_distance(ep.pi, ep.pj, a.box, v);
         valid = d < a.rc && d > 0.f;
     }
     if (kq == 0) {
@@ -169,10 +172,12 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMe
             fc = 0.5f * (cs + 1.0f);
             dfc = -0.5f * 3.14159265358979f * a.inv_rc * sn;
         }
-        tm->row[e] = e < ne ? ep.i : 0x7fffffff;
-        tm->col[e] = valid ? ep.j : -1;
-        tm->fc[e] = fc;
-        tm->dfc[e] = dfc;
+        EdgeMeta m;
+        m.row = e < ne ? ep.i : 0x7fffffff;
+        m.col = valid ? ep.j : -1;
+        m.fc = fc;
+        m.dfc = dfc;
+        tm[e] = m;
     }
     uint8_t* b_hi = smem + SM_X;
     uint8_t* b_lo = b_hi + RBF_TERM;
@@ -216,7 +221,8 @@ __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_base, uin
 // Wait for the tensor-core commit; returns false (uniformly) on timeout.
 __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, DevMeta* meta)
 {
-    bool ok = mbar_wait_bounded(bar, phase, WAIT_POLLS);
+    bool ok = true;
+    if ((threadIdx.x >> 5) == 0) ok = mbar_wait_bounded(bar, phase, WAIT_POLLS);   // the others sleep below
     phase ^= 1u;
     int bad = __syncthreads_or(!ok);
     if (bad) {
@@ -234,7 +240,7 @@ __device__ __forceinline__ void gather(const float* __restrict__ src, const Tile
 {
 #pragma unroll
     for (int q = 0; q < N; ++q) {
-        const int j = tm->col[e + q];
+        const int j = tm[e + q].col;
         dst[q] = j >= 0 ? __ldg(src + (size_t)j * FP + f) : 0.f;
     }
 }
@@ -250,7 +256,7 @@ struct ChunkSeg {
 
 __device__ __forceinline__ void seg_begin(ChunkSeg& c, const TileMeta* tm, int eb)
 {
-    c.rfirst = tm->row[eb];
+    c.rfirst = tm[eb].row;
     c.lrow = c.rfirst;
     c.acc = 0.f;
     c.pf = 0.f;
@@ -276,7 +282,7 @@ __device__ __forceinline__ void merge_chunks(const TileMeta* tm, const float* pf
         const int eb = c * 32;
         if (eb >= ne) break;
         const int last = min(eb + 31, ne - 1);
-        const int rfirst = tm->row[eb], rlast = tm->row[last];
+        const int rfirst = tm[eb].row, rlast = tm[last].row;
         const float v = pf[c * 128 + f];
         if (rfirst == cur) {
             acc += v;
@@ -310,7 +316,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     if (a.meta->n_edges > a.cap) return;
     const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
     if (r0 >= r1) return;
-    const long long e0 = a.row_ptr[r0], e1 = a.row_ptr[r1];
+    const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qd = warp & 3, cg = warp >> 2;        // TMEM lane quadrant, 32-edge column chunk
     const int f = qd * 32 + lane;                   // this thread's output feature
@@ -397,8 +403,9 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
                 for (int q = 0; q < 32; ++q) {
                     const int e = eb + q;
                     if (e >= ne) break;
-                    seg_row(c, tm->row[e], a.out, f);
-                    if (tm->col[e] >= 0) c.acc = fmaf(tm->fc[e] * fmaf(s2, r[q], b2), hv[q], c.acc);
+                    const EdgeMeta m = tm[e];
+                    seg_row(c, m.row, a.out, f);
+                    if (m.col >= 0) c.acc = fmaf(m.fc * fmaf(s2, r[q], b2), hv[q], c.acc);
                 }
                 if (c.lrow == c.rfirst) pf = c.acc; else { pf = c.pf; pl = c.acc; }
             }
@@ -446,7 +453,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     if (a.meta->n_edges > a.cap) return;
     const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
     if (r0 >= r1) return;
-    const long long e0 = a.row_ptr[r0], e1 = a.row_ptr[r1];
+    const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qd = warp & 3, cg = warp >> 2;
     const int f = qd * 32 + lane;
@@ -554,15 +561,15 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                     const int e = eb + hh * 16 + q;
                     float tval = 0.f;
                     if (e < ne) {
-                        const int row = tm->row[e];
-                        if (row != c.lrow) {
-                            seg_row(c, row, a.out, f);
-                            u_row = __ldg(a.u + (size_t)row * FP + f);
+                        const EdgeMeta m = tm[e];
+                        if (m.row != c.lrow) {
+                            seg_row(c, m.row, a.out, f);
+                            u_row = __ldg(a.u + (size_t)m.row * FP + f);
                         }
-                        if (tm->col[e] >= 0) {
+                        if (m.col >= 0) {
                             const float z = fmaf(s2, r[q], b2);
-                            const float fcv = tm->fc[e];
-                            const float wd = fmaf(tm->dfc[e], z, fcv * s2 * rd[q]);
+                            const float fcv = m.fc;
+                            const float wd = fmaf(m.dfc, z, fcv * s2 * rd[q]);
                             c.acc = fmaf(fcv * z, uv[q], c.acc);
                             tval = wd * u_row * hv[q];
                         }
@@ -597,7 +604,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             const int t = threadIdx.x;
             if (t < ne) {
                 const float sv = ps_s[t] + ps_s[TILE_E + t] + ps_s[2 * TILE_E + t] + ps_s[3 * TILE_E + t];
-                float* dst = a.s_edge + (t0 + t);
+                float* dst = a.s_edge + a.cidx[t0 + t];
                 *dst = a.accumulate_s ? *dst + sv : sv;
             }
         }
@@ -622,6 +629,74 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 }
 
 // ---------------------------------------------------------------------------
+// cutoff masking: per CTA row range, the listed edges with d < r_c, in order
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) k_compact(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ part,
+                                                  const int32_t* __restrict__ erow, const int32_t* __restrict__ col,
+                                                  const float4* __restrict__ pos4, Box box, float rc, long long cap,
+                                                  const DevMeta* meta, int32_t* __restrict__ crow,
+                                                  int32_t* __restrict__ ccol, int32_t* __restrict__ cidx,
+                                                  int32_t* __restrict__ ccount)
+{
+    __shared__ int wcount[32];
+    __shared__ int total_s;
+    const int c = blockIdx.x;
+    const int r0 = part[c], r1 = part[c + 1];
+    if (meta->n_edges > cap || r0 >= r1) {
+        if (threadIdx.x == 0) ccount[c] = 0;
+        return;
+    }
+    const long long e0 = row_ptr[r0], e1 = row_ptr[r1];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long base = e0;
+    for (long long eb = e0; eb < e1; eb += blockDim.x) {
+        const long long e = eb + threadIdx.x;
+        bool valid = false;
+        int i = 0, j = 0;
+        if (e < e1) {
+            i = erow[e];
+            j = col[e];
+            float3 v;
+            const float d = edge_distance(pos4[i], pos4[j], box, v);
+            valid = d < rc && d > 0.f;
+        }
+        const unsigned mask = __ballot_sync(0xffffffffu, valid);
+        if (lane == 0) wcount[warp] = __popc(mask);
+        __syncthreads();
+        if (warp == 0) {
+            int v = wcount[lane];
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            wcount[lane] = incl - v;
+            if (lane == 31) total_s = incl;
+        }
+        __syncthreads();
+        if (valid) {
+            const long long k = base + wcount[warp] + __popc(mask & ((1u << lane) - 1u));
+            crow[k] = i;
+            ccol[k] = j;
+            cidx[k] = (int32_t)e;
+        }
+        base += total_s;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) ccount[c] = (int32_t)(base - e0);
+}
+
+cudaError_t launch_compact(schnet_ctx* c)
+{
+    Workspace& w = c->ws;
+    k_compact<<<c->ncta, 1024, 0, c->s>>>(w.row_ptr, w.part, w.erow, w.col, w.pos4, c->box, c->cfg.cutoff, c->cap,
+                                          w.meta, w.crow, w.ccol, w.cidx, w.ccount);
+    c->launches += 1;
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // launchers
 // ---------------------------------------------------------------------------
 static MPArgs make_args(schnet_ctx* c, int layer)
@@ -629,8 +704,10 @@ static MPArgs make_args(schnet_ctx* c, int layer)
     Workspace& w = c->ws;
     MPArgs a;
     a.pos4 = w.pos4;
-    a.erow = w.erow;
-    a.col = w.col;
+    a.crow = w.crow;
+    a.ccol = w.ccol;
+    a.cidx = w.cidx;
+    a.ccount = w.ccount;
     a.row_ptr = w.row_ptr;
     a.part = w.part;
     a.meta = w.meta;

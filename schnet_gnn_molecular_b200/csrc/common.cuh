@@ -78,6 +78,15 @@ __device__ __forceinline__ float3 min_image(float3 v, const Box& b)
     return v;
 }
 
+// Single-precision distance of an edge (minimum image).  Every kernel that
+// decides whether an edge lies inside the cutoff uses this one expression, so
+// the masking, the filter and the force assembly agree edge by edge.
+__device__ __forceinline__ float edge_distance(float4 pi, float4 pj, const Box& b, float3& v)
+{
+    v = min_image(make_float3(pj.x - pi.x, pj.y - pi.y, pj.z - pi.z), b);
+    return sqrtf(v.x * v.x + v.y * v.y + v.z * v.z);
+}
+
 // ---------------------------------------------------------------------------
 // shared-memory / mbarrier / tcgen05 wrappers (sm_100a)
 // ---------------------------------------------------------------------------

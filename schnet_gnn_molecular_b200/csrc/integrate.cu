@@ -34,9 +34,8 @@ __global__ void k_forces(int n, const int32_t* __restrict__ row_ptr, const int32
         const int a = row_ptr[i], b = row_ptr[i + 1];
         for (int e = a + lane; e < b; e += 32) {
             const int j = col[e];
-            const float4 pj = pos4[j];
-            float3 v = min_image(make_float3(pj.x - pi.x, pj.y - pi.y, pj.z - pi.z), box);
-            float d = sqrtf(v.x * v.x + v.y * v.y + v.z * v.z);
+            float3 v;
+            const float d = edge_distance(pi, pos4[j], box, v);
             if (d < rc && d > 0.f) {
                 const int re = rev[e];
                 float D = s_edge[e] + (re >= 0 ? s_edge[re] : 0.f);

@@ -45,6 +45,8 @@ struct Workspace {
     int32_t *row_ptr, *rowcnt;    // [N+1]
     int32_t *col, *coltmp, *rev, *erow;  // [cap]
     float* s_edge;                // [cap]
+    int32_t *crow, *ccol, *cidx;  // [cap] edges with d < r_c, per CTA row range
+    int32_t* ccount;              // [ncta]
     int32_t* part;                // [ncta+1]
     // cell list
     int32_t *cell_of, *cell_atoms;       // [N]
@@ -133,6 +135,7 @@ cudaError_t launch_aw_first(schnet_ctx* c, const int32_t* types);
 cudaError_t launch_aw_fwd(schnet_ctx* c, int layer);
 cudaError_t launch_aw_bwd_top(schnet_ctx* c);
 cudaError_t launch_aw_bwd(schnet_ctx* c, int layer);
+cudaError_t launch_compact(schnet_ctx* c);
 cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer);
 cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s);
 cudaError_t cfconv_init_attributes();

@@ -17,7 +17,7 @@ SOURCES = ["api.cu", "neighbors.cu", "cfconv.cu", "atomwise.cu", "integrate.cu"]
 HEADERS = ["common.cuh", "internal.h", os.path.join("..", "..", "include", "schnet.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-ftz=true",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr", "-Xcompiler", "-fvisibility=hidden"]
 
 

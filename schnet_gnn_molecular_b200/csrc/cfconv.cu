@@ -57,10 +57,12 @@ constexpr uint32_t SM_FWD_A = 131072;                  // fwd: a hi/lo (64 KB)
 constexpr uint32_t SM_BWD_Y = 163840;                  // bwd: ssp'(p) p' hi/lo (64 KB); partial sums after GEMM2
 constexpr uint32_t SM_META_FWD = 196608;
 constexpr uint32_t SM_META_BWD = 229376;
-constexpr uint32_t TILEMETA_BYTES = 2048;
+constexpr uint32_t TILEMETA_BYTES = 2048 + 64;         // per-edge records + per-chunk row summary
 constexpr uint32_t PART_BYTES = 2 * 4 * 128 * 4;       // first/last-row partial per chunk and feature
-constexpr uint32_t SMEM_FWD = SM_META_FWD + TILEMETA_BYTES + PART_BYTES + 16;
+// forward: two metadata buffers (tile t and the next tile are live together)
+constexpr uint32_t SMEM_FWD = SM_META_FWD + 2 * TILEMETA_BYTES + PART_BYTES + 16;
 constexpr uint32_t SMEM_BWD = SM_META_BWD + TILEMETA_BYTES + 16;
+static_assert(SMEM_BWD <= 232448, "backward shared memory exceeds the per-block limit");
 
 constexpr uint32_t RBF_TERM = TILE_E * KP * 2;   // 16 KB: one 16-bit term of a [128 x 64] tile
 constexpr uint32_t ACT_TERM = TILE_E * FP * 2;   // 32 KB: one 16-bit term of a [128 x 128] tile
@@ -72,7 +74,19 @@ struct EdgeMeta {          // one 16-byte record per edge of the tile
     float fc;
     float dfc;
 };
-typedef EdgeMeta TileMeta;
+// Row summary of one 32-edge chunk, written once per tile by warp votes in
+// stage R: first and last row, which edges belong to the first row, and
+// whether any third row occurs (then the general segmented path is taken).
+struct ChunkInfo {
+    int32_t rfirst, rlast;
+    uint32_t firstmask;
+    int32_t other;
+};
+
+struct TileMeta {
+    EdgeMeta e[TILE_E];
+    ChunkInfo c[TILE_E / 32];
+};
 
 __device__ __forceinline__ void copy_weights(uint8_t* smem, const uint8_t* __restrict__ img)
 {
@@ -153,7 +167,7 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
 // image), cutoff mask, Gaussian expansion (and its d-derivative when BWD)
 // written as hi/lo 16-bit K-major B operands.
 template <int FMT, bool BWD>
-__device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMeta* tm, const EdgePre& ep, int ne)
+__device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMeta* tmeta, const EdgePre& ep, int ne)
 {
     const int e = threadIdx.x & (TILE_E - 1);
     const int kq = threadIdx.x >> 7;
@@ -177,10 +191,19 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMe
         m.col = valid ? ep.j : -1;
         m.fc = fc;
         m.dfc = dfc;
-        tm[e] = m;
+        tmeta->e[e] = m;
+        // warp w of this quarter holds edges 32w .. 32w+31: summarise the chunk's rows
+        const int lane = threadIdx.x & 31, w = e >> 5;
+        const int nv = min(max(ne - 32 * w, 0), 32);
+        const int rfirst = __shfl_sync(0xffffffffu, m.row, 0);
+        const int rlast = __shfl_sync(0xffffffffu, m.row, nv > 0 ? nv - 1 : 0);
+        const unsigned fm = __ballot_sync(0xffffffffu, e < ne && m.row == rfirst);
+        const int oth = __any_sync(0xffffffffu, e < ne && m.row != rfirst && m.row != rlast);
+        if (lane == 0) tmeta->c[w] = ChunkInfo{rfirst, rlast, fm, oth};
     }
     uint8_t* b_hi = smem + SM_X;
     uint8_t* b_lo = b_hi + RBF_TERM;
+    (void)tmeta;
     uint8_t* p_hi = smem + SM_X + 2 * RBF_TERM;   // derivative tile (backward)
     uint8_t* p_lo = p_hi + RBF_TERM;
 #pragma unroll
@@ -240,7 +263,7 @@ __device__ __forceinline__ void gather(const float* __restrict__ src, const Tile
 {
 #pragma unroll
     for (int q = 0; q < N; ++q) {
-        const int j = tm[e + q].col;
+        const int j = tm->e[e + q].col;
         dst[q] = j >= 0 ? __ldg(src + (size_t)j * FP + f) : 0.f;
     }
 }
@@ -256,7 +279,7 @@ struct ChunkSeg {
 
 __device__ __forceinline__ void seg_begin(ChunkSeg& c, const TileMeta* tm, int eb)
 {
-    c.rfirst = tm[eb].row;
+    c.rfirst = tm->e[eb].row;
     c.lrow = c.rfirst;
     c.acc = 0.f;
     c.pf = 0.f;
@@ -282,7 +305,8 @@ __device__ __forceinline__ void merge_chunks(const TileMeta* tm, const float* pf
         const int eb = c * 32;
         if (eb >= ne) break;
         const int last = min(eb + 31, ne - 1);
-        const int rfirst = tm[eb].row, rlast = tm[last].row;
+        const int rfirst = tm->c[c].rfirst, rlast = tm->c[c].rlast;
+        (void)last;
         const float v = pf[c * 128 + f];
         if (rfirst == cur) {
             acc += v;
@@ -300,6 +324,90 @@ __device__ __forceinline__ void merge_chunks(const TileMeta* tm, const float* pf
     }
 }
 
+// pairwise sum of N values (fixed order)
+template <int N>
+__device__ __forceinline__ float tree_sum(float (&v)[N])
+{
+#pragma unroll
+    for (int w = N / 2; w >= 1; w >>= 1)
+#pragma unroll
+        for (int q = 0; q < w; ++q) v[q] += v[q + w];
+    return v[0];
+}
+
+// Reduce a chunk's per-edge terms t[q] (edge eb + q) to the first-row and
+// last-row partials.  One or two rows: branch-free predicated sums (edge-less
+// rows strictly between them are written as zeros).  Three or more rows: the
+// serial segmented sum writes the inner rows out.
+template <int N>
+__device__ __forceinline__ void chunk_partials(const TileMeta* tm, int cidx, int eb, int ne, float (&t)[N],
+                                               float* __restrict__ out, int f, float& pf, float& pl)
+{
+    const ChunkInfo ci = tm->c[cidx];
+    if (!ci.other) {
+        if (ci.rfirst == ci.rlast) {
+            pf = tree_sum<N>(t);
+            pl = 0.f;
+        } else {
+            float u[N];
+#pragma unroll
+            for (int q = 0; q < N; ++q) {
+                const bool first = (ci.firstmask >> q) & 1u;
+                u[q] = first ? 0.f : t[q];
+                t[q] = first ? t[q] : 0.f;
+            }
+            pf = tree_sum<N>(t);
+            pl = tree_sum<N>(u);
+            for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) out[(size_t)rr * FP + f] = 0.f;
+        }
+        return;
+    }
+    ChunkSeg c{0, 0, 0.f, 0.f};
+    seg_begin(c, tm, eb);
+#pragma unroll
+    for (int q = 0; q < N; ++q) {
+        const int e = eb + q;
+        if (e >= ne) break;
+        seg_row(c, tm->e[e].row, out, f);
+        c.acc += t[q];
+    }
+    if (c.lrow == c.rfirst) { pf = c.acc; pl = 0.f; } else { pf = c.pf; pl = c.acc; }
+}
+
+// forward epilogue 1 for this warp's 32 edges: a = ssp(s1 P + b1) -> MN-major B operand
+template <int FMT>
+__device__ __forceinline__ void fwd_e1(uint32_t tP, float s1, float b1, uint8_t* smem, int cg, int f)
+{
+    float r[32];
+    tmem_ld32(tP, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < 32; ++q) r[q] = ssp(fmaf(s1, r[q], b1));
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        const uint32_t off = mnmajor_off(cg * 32 + g * 8, f, TILE_E);
+        store8<FMT>(smem + SM_FWD_A, smem + SM_FWD_A + ACT_TERM, off, r + g * 8);
+    }
+}
+
+// forward epilogue 2 for this warp's chunk: W = f_c (s2 Q + b2), terms h_j W, chunk partials
+__device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta* tm, int cg, int ne, float s2, float b2,
+                                       const float (&hv)[32], float* __restrict__ out, int f, float& pf, float& pl)
+{
+    float r[32];
+    tmem_ld32(tQ, r);
+    tmem_ld_wait();
+    const int eb = cg * 32;
+    pf = pl = 0.f;
+    if (eb >= ne) return;
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+        const EdgeMeta m = tm->e[eb + q];   // padding and masked edges have col < 0
+        r[q] = m.col >= 0 ? m.fc * fmaf(s2, r[q], b2) * hv[q] : 0.f;
+    }
+    chunk_partials<32>(tm, cg, eb, ne, r, out, f, pf, pl);
+}
+
 // ---------------------------------------------------------------------------
 // forward: m_i = sum_j h_j (.) W(d_ij)
 // ---------------------------------------------------------------------------
@@ -307,11 +415,11 @@ template <int FMT, int NW>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
-    TileMeta* tm = reinterpret_cast<TileMeta*>(smem + SM_META_FWD);
-    float* pf_s = reinterpret_cast<float*>(smem + SM_META_FWD + TILEMETA_BYTES);
+    auto tmb = [&](int t) { return reinterpret_cast<TileMeta*>(smem + SM_META_FWD + (t & 1) * TILEMETA_BYTES); };
+    float* pf_s = reinterpret_cast<float*>(smem + SM_META_FWD + 2 * TILEMETA_BYTES);
     float* pl_s = pf_s + 4 * 128;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_FWD + TILEMETA_BYTES + PART_BYTES);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_FWD + TILEMETA_BYTES + PART_BYTES + 8);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_FWD + 2 * TILEMETA_BYTES + PART_BYTES);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_FWD + 2 * TILEMETA_BYTES + PART_BYTES + 8);
 
     if (a.meta->n_edges > a.cap) return;
     const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
@@ -346,11 +454,15 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     float acc = 0.f;
     uint32_t phase = 0;
     bool ok = true;
+    const int ntiles = (int)((e1 - e0 + TILE_E - 1) / TILE_E);
+    auto tile_ne = [&](int t) { return (int)min((long long)TILE_E, e1 - e0 - (long long)t * TILE_E); };
 
-    EdgePre ep = prefetch_edge(a, e0, (int)min((long long)TILE_E, e1 - e0));
-    for (long long t0 = e0; t0 < e1 && ok; t0 += TILE_E) {
-        const int ne = (int)min((long long)TILE_E, e1 - t0);
-        stage_rbf<FMT, false>(a, smem, tm, ep, ne);
+    // Software pipeline: tile t's GEMM2 runs while stage R of tile t+1 fills the
+    // Gaussian operand; tile t's epilogue 2 runs while GEMM1 of tile t+1 runs.
+    if (ntiles > 0) {
+        EdgePre ep = prefetch_edge(a, e0, tile_ne(0));
+        stage_rbf<FMT, false>(a, smem, tmb(0), ep, tile_ne(0));
+        if (ntiles > 1) ep = prefetch_edge(a, e0 + TILE_E, tile_ne(1));
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -359,63 +471,59 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
             issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
             mma_commit(bar);
         }
-        if (!(ok = wait_mma(bar, phase, a.meta))) break;
-
-        // epilogue 1: a = ssp(s1 P + b1) for this warp's 32 edges -> MN-major B operand
-        {
-            float r[32];
-            tmem_ld32(tP, r);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 32; ++q) r[q] = ssp(fmaf(s1, r[q], b1));
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                const uint32_t off = mnmajor_off(cg * 32 + g * 8, f, TILE_E);
-                store8<FMT>(smem + SM_FWD_A, smem + SM_FWD_A + ACT_TERM, off, r + g * 8);
+        ok = wait_mma(bar, phase, a.meta);
+        if (ok) {
+            fwd_e1<FMT>(tP, s1, b1, smem, cg, f);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                tc_fence_after();
+                issue_gemm<NW>(tmem + 128, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_FWD_A, ACT_TERM, FP / 16,
+                               id_mn);
+                mma_commit(bar);
             }
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            tc_fence_after();
-            issue_gemm<NW>(tmem + 128, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_FWD_A, ACT_TERM, FP / 16,
-                           id_mn);
-            mma_commit(bar);
-        }
-        // this chunk's h_j rows are fetched while GEMM2 runs
-        const int eb = cg * 32;
-        float hv[32];
-        gather<32>(a.h, tm, eb, f, hv);
-        if (!(ok = wait_mma(bar, phase, a.meta))) break;
-        if (t0 + TILE_E < e1) ep = prefetch_edge(a, t0 + TILE_E, (int)min((long long)TILE_E, e1 - t0 - TILE_E));
-
-        // epilogue 2: W = f_c (s2 Q + b2); segmented sum of h_j (.) W over this chunk
-        {
-            float r[32];
-            tmem_ld32(tQ, r);
-            tmem_ld_wait();
-            float pf = 0.f, pl = 0.f;
-            if (eb < ne) {
-                ChunkSeg c{0, 0, 0.f, 0.f};
-                seg_begin(c, tm, eb);
-#pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int e = eb + q;
-                    if (e >= ne) break;
-                    const EdgeMeta m = tm[e];
-                    seg_row(c, m.row, a.out, f);
-                    if (m.col >= 0) c.acc = fmaf(m.fc * fmaf(s2, r[q], b2), hv[q], c.acc);
-                }
-                if (c.lrow == c.rfirst) pf = c.acc; else { pf = c.pf; pl = c.acc; }
+        for (int t = 0; t < ntiles && ok; ++t) {
+            const int ne = tile_ne(t);
+            const bool next = t + 1 < ntiles;
+            TileMeta* tm = tmb(t);
+            // (GEMM2 of tile t in flight) Gaussians of the next tile, then this chunk's h_j rows
+            if (next) {
+                stage_rbf<FMT, false>(a, smem, tmb(t + 1), ep, tile_ne(t + 1));
+                fence_proxy_async_smem();
+                if (t + 2 < ntiles) ep = prefetch_edge(a, e0 + (long long)(t + 2) * TILE_E, tile_ne(t + 2));
             }
+            float hv[32];
+            gather<32>(a.h, tm, cg * 32, f, hv);
+            if (!(ok = wait_mma(bar, phase, a.meta))) break;      // GEMM2(t) done; next tile's operand ready
+            if (next && threadIdx.x == 0) {
+                issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
+                mma_commit(bar);
+            }
+            // (GEMM1 of tile t+1 in flight) epilogue 2 and the in-order merge of tile t
+            float pf, pl;
+            fwd_e2(tQ, tm, cg, ne, s2, b2, hv, a.out, f, pf, pl);
             pf_s[cg * 128 + f] = pf;
             pl_s[cg * 128 + f] = pl;
+            __syncthreads();
+            if (threadIdx.x < 128) merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
+            if (next) {
+                if (!(ok = wait_mma(bar, phase, a.meta))) break;  // GEMM1(t+1) done
+                fwd_e1<FMT>(tP, s1, b1, smem, cg, f);
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                if (threadIdx.x == 0) {
+                    tc_fence_after();
+                    issue_gemm<NW>(tmem + 128, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_FWD_A, ACT_TERM,
+                                   FP / 16, id_mn);
+                    mma_commit(bar);
+                }
+            } else {
+                __syncthreads();
+            }
         }
-        __syncthreads();
-        if (threadIdx.x < 128) merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
-        tc_fence_before();
-        __syncthreads();   // tile metadata, partials and operand tiles are rewritten next
     }
 
     if (ok) {
@@ -442,7 +550,7 @@ template <int FMT, int NW>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
-    TileMeta* tm = reinterpret_cast<TileMeta*>(smem + SM_META_BWD);
+    TileMeta* tm = reinterpret_cast<TileMeta*>(smem + SM_META_BWD);   // single buffer
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_BWD + TILEMETA_BYTES);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_BWD + TILEMETA_BYTES + 8);
     // after GEMM2 the ssp'(p)p' tile is dead: its space holds the partial sums
@@ -542,10 +650,16 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 
         // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 Q + b2, z' = s2 Q')
         {
-            ChunkSeg c{0, 0, 0.f, 0.f};
             const bool active = eb < ne;
-            if (active) seg_begin(c, tm, eb);
-            float u_row = active ? __ldg(a.u + (size_t)c.rfirst * FP + f) : 0.f;
+            const ChunkInfo ci = tm->c[cg];
+            // one or two rows in the chunk (the usual case): predicated first/last-row sums;
+            // otherwise the serial segmented sum with a row change test per edge
+            const float u_first = active ? __ldg(a.u + (size_t)ci.rfirst * FP + f) : 0.f;
+            const float u_last = active ? __ldg(a.u + (size_t)ci.rlast * FP + f) : 0.f;
+            float sf = 0.f, sl = 0.f;
+            ChunkSeg c{0, 0, 0.f, 0.f};
+            if (active && ci.other) seg_begin(c, tm, eb);
+            float u_row = u_first;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 if (hh == 1) {
@@ -556,25 +670,43 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                 tmem_ld16(tQ + hh * 16, r);
                 tmem_ld16(tQd + hh * 16, rd);
                 tmem_ld_wait();
+                if (!ci.other) {
 #pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const int e = eb + hh * 16 + q;
-                    float tval = 0.f;
-                    if (e < ne) {
-                        const EdgeMeta m = tm[e];
-                        if (m.row != c.lrow) {
-                            seg_row(c, m.row, a.out, f);
-                            u_row = __ldg(a.u + (size_t)m.row * FP + f);
-                        }
+                    for (int q = 0; q < 16; ++q) {
+                        const int qq = hh * 16 + q;
+                        const EdgeMeta m = tm->e[eb + qq];
+                        float tval = 0.f;
                         if (m.col >= 0) {
                             const float z = fmaf(s2, r[q], b2);
-                            const float fcv = m.fc;
-                            const float wd = fmaf(m.dfc, z, fcv * s2 * rd[q]);
-                            c.acc = fmaf(fcv * z, uv[q], c.acc);
-                            tval = wd * u_row * hv[q];
+                            const float wd = fmaf(m.dfc, z, m.fc * s2 * rd[q]);
+                            const bool first = (ci.firstmask >> qq) & 1u;
+                            const float dt = m.fc * z * uv[q];
+                            sf += first ? dt : 0.f;
+                            sl += first ? 0.f : dt;
+                            tval = wd * (first ? u_first : u_last) * hv[q];
                         }
+                        rd[q] = tval;
                     }
-                    rd[q] = tval;
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int e = eb + hh * 16 + q;
+                        float tval = 0.f;
+                        if (e < ne) {
+                            const EdgeMeta m = tm->e[e];
+                            if (m.row != c.lrow) {
+                                seg_row(c, m.row, a.out, f);
+                                u_row = __ldg(a.u + (size_t)m.row * FP + f);
+                            }
+                            if (m.col >= 0) {
+                                const float z = fmaf(s2, r[q], b2);
+                                const float wd = fmaf(m.dfc, z, m.fc * s2 * rd[q]);
+                                c.acc = fmaf(m.fc * z, uv[q], c.acc);
+                                tval = wd * u_row * hv[q];
+                            }
+                        }
+                        rd[q] = tval;
+                    }
                 }
                 // transpose-reduce the 16 per-edge values over the warp's 32 features:
                 // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
@@ -593,7 +725,20 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             }
             float pf = 0.f, pl = 0.f;
             if (active) {
-                if (c.lrow == c.rfirst) pf = c.acc; else { pf = c.pf; pl = c.acc; }
+                if (!ci.other) {
+                    if (ci.rfirst == ci.rlast) {
+                        pf = sf + sl;
+                    } else {
+                        pf = sf;
+                        pl = sl;
+                        for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
+                    }
+                } else if (c.lrow == c.rfirst) {
+                    pf = c.acc;
+                } else {
+                    pf = c.pf;
+                    pl = c.acc;
+                }
             }
             pf_s[cg * 128 + f] = pf;
             pl_s[cg * 128 + f] = pl;

@@ -145,20 +145,29 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
 struct EdgePre {
     int i, j;
     float4 pi, pj;
+    int gidx;      // backward: index of the edge in the full list (where s_e is stored)
+    float sold;    // backward: s_e accumulated by the later interactions so far
 };
 
+template <bool BWD = false>
 __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, int ne)
 {
     EdgePre p;
     p.i = 0;
     p.j = -1;
     p.pi = p.pj = make_float4(0.f, 0.f, 0.f, 0.f);
+    p.gidx = 0;
+    p.sold = 0.f;
     const int t = threadIdx.x & (TILE_E - 1);
     if (t < ne) {
         p.i = __ldg(a.crow + e0 + t);
         p.j = __ldg(a.ccol + e0 + t);
         p.pi = __ldg(a.pos4 + p.i);
         p.pj = __ldg(a.pos4 + p.j);
+        if (BWD && threadIdx.x < TILE_E) {
+            p.gidx = __ldg(a.cidx + e0 + t);
+            if (a.accumulate_s) p.sold = a.s_edge[p.gidx];
+        }
     }
     return p;
 }
@@ -546,17 +555,46 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 // ---------------------------------------------------------------------------
 // backward: dh_i = sum_j u_j (.) W_ij ;  s_e = sum_f W'_e,f u_i,f h_j,f
 // ---------------------------------------------------------------------------
+// backward epilogue 1 for this warp's 32 edges: a = ssp(p), b = ssp'(p) p'  (p = s1 P + b1, p' = s1 P')
+template <int FMT>
+__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1, float b1, uint8_t* smem, uint32_t col0,
+                                       int f)
+{
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        float r[16], rd[16];
+        tmem_ld16(tP + hh * 16, r);
+        tmem_ld16(tPd + hh * 16, rd);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            float sv, gv;
+            ssp_and_grad(fmaf(s1, r[q], b1), sv, gv);
+            r[q] = sv;
+            rd[q] = gv * s1 * rd[q];
+        }
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            const uint32_t off = mnmajor_off(col0 + hh * 16 + g * 8, f, TILE_E);
+            store8<FMT>(smem + SM_X, smem + SM_X + ACT_TERM, off, r + g * 8);
+            store8<FMT>(smem + SM_BWD_Y, smem + SM_BWD_Y + ACT_TERM, off, rd + g * 8);
+        }
+    }
+}
+
 template <int FMT, int NW>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
-    TileMeta* tm = reinterpret_cast<TileMeta*>(smem + SM_META_BWD);   // single buffer
+    TileMeta* tm = reinterpret_cast<TileMeta*>(smem + SM_META_BWD);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_BWD + TILEMETA_BYTES);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_BWD + TILEMETA_BYTES + 8);
-    // after GEMM2 the ssp'(p)p' tile is dead: its space holds the partial sums
+    // after GEMM2 the ssp'(p)p' tile is dead: its space holds the partial sums and,
+    // behind them, the next tile's metadata until the merge has finished with tm
     float* pf_s = reinterpret_cast<float*>(smem + SM_BWD_Y);
     float* pl_s = pf_s + 4 * 128;
     float* ps_s = pl_s + 4 * 128;   // [quadrant][edge] per-edge partial of s_e
+    TileMeta* tm_next = reinterpret_cast<TileMeta*>(smem + SM_BWD_Y + 8192);
 
     if (a.meta->n_edges > a.cap) return;
     const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
@@ -593,11 +631,18 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     float acc = 0.f;
     uint32_t phase = 0;
     bool ok = true;
+    const int ntiles = (int)((e1 - e0 + TILE_E - 1) / TILE_E);
+    auto tile_ne = [&](int t) { return (int)min((long long)TILE_E, e1 - e0 - (long long)t * TILE_E); };
+    int cur_g = 0, nxt_g = 0;           // threads < 128: s_e slot of edge threadIdx.x (this / next tile)
+    float cur_so = 0.f, nxt_so = 0.f;
 
-    EdgePre ep = prefetch_edge(a, e0, (int)min((long long)TILE_E, e1 - e0));
-    for (long long t0 = e0; t0 < e1 && ok; t0 += TILE_E) {
-        const int ne = (int)min((long long)TILE_E, e1 - t0);
-        stage_rbf<FMT, true>(a, smem, tm, ep, ne);
+    // Software pipeline: epilogue 2 of tile t runs while GEMM1 of tile t+1 runs.
+    if (ntiles > 0) {
+        EdgePre ep = prefetch_edge<true>(a, e0, tile_ne(0));
+        stage_rbf<FMT, true>(a, smem, tm, ep, tile_ne(0));
+        cur_g = ep.gidx;
+        cur_so = ep.sold;
+        if (ntiles > 1) ep = prefetch_edge<true>(a, e0 + TILE_E, tile_ne(1));
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -608,153 +653,173 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                            KP / 16, id);
             mma_commit(bar);
         }
-        if (!(ok = wait_mma(bar, phase, a.meta))) break;
-
-        // epilogue 1: a = ssp(p), b = ssp'(p) p'   (p = s1 P + b1, p' = s1 P'), 16 edges at a time
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float r[16], rd[16];
-            tmem_ld16(tP + hh * 16, r);
-            tmem_ld16(tPd + hh * 16, rd);
-            tmem_ld_wait();
-#pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                float sv, gv;
-                ssp_and_grad(fmaf(s1, r[q], b1), sv, gv);
-                r[q] = sv;
-                rd[q] = gv * s1 * rd[q];
-            }
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                const uint32_t off = mnmajor_off(col0 + hh * 16 + g * 8, f, TILE_E);
-                store8<FMT>(smem + SM_X, smem + SM_X + ACT_TERM, off, r + g * 8);
-                store8<FMT>(smem + SM_BWD_Y, smem + SM_BWD_Y + ACT_TERM, off, rd + g * 8);
+        ok = wait_mma(bar, phase, a.meta);
+        if (ok) {
+            bwd_e1<FMT>(tP, tPd, s1, b1, smem, col0, f);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                tc_fence_after();
+                issue_gemm<NW>(tmem + 256, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_X, ACT_TERM, FP / 16, id_mn);
+                issue_gemm<NW>(tmem + 384, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_BWD_Y, ACT_TERM, FP / 16,
+                               id_mn);
+                mma_commit(bar);
             }
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            tc_fence_after();
-            issue_gemm<NW>(tmem + 256, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_X, ACT_TERM, FP / 16, id_mn);
-            issue_gemm<NW>(tmem + 384, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_BWD_Y, ACT_TERM, FP / 16,
-                           id_mn);
-            mma_commit(bar);
-        }
-        const int eb = (int)col0;
-        float uv[16], hv[16];
-        gather<16>(a.u, tm, eb, f, uv);
-        gather<16>(a.h, tm, eb, f, hv);
-        if (!(ok = wait_mma(bar, phase, a.meta))) break;
-        if (t0 + TILE_E < e1) ep = prefetch_edge(a, t0 + TILE_E, (int)min((long long)TILE_E, e1 - t0 - TILE_E));
-
-        // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 Q + b2, z' = s2 Q')
-        {
-            const bool active = eb < ne;
-            const ChunkInfo ci = tm->c[cg];
-            // one or two rows in the chunk (the usual case): predicated first/last-row sums;
-            // otherwise the serial segmented sum with a row change test per edge
-            const float u_first = active ? __ldg(a.u + (size_t)ci.rfirst * FP + f) : 0.f;
-            const float u_last = active ? __ldg(a.u + (size_t)ci.rlast * FP + f) : 0.f;
-            float sf = 0.f, sl = 0.f;
-            ChunkSeg c{0, 0, 0.f, 0.f};
-            if (active && ci.other) seg_begin(c, tm, eb);
-            float u_row = u_first;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                if (hh == 1) {
-                    gather<16>(a.u, tm, eb + 16, f, uv);
-                    gather<16>(a.h, tm, eb + 16, f, hv);
+        for (int t = 0; t < ntiles && ok; ++t) {
+            const int ne = tile_ne(t);
+            const bool next = t + 1 < ntiles;
+            const long long t0 = e0 + (long long)t * TILE_E;
+            const int eb = (int)col0;
+            float uv[16], hv[16];
+            gather<16>(a.u, tm, eb, f, uv);
+            gather<16>(a.h, tm, eb, f, hv);
+            if (!(ok = wait_mma(bar, phase, a.meta))) break;            // GEMM2(t) done
+            if (next) {
+                // Gaussians of the next tile into the (now dead) ssp(p) region; its metadata is staged
+                stage_rbf<FMT, true>(a, smem, tm_next, ep, tile_ne(t + 1));
+                nxt_g = ep.gidx;
+                nxt_so = ep.sold;
+                if (t + 2 < ntiles) ep = prefetch_edge<true>(a, e0 + (long long)(t + 2) * TILE_E, tile_ne(t + 2));
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                if (threadIdx.x == 0) {
+                    tc_fence_after();
+                    issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
+                    issue_gemm<NW>(tmem + 128, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X + 2 * RBF_TERM,
+                                   RBF_TERM, KP / 16, id);
+                    mma_commit(bar);
                 }
-                float r[16], rd[16];
-                tmem_ld16(tQ + hh * 16, r);
-                tmem_ld16(tQd + hh * 16, rd);
-                tmem_ld_wait();
-                if (!ci.other) {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int qq = hh * 16 + q;
-                        const EdgeMeta m = tm->e[eb + qq];
-                        float tval = 0.f;
-                        if (m.col >= 0) {
-                            const float z = fmaf(s2, r[q], b2);
-                            const float wd = fmaf(m.dfc, z, m.fc * s2 * rd[q]);
-                            const bool first = (ci.firstmask >> qq) & 1u;
-                            const float dt = m.fc * z * uv[q];
-                            sf += first ? dt : 0.f;
-                            sl += first ? 0.f : dt;
-                            tval = wd * (first ? u_first : u_last) * hv[q];
-                        }
-                        rd[q] = tval;
+            }
+            // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 Q + b2, z' = s2 Q')
+            {
+                const bool active = eb < ne;
+                const ChunkInfo ci = tm->c[cg];
+                // one or two rows in the chunk (the usual case): predicated first/last-row sums;
+                // otherwise the serial segmented sum with a row change test per edge
+                const float u_first = active ? __ldg(a.u + (size_t)ci.rfirst * FP + f) : 0.f;
+                const float u_last = active ? __ldg(a.u + (size_t)ci.rlast * FP + f) : 0.f;
+                float sf = 0.f, sl = 0.f;
+                ChunkSeg c{0, 0, 0.f, 0.f};
+                if (active && ci.other) seg_begin(c, tm, eb);
+                float u_row = u_first;
+    #pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    if (hh == 1) {
+                        gather<16>(a.u, tm, eb + 16, f, uv);
+                        gather<16>(a.h, tm, eb + 16, f, hv);
                     }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int e = eb + hh * 16 + q;
-                        float tval = 0.f;
-                        if (e < ne) {
-                            const EdgeMeta m = tm->e[e];
-                            if (m.row != c.lrow) {
-                                seg_row(c, m.row, a.out, f);
-                                u_row = __ldg(a.u + (size_t)m.row * FP + f);
-                            }
+                    float r[16], rd[16];
+                    tmem_ld16(tQ + hh * 16, r);
+                    tmem_ld16(tQd + hh * 16, rd);
+                    tmem_ld_wait();
+                    if (!ci.other) {
+    #pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const int qq = hh * 16 + q;
+                            const EdgeMeta m = tm->e[eb + qq];
+                            float tval = 0.f;
                             if (m.col >= 0) {
                                 const float z = fmaf(s2, r[q], b2);
                                 const float wd = fmaf(m.dfc, z, m.fc * s2 * rd[q]);
-                                c.acc = fmaf(m.fc * z, uv[q], c.acc);
-                                tval = wd * u_row * hv[q];
+                                const bool first = (ci.firstmask >> qq) & 1u;
+                                const float dt = m.fc * z * uv[q];
+                                sf += first ? dt : 0.f;
+                                sl += first ? 0.f : dt;
+                                tval = wd * (first ? u_first : u_last) * hv[q];
                             }
+                            rd[q] = tval;
                         }
-                        rd[q] = tval;
-                    }
-                }
-                // transpose-reduce the 16 per-edge values over the warp's 32 features:
-                // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
-#pragma unroll
-                for (int sh = 16; sh >= 2; sh >>= 1) {
-                    const bool upper = (lane & sh) != 0;
-#pragma unroll
-                    for (int k = 0; k < sh / 2; ++k) {
-                        float send = upper ? rd[k] : rd[k + sh / 2];
-                        float keep = upper ? rd[k + sh / 2] : rd[k];
-                        rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
-                    }
-                }
-                rd[0] += __shfl_xor_sync(0xffffffffu, rd[0], 1);
-                if ((lane & 1) == 0) ps_s[qd * TILE_E + eb + hh * 16 + (lane >> 1)] = rd[0];
-            }
-            float pf = 0.f, pl = 0.f;
-            if (active) {
-                if (!ci.other) {
-                    if (ci.rfirst == ci.rlast) {
-                        pf = sf + sl;
                     } else {
-                        pf = sf;
-                        pl = sl;
-                        for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
+    #pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const int e = eb + hh * 16 + q;
+                            float tval = 0.f;
+                            if (e < ne) {
+                                const EdgeMeta m = tm->e[e];
+                                if (m.row != c.lrow) {
+                                    seg_row(c, m.row, a.out, f);
+                                    u_row = __ldg(a.u + (size_t)m.row * FP + f);
+                                }
+                                if (m.col >= 0) {
+                                    const float z = fmaf(s2, r[q], b2);
+                                    const float wd = fmaf(m.dfc, z, m.fc * s2 * rd[q]);
+                                    c.acc = fmaf(m.fc * z, uv[q], c.acc);
+                                    tval = wd * u_row * hv[q];
+                                }
+                            }
+                            rd[q] = tval;
+                        }
                     }
-                } else if (c.lrow == c.rfirst) {
-                    pf = c.acc;
-                } else {
-                    pf = c.pf;
-                    pl = c.acc;
+                    // transpose-reduce the 16 per-edge values over the warp's 32 features:
+                    // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
+    #pragma unroll
+                    for (int sh = 16; sh >= 2; sh >>= 1) {
+                        const bool upper = (lane & sh) != 0;
+    #pragma unroll
+                        for (int k = 0; k < sh / 2; ++k) {
+                            float send = upper ? rd[k] : rd[k + sh / 2];
+                            float keep = upper ? rd[k + sh / 2] : rd[k];
+                            rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+                        }
+                    }
+                    rd[0] += __shfl_xor_sync(0xffffffffu, rd[0], 1);
+                    if ((lane & 1) == 0) ps_s[qd * TILE_E + eb + hh * 16 + (lane >> 1)] = rd[0];
+                }
+                float pf = 0.f, pl = 0.f;
+                if (active) {
+                    if (!ci.other) {
+                        if (ci.rfirst == ci.rlast) {
+                            pf = sf + sl;
+                        } else {
+                            pf = sf;
+                            pl = sl;
+                            for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
+                        }
+                    } else if (c.lrow == c.rfirst) {
+                        pf = c.acc;
+                    } else {
+                        pf = c.pf;
+                        pl = c.acc;
+                    }
+                }
+                pf_s[cg * 128 + f] = pf;
+                pl_s[cg * 128 + f] = pl;
+            }
+            __syncthreads();
+            if (threadIdx.x < 128) {
+                merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
+                if ((int)threadIdx.x < ne) {
+                    const int q = threadIdx.x;
+                    const float sv = ps_s[q] + ps_s[TILE_E + q] + ps_s[2 * TILE_E + q] + ps_s[3 * TILE_E + q];
+                    a.s_edge[cur_g] = a.accumulate_s ? cur_so + sv : sv;
                 }
             }
-            pf_s[cg * 128 + f] = pf;
-            pl_s[cg * 128 + f] = pl;
-        }
-        __syncthreads();
-        if (threadIdx.x < 128) {
-            merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
-            const int t = threadIdx.x;
-            if (t < ne) {
-                const float sv = ps_s[t] + ps_s[TILE_E + t] + ps_s[2 * TILE_E + t] + ps_s[3 * TILE_E + t];
-                float* dst = a.s_edge + a.cidx[t0 + t];
-                *dst = a.accumulate_s ? *dst + sv : sv;
+            if (next) {
+                __syncthreads();                                        // merge done with tm
+                for (int i = threadIdx.x; i < (int)(sizeof(TileMeta) / 4); i += NT)
+                    reinterpret_cast<uint32_t*>(tm)[i] = reinterpret_cast<const uint32_t*>(tm_next)[i];
+                cur_g = nxt_g;
+                cur_so = nxt_so;
+                if (!(ok = wait_mma(bar, phase, a.meta))) break;        // GEMM1(t+1) done
+                bwd_e1<FMT>(tP, tPd, s1, b1, smem, col0, f);
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                if (threadIdx.x == 0) {
+                    tc_fence_after();
+                    issue_gemm<NW>(tmem + 256, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_X, ACT_TERM, FP / 16,
+                                   id_mn);
+                    issue_gemm<NW>(tmem + 384, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_BWD_Y, ACT_TERM, FP / 16,
+                                   id_mn);
+                    mma_commit(bar);
+                }
+            } else {
+                __syncthreads();
             }
         }
-        tc_fence_before();
-        __syncthreads();
     }
 
     if (ok) {

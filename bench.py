@@ -92,6 +92,20 @@ def _dist():
     return ws, rank, local
 
 
+def aggregate_ranks(ms_local: float, atoms_local: int, steps: int, dist=None, device=None):
+    """Whole-job timing over ranks: the slowest rank's device time and the atoms
+    advanced by all ranks.  Returns (max_ms, total_atoms, atom_steps_per_s)."""
+    import torch
+    ms, atoms = float(ms_local), int(atoms_local)
+    if dist is not None and dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        a = torch.tensor([atoms], dtype=torch.int64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(a, op=dist.ReduceOp.SUM)
+        ms, atoms = float(t.item()), int(a.item())
+    return ms, atoms, atoms * steps / (ms * 1e-3)
+
+
 def _workload(name):
     from schnet_gnn_molecular_b200 import workloads
     if name in workloads.ALL:
@@ -225,14 +239,13 @@ def run_native(args):
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
     launches = model.kernel_launches() - l0
+    free_b, total_b = torch.cuda.mem_get_info(dev)
+    memory = {"workspace_MB": round(model.workspace_bytes / 1e6, 1),
+              "torch_peak_allocated_MB": round(torch.cuda.max_memory_allocated(dev) / 1e6, 1),
+              "device_used_MB": round((total_b - free_b) / 1e6, 1),
+              "note": "device_used includes the CUDA context, the library image and the captured graphs"}
     clk = clocks.stop() if clocks else None
-    t_max = ms
-    if ws > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
-    atoms_total = w.n_atoms * ws
-    value = atoms_total * steps / (t_max * 1e-3)
+    t_max, atoms_total, value = aggregate_ranks(ms, w.n_atoms, steps, dist, dev)
     step_s = t_max * 1e-3 / steps
     ns_day_rep = (1.0 / step_s) * w.dt_fs * 86400 * 1e-6
 
@@ -278,6 +291,7 @@ def run_native(args):
                "ns_per_day_per_replica": round(ns_day_rep, 2),
                "ns_per_day_aggregate": round(ns_day_rep * w.n_replicas * ws, 1),
                "config": cfg, "gpu_launches": int(launches), "clocks": clk, "roofline": roofline,
+               "memory": memory,
                "status": {"warmup": nat_status(flagged[0]), "timed": nat_status(flagged[1])}}
         if not args.no_e2e:
             out["e2e"] = e2e(model, w, pos, vel, types, mass, kw, args)
@@ -314,6 +328,52 @@ def e2e(model, w, pos, vel, types, mass, kw, args):
     return {"value": round(w.n_atoms * n / dt, 1), "unit": "atom-steps/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": n,
             "how": "schnet_step_host, one step per call, pinned host buffers, wall clock"}
+
+
+def run_drift(args):
+    """NVE drift: velocity Verlet (gamma = 0) on the workload for --drift-steps steps;
+    total energy (potential + kinetic, summed over replicas) read after every rebuild
+    interval; reported as the least-squares slope per atom."""
+    import torch
+    from schnet_gnn_molecular_b200 import api
+    w = _workload(args.workload).with_(gamma_per_ps=0.0)
+    pos, types, weights, mass, vel = _inputs(w, 0)
+    dev = torch.device("cuda:0")
+    model = api.from_workload(w, weights, device="cuda:0", edge_capacity=args.edge_capacity)
+    p, v = torch.tensor(pos, device=dev), torch.tensor(vel, device=dev)
+    t, m = torch.tensor(types, device=dev), torch.tensor(mass, device=dev)
+    kw = dict(dt=w.dt_fs, gamma=0.0, temperature=w.temperature, n_rebuild=w.n_rebuild, seed=1234)
+    chunk = w.n_rebuild
+    n_chunks = max(1, args.drift_steps // chunk)
+    ep, _, st = model.step(p, v, t, m, 0, step0=0, raise_on_flag=False, **kw)   # initial forces
+    ek0 = 0.5 * float((mass.astype(np.float64)[:, None] * vel.astype(np.float64) ** 2).sum()) / ACC
+    times, etot, flags = [0.0], [float(ep.sum()) + ek0], int(st)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for c in range(n_chunks):
+        ep, ek, st = model.step(p, v, t, m, chunk, step0=c * chunk, resume=c > 0, raise_on_flag=False, **kw)
+        flags |= int(st)
+        times.append((c + 1) * chunk * w.dt_fs * 1e-6)          # ns
+        etot.append(float((ep + ek).sum()))
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    tt, ee = np.array(times), np.array(etot) / w.n_atoms
+    slope, icpt = np.polyfit(tt, ee, 1)
+    resid = ee - (slope * tt + icpt)
+    kcal_to_uev = 4.3364e4                   # 1 kcal/mol = 43.364 meV
+    ekin0 = float(ek.sum()) / w.n_atoms
+    out = {"metric": "NVE energy drift (velocity Verlet)", "value": float(slope), "unit": "kcal/mol/atom/ns",
+           "ueV_per_atom_per_ps": float(slope) * kcal_to_uev / 1e3, "steps": n_chunks * chunk,
+           "dt_fs": w.dt_fs, "simulated_ns": float(tt[-1]), "higher_is_better": False,
+           "etot_per_atom_first_last": [float(ee[0]), float(ee[-1])],
+           "etot_per_atom_rms_about_fit": float(np.sqrt((resid ** 2).mean())),
+           "ekin_per_atom_last": ekin0, "status": nat_status(flags),
+           "ms_per_step": round(ms / (n_chunks * chunk), 4),
+           "config": {"workload": w.name, "replicas": w.n_replicas, "atoms": w.n_atoms, "n_rebuild": w.n_rebuild,
+                      "skin_A": w.skin, "read_every_steps": chunk}, "data": "synthetic"}
+    model.close()
+    print(json.dumps(out), flush=True)
 
 
 def run_reference(args):
@@ -381,10 +441,14 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=150.0, help="seconds for the reference arm's timed steps")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nve-drift", action="store_true", help="measure NVE energy drift instead of throughput")
+    ap.add_argument("--drift-steps", type=int, default=10000)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.nve_drift:
+        run_drift(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_native(args)

@@ -151,3 +151,13 @@ def schnet_weights(rng: np.random.Generator, n_types: int, F: int, K: int, L: in
 def standard_normals(n: int, rng: np.random.Generator) -> np.ndarray:
     """Raw N(0,1) deviates [n,3] (callers scale them into velocities)."""
     return rng.normal(size=(n, 3))
+
+
+def random_rotation(rng: np.random.Generator) -> np.ndarray:
+    """Uniformly distributed 3x3 rotation matrix (QR of a Gaussian matrix with the
+    sign convention that makes the factorisation unique, then det fixed to +1)."""
+    q, r = np.linalg.qr(rng.normal(size=(3, 3)))
+    q = q * np.sign(np.diag(r))
+    if np.linalg.det(q) < 0:
+        q[:, 0] = -q[:, 0]
+    return q

@@ -46,6 +46,7 @@ class Workload:
     radius: float | None = None  # confinement radius for compact chains
     rg_target: float = 12.0
     mass: float = 72.0         # amu per bead (MARTINI-style bead, see the mass reading)
+    pool: int = 0              # >0: replicas r >= pool are random rotations of replica r % pool
 
     @property
     def n_atoms(self) -> int:
@@ -70,7 +71,9 @@ PROTEIN64_BF16 = PROTEIN64.with_(name="cg_protein_64x269_bf16w", weight_dtype="b
 
 
 def sweep(n_replicas: int) -> Workload:
-    return PROTEIN64.with_(name=f"cg_protein_{n_replicas}x269", n_replicas=n_replicas, seed=3000)
+    """Replica-count sweep: 64 independently drawn chains, the rest rotated copies
+    (same per-replica work; drawing 1024 chains would take minutes)."""
+    return PROTEIN64.with_(name=f"cg_protein_{n_replicas}x269", n_replicas=n_replicas, seed=3000, pool=64)
 
 
 def globule(beads: int) -> Workload:
@@ -93,6 +96,11 @@ ALL = {w.name: w for w in [TINY, PROTEIN64, PROTEIN64_FP16, PROTEIN64_BF16, BOX1
 def _positions(w: Workload) -> np.ndarray:
     out = np.zeros((w.n_atoms, 3))
     for r in range(w.n_replicas):
+        if w.pool and r >= w.pool:
+            base = out[(r % w.pool) * w.beads:(r % w.pool + 1) * w.beads]
+            rot = inputs.random_rotation(np.random.default_rng(w.seed + r))
+            out[r * w.beads:(r + 1) * w.beads] = base @ rot.T
+            continue
         rng = np.random.default_rng(w.seed + r)
         if w.geometry == "chain":
             p = inputs.chain(w.beads, rng)

@@ -30,11 +30,25 @@ def _unit_vectors(rng: np.random.Generator, m: int) -> np.ndarray:
 
 def chain(n: int, rng: np.random.Generator, bond: float = 3.8, min_dist: float = 3.0,
           confine_radius: float | None = None, batch: int = 64) -> np.ndarray:
-    """Self-avoiding random walk of n beads (float64 [n,3]); optional confinement."""
+    """Self-avoiding random walk of n beads (float64 [n,3]); optional confinement.
+
+    The clash test of a candidate against beads 0..t-2 only visits beads in grid
+    cells (edge min_dist) near bead t-1; beads outside are farther than min_dist
+    from every candidate, so the accepted walk is the same as an all-pairs test."""
     pos = np.zeros((n, 3))
     if n == 0:
         return pos
     md2 = min_dist * min_dist
+    cell = min_dist
+    grid: dict = {}
+
+    def add(k):
+        key = tuple(np.floor(pos[k] / cell).astype(np.int64))
+        grid.setdefault(key, []).append(k)
+
+    reach = int(math.ceil((bond + min_dist) / cell)) + 1
+    offs = np.arange(-reach, reach + 1)
+    add(0)
     t = 1
     stuck = 0
     while t < n:
@@ -43,11 +57,22 @@ def chain(n: int, rng: np.random.Generator, bond: float = 3.8, min_dist: float =
         if confine_radius is not None:
             ok &= (cand * cand).sum(1) <= confine_radius * confine_radius
         if t > 1:
-            d2 = ((cand[:, None, :] - pos[None, :t - 1, :]) ** 2).sum(-1)
-            ok &= (d2 >= md2).all(1)
-        idx = np.flatnonzero(ok)
-        if idx.size:
-            pos[t] = cand[idx[0]]
+            c0 = np.floor(pos[t - 1] / cell).astype(np.int64)
+            near = []
+            for dx in offs:
+                for dy in offs:
+                    for dz in offs:
+                        near.extend(grid.get((c0[0] + dx, c0[1] + dy, c0[2] + dz), ()))
+            if near:
+                idx = np.unique(np.asarray(near, dtype=np.int64))
+                idx = idx[idx < t - 1]
+                if idx.size:
+                    d2 = ((cand[:, None, :] - pos[None, idx, :]) ** 2).sum(-1)
+                    ok &= (d2 >= md2).all(1)
+        acc = np.flatnonzero(ok)
+        if acc.size:
+            pos[t] = cand[acc[0]]
+            add(t)
             t += 1
             stuck = 0
         else:

@@ -106,9 +106,12 @@ def test_sixteen_bit_filter_weights(dtype):
     x64 = pos.astype(np.float64)
     ro = w.replica_offsets()
     Eq, eps_q, Fq = oracle.energy_forces(oracle_model(w, weights, dequant=dtype), x64, types, ro)
+    E32, eps32, F32 = oracle.energy_forces(oracle_model(w, weights), x64, types, w.replica_offsets())
+    print(f"[errors {dtype}] energy vs dequantized {energy_rel(E, Eq, eps_q, ro):.3e}, forces vs dequantized "
+          f"{rel_frobenius(F, Fq):.3e}, energy vs fp32 weights {energy_rel(E, E32, eps32, ro):.3e}, forces vs "
+          f"fp32 weights {rel_frobenius(F, F32):.3e}")
     assert energy_rel(E, Eq, eps_q, ro) <= ENERGY_RTOL
     assert rel_frobenius(F, Fq) <= FORCE_RTOL_DEQUANT
-    E32, _, F32 = oracle.energy_forces(oracle_model(w, weights), x64, types, w.replica_offsets())
     assert rel_frobenius(F, F32) <= FORCE_RTOL_16BIT
 
 
@@ -182,5 +185,7 @@ def test_protein64_sampled_replicas():
     for r in (0, 37, 63):
         sl = slice(r * w.beads, (r + 1) * w.beads)
         Eo, eps_o, Fo = oracle.energy_forces(m, pos[sl].astype(np.float64), types[sl])
+        print(f"[errors fp32 replica {r}] energy {energy_rel(E[r:r + 1], Eo, eps_o):.3e}, "
+              f"forces {rel_frobenius(F[sl], Fo):.3e}")
         assert energy_rel(E[r:r + 1], Eo, eps_o) <= ENERGY_RTOL
         assert rel_frobenius(F[sl], Fo) <= FORCE_RTOL

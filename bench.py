@@ -46,11 +46,13 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling during the timed region."""
+    """nvidia-smi clock/throttle sampling (every 200 ms).  Started before the warm-up so
+    that the tool is already polling when the timed region begins; ``stop(t0, t1)``
+    keeps the samples whose timestamps fall inside [t0, t1] (host wall clock)."""
 
     def __init__(self, index=0):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+        q = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
@@ -60,29 +62,35 @@ class ClockSampler:
         except Exception:
             self.p = None
 
-    def stop(self):
+    def stop(self, t0=None, t1=None):
         if self.p is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.p.terminate()
         self.p.wait(timeout=10)
         self.f.flush()
         self.f.seek(0)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        rows = []
         for line in self.f.read().splitlines():
             t = [x.strip() for x in line.split(",")]
-            if len(t) < 8:
+            if len(t) < 9:
                 continue
             try:
-                sm.append(float(t[0])); mx.append(float(t[1]))
+                ts = datetime.datetime.strptime(t[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(t[1]), float(t[2]), t[5:9]))
             except ValueError:
                 continue
-            for n, v in zip(names, t[4:8]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
         os.unlink(self.f.name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [r for r in rows if t0 is None or (t0 <= r[0] <= t1)]
+        window = "timed region"
+        if not inside:                       # region shorter than the sampling period
+            inside = [min(rows, key=lambda r: abs(r[0] - t1))] if rows and t1 is not None else rows
+            window = "nearest sample to the end of the timed region"
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = {n for r in inside for n, v in zip(names, r[3]) if v.lower().startswith("active")}
+        sm = [r[1] for r in inside]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(r[2] for r in inside) if inside else None,
+                "reasons": sorted(reasons), "samples": len(inside), "window": window}
 
 
 def _dist():
@@ -219,22 +227,25 @@ def run_native(args):
     m = torch.tensor(mass, device=dev)
     kw = dict(dt=w.dt_fs, gamma=w.gamma_per_ps, temperature=w.temperature, n_rebuild=n_rb, seed=1234)
     # warm-up: initial build + forces, graph capture, W steps
+    clocks = ClockSampler(local) if rank == 0 else None
     flagged = []
     _, _, st = model.step(p, v, t, m, args.warmup, step0=0, raise_on_flag=False, **kw)
     flagged.append(st)
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local) if rank == 0 else None
+    edges_start = _edge_stats(model, p.cpu().numpy(), w) if rank == 0 else None
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
     l0 = model.kernel_launches()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
     ev0.record()
     _, _, st = model.step(p, v, t, m, steps, step0=args.warmup, resume=True, raise_on_flag=False, **kw)
     ev1.record()
     flagged.append(st)
     torch.cuda.synchronize()
+    wall1 = time.time()
     if ws > 1:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
@@ -244,7 +255,7 @@ def run_native(args):
               "torch_peak_allocated_MB": round(torch.cuda.max_memory_allocated(dev) / 1e6, 1),
               "device_used_MB": round((total_b - free_b) / 1e6, 1),
               "note": "device_used includes the CUDA context, the library image and the captured graphs"}
-    clk = clocks.stop() if clocks else None
+    clk = clocks.stop(wall0, wall1) if clocks else None
     t_max, atoms_total, value = aggregate_ranks(ms, w.n_atoms, steps, dist, dev)
     step_s = t_max * 1e-3 / steps
     ns_day_rep = (1.0 / step_s) * w.dt_fs * 86400 * 1e-6
@@ -281,6 +292,9 @@ def run_native(args):
                "F": w.F, "K": w.K, "L": w.L, "cutoff_A": w.cutoff, "skin_A": w.skin, "n_rebuild": n_rb,
                "dt_fs": w.dt_fs, "integrator": "BAOAB" if w.gamma_per_ps > 0 else "velocity Verlet",
                "weight_dtype": w.weight_dtype, "edges_listed": E_list, "edges_within_cutoff": E_cut,
+               "edges_within_cutoff_at_start": edges_start[1],
+               "edges_note": "no bonded terms: chains slowly expand, so the graph shrinks during the run; "
+                             "edges_within_cutoff is counted after the timed steps",
                "l2": "no flush: state carried step to step; per-step working set "
                      f"{(E_list * 20 + w.n_atoms * 128 * 4 * (2 * w.L + 4)) / 1e6:.0f} MB > 126 MB L2",
                "parallelism": f"replicas x{ws} ranks (independent)"}
@@ -346,6 +360,7 @@ def run_drift(args):
     chunk = w.n_rebuild
     n_chunks = max(1, args.drift_steps // chunk)
     ep, _, st = model.step(p, v, t, m, 0, step0=0, raise_on_flag=False, **kw)   # initial forces
+    edges0 = _edge_stats(model, pos, w)[1]
     ek0 = 0.5 * float((mass.astype(np.float64)[:, None] * vel.astype(np.float64) ** 2).sum()) / ACC
     times, etot, flags = [0.0], [float(ep.sum()) + ek0], int(st)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -358,6 +373,8 @@ def run_drift(args):
     ev1.record()
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1)
+    model.build_neighbors(p)
+    edges1 = _edge_stats(model, p.cpu().numpy(), w)[1]
     tt, ee = np.array(times), np.array(etot) / w.n_atoms
     slope, icpt = np.polyfit(tt, ee, 1)
     resid = ee - (slope * tt + icpt)
@@ -370,6 +387,8 @@ def run_drift(args):
            "etot_per_atom_rms_about_fit": float(np.sqrt((resid ** 2).mean())),
            "ekin_per_atom_last": ekin0, "status": nat_status(flags),
            "ms_per_step": round(ms / (n_chunks * chunk), 4),
+           "edges_within_cutoff_first_last": [edges0, edges1],
+           "note": "no bonded terms: the chains expand during the run, so the graph shrinks",
            "config": {"workload": w.name, "replicas": w.n_replicas, "atoms": w.n_atoms, "n_rebuild": w.n_rebuild,
                       "skin_A": w.skin, "read_every_steps": chunk}, "data": "synthetic"}
     model.close()

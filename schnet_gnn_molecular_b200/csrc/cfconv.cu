@@ -36,10 +36,11 @@ struct MPArgs {
     long long cap;
     Box box;
     float rc, inv_rc;
-    float mu0, dmu, inv2s2, invs2;
-    int K;
+    float mu0, dmu;       // Gaussian centres mu_k = mu0 + k dmu
+    float ngc;            // -log2(e) / (2 sigma^2): e_k = 2^(ngc (d - mu_k)^2)
     const uint8_t* img;   // this layer's packed W1^T / W2^T images
-    const float *s1, *s2, *b1, *b2;  // this layer's scales and biases [FP]
+    const float *s1, *s2, *b1;  // this layer's channel scales and first-layer bias [FP]
+    const float* b2s;     // second-layer bias folded with the base-2 softplus shift [FP]
     const float* h;       // [N][FP]
     const float* u;       // [N][FP]   (backward)
     float* out;           // m (forward) or dh (backward)   [N][FP]
@@ -83,10 +84,19 @@ struct ChunkInfo {
     int32_t other;
 };
 
+// Per-edge records of one tile, stored as arrays so that an epilogue thread
+// reads four consecutive edges with one 16-byte shared load.  A masked edge
+// (d >= r_c, or d = 0) keeps a valid column index and gets f_c = f_c' = 0, so
+// it contributes exactly zero without a branch; padding edges past the end of
+// the run get row = INT_MAX, column 0 and f_c = f_c' = 0.
 struct TileMeta {
-    EdgeMeta e[TILE_E];
+    int32_t row[TILE_E];
+    int32_t col[TILE_E];
+    float fc[TILE_E];
+    float dfc[TILE_E];
     ChunkInfo c[TILE_E / 32];
 };
+static_assert(sizeof(TileMeta) == TILEMETA_BYTES, "tile metadata layout");
 
 __device__ __forceinline__ void copy_weights(uint8_t* smem, const uint8_t* __restrict__ img)
 {
@@ -174,7 +184,10 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
 
 // Stage R: four threads per edge (one per 16 Gaussians): distance (minimum
 // image), cutoff mask, Gaussian expansion (and its d-derivative when BWD)
-// written as hi/lo 16-bit K-major B operands.
+// written as hi/lo 16-bit K-major B operands.  The derivative operand holds
+// (d e_k / d d) / (2 ln 2); the backward epilogue folds the factor back in.
+// Gaussian columns past K meet zero weight rows, and masked or padding edges
+// have f_c = f_c' = 0, so neither needs a mask here (both stay finite).
 template <int FMT, bool BWD>
 __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMeta* tmeta, const EdgePre& ep, int ne)
 {
@@ -195,37 +208,36 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMe
             fc = 0.5f * (cs + 1.0f);
             dfc = -0.5f * 3.14159265358979f * a.inv_rc * sn;
         }
-        EdgeMeta m;
-        m.row = e < ne ? ep.i : 0x7fffffff;
-        m.col = valid ? ep.j : -1;
-        m.fc = fc;
-        m.dfc = dfc;
-        tmeta->e[e] = m;
+        const int row = e < ne ? ep.i : 0x7fffffff;
+        tmeta->row[e] = row;
+        tmeta->col[e] = e < ne ? ep.j : 0;
+        tmeta->fc[e] = fc;
+        if (BWD) tmeta->dfc[e] = dfc;
         // warp w of this quarter holds edges 32w .. 32w+31: summarise the chunk's rows
         const int lane = threadIdx.x & 31, w = e >> 5;
         const int nv = min(max(ne - 32 * w, 0), 32);
-        const int rfirst = __shfl_sync(0xffffffffu, m.row, 0);
-        const int rlast = __shfl_sync(0xffffffffu, m.row, nv > 0 ? nv - 1 : 0);
-        const unsigned fm = __ballot_sync(0xffffffffu, e < ne && m.row == rfirst);
-        const int oth = __any_sync(0xffffffffu, e < ne && m.row != rfirst && m.row != rlast);
+        const int rfirst = __shfl_sync(0xffffffffu, row, 0);
+        const int rlast = __shfl_sync(0xffffffffu, row, nv > 0 ? nv - 1 : 0);
+        const unsigned fm = __ballot_sync(0xffffffffu, e < ne && row == rfirst);
+        const int oth = __any_sync(0xffffffffu, e < ne && row != rfirst && row != rlast);
         if (lane == 0) tmeta->c[w] = ChunkInfo{rfirst, rlast, fm, oth};
     }
     uint8_t* b_hi = smem + SM_X;
     uint8_t* b_lo = b_hi + RBF_TERM;
-    (void)tmeta;
     uint8_t* p_hi = smem + SM_X + 2 * RBF_TERM;   // derivative tile (backward)
     uint8_t* p_lo = p_hi + RBF_TERM;
+    const float dm = d - fmaf((float)(kq * 16), a.dmu, a.mu0);   // d - mu of this thread's first Gaussian
 #pragma unroll
     for (int g = 0; g < 2; ++g) {
         const int kg = kq * 2 + g;
         float gv[8], dv[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const int k = kg * 8 + q;
-            float x = d - (a.mu0 + (float)k * a.dmu);
-            float gg = (valid && k < a.K) ? __expf(-x * x * a.inv2s2) : 0.f;
+            const float x = fmaf(-(float)(g * 8 + q), a.dmu, dm);
+            const float t = x * a.ngc;
+            const float gg = ex2_mufu(t * x);
             gv[q] = gg;
-            dv[q] = -x * a.invs2 * gg;
+            dv[q] = t * gg;
         }
         const uint32_t off = kmajor_off(e, kg * 8, TILE_E);
         store8<FMT>(b_hi, b_lo, off, gv);
@@ -265,15 +277,32 @@ __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, DevMeta
     return true;
 }
 
-// x_j,f (one feature per thread) for n consecutive edges starting at e; masked edges read nothing
+// x_j,f (one feature per thread, src_f = x + f) for N consecutive edges starting at e;
+// the column indices come four at a time from the tile's column array
 template <int N>
-__device__ __forceinline__ void gather(const float* __restrict__ src, const TileMeta* tm, int e, int f,
-                                       float (&dst)[N])
+__device__ __forceinline__ void gather(const float* __restrict__ src_f, const TileMeta* tm, int e, float (&dst)[N])
 {
 #pragma unroll
-    for (int q = 0; q < N; ++q) {
-        const int j = tm->e[e + q].col;
-        dst[q] = j >= 0 ? __ldg(src + (size_t)j * FP + f) : 0.f;
+    for (int q = 0; q < N; q += 4) {
+        const int4 j = *reinterpret_cast<const int4*>(tm->col + e + q);
+        dst[q] = __ldg(src_f + (size_t)j.x * FP);
+        dst[q + 1] = __ldg(src_f + (size_t)j.y * FP);
+        dst[q + 2] = __ldg(src_f + (size_t)j.z * FP);
+        dst[q + 3] = __ldg(src_f + (size_t)j.w * FP);
+    }
+}
+
+// N per-edge values of the tile's array v starting at edge e (16-byte loads)
+template <int N>
+__device__ __forceinline__ void load_edges(const float* v, int e, float (&dst)[N])
+{
+#pragma unroll
+    for (int q = 0; q < N; q += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(v + e + q);
+        dst[q] = x.x;
+        dst[q + 1] = x.y;
+        dst[q + 2] = x.z;
+        dst[q + 3] = x.w;
     }
 }
 
@@ -288,7 +317,7 @@ struct ChunkSeg {
 
 __device__ __forceinline__ void seg_begin(ChunkSeg& c, const TileMeta* tm, int eb)
 {
-    c.rfirst = tm->e[eb].row;
+    c.rfirst = tm->row[eb];
     c.lrow = c.rfirst;
     c.acc = 0.f;
     c.pf = 0.f;
@@ -377,21 +406,23 @@ __device__ __forceinline__ void chunk_partials(const TileMeta* tm, int cidx, int
     for (int q = 0; q < N; ++q) {
         const int e = eb + q;
         if (e >= ne) break;
-        seg_row(c, tm->e[e].row, out, f);
+        seg_row(c, tm->row[e], out, f);
         c.acc += t[q];
     }
     if (c.lrow == c.rfirst) { pf = c.acc; pl = 0.f; } else { pf = c.pf; pl = c.acc; }
 }
 
-// forward epilogue 1 for this warp's 32 edges: a = ssp(s1 P + b1) -> MN-major B operand
+// forward epilogue 1 for this warp's 32 edges: a = sp2(s1 log2e P + b1 log2e) -> MN-major
+// B operand (the base-2 softplus; ssp = ln2 (a - 1), with ln2 and the shift folded
+// into the second layer's scale and bias)
 template <int FMT>
-__device__ __forceinline__ void fwd_e1(uint32_t tP, float s1, float b1, uint8_t* smem, int cg, int f)
+__device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_t* smem, int cg, int f)
 {
     float r[32];
     tmem_ld32(tP, r);
     tmem_ld_wait();
 #pragma unroll
-    for (int q = 0; q < 32; ++q) r[q] = ssp(fmaf(s1, r[q], b1));
+    for (int q = 0; q < 32; ++q) r[q] = sp2(fmaf(s1L, r[q], b1L));
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         const uint32_t off = mnmajor_off(cg * 32 + g * 8, f, TILE_E);
@@ -399,8 +430,8 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1, float b1, uint8_t*
     }
 }
 
-// forward epilogue 2 for this warp's chunk: W = f_c (s2 Q + b2), terms h_j W, chunk partials
-__device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta* tm, int cg, int ne, float s2, float b2,
+// forward epilogue 2 for this warp's chunk: W = f_c (s2 ln2 Q + b2s), terms h_j W, chunk partials
+__device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta* tm, int cg, int ne, float s2L, float b2s,
                                        const float (&hv)[32], float* __restrict__ out, int f, float& pf, float& pl)
 {
     float r[32];
@@ -409,11 +440,10 @@ __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta* tm, int cg, 
     const int eb = cg * 32;
     pf = pl = 0.f;
     if (eb >= ne) return;
+    float fc[32];
+    load_edges<32>(tm->fc, eb, fc);
 #pragma unroll
-    for (int q = 0; q < 32; ++q) {
-        const EdgeMeta m = tm->e[eb + q];   // padding and masked edges have col < 0
-        r[q] = m.col >= 0 ? m.fc * fmaf(s2, r[q], b2) * hv[q] : 0.f;
-    }
+    for (int q = 0; q < 32; ++q) r[q] = fc[q] * fmaf(s2L, r[q], b2s) * hv[q];
     chunk_partials<32>(tm, cg, eb, ne, r, out, f, pf, pl);
 }
 
@@ -458,7 +488,9 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     const uint32_t id = idesc_f16(128, TILE_E, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, TILE_E, FMT, 1);
 
-    const float s1 = a.s1[f], b1 = a.b1[f], s2 = a.s2[f], b2 = a.b2[f];
+    const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF;
+    const float s2L = a.s2[f] * LN2F, b2s = a.b2s[f];
+    const float* h_f = a.h + f;
     int cur = r0;          // carried row and partial sum (threads 0..127, feature = threadIdx.x)
     float acc = 0.f;
     uint32_t phase = 0;
@@ -482,7 +514,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         }
         ok = wait_mma(bar, phase, a.meta);
         if (ok) {
-            fwd_e1<FMT>(tP, s1, b1, smem, cg, f);
+            fwd_e1<FMT>(tP, s1L, b1L, smem, cg, f);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncthreads();
@@ -504,7 +536,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
                 if (t + 2 < ntiles) ep = prefetch_edge(a, e0 + (long long)(t + 2) * TILE_E, tile_ne(t + 2));
             }
             float hv[32];
-            gather<32>(a.h, tm, cg * 32, f, hv);
+            gather<32>(h_f, tm, cg * 32, hv);
             if (!(ok = wait_mma(bar, phase, a.meta))) break;      // GEMM2(t) done; next tile's operand ready
             if (next && threadIdx.x == 0) {
                 issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
@@ -512,14 +544,14 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
             }
             // (GEMM1 of tile t+1 in flight) epilogue 2 and the in-order merge of tile t
             float pf, pl;
-            fwd_e2(tQ, tm, cg, ne, s2, b2, hv, a.out, f, pf, pl);
+            fwd_e2(tQ, tm, cg, ne, s2L, b2s, hv, a.out, f, pf, pl);
             pf_s[cg * 128 + f] = pf;
             pl_s[cg * 128 + f] = pl;
             __syncthreads();
             if (threadIdx.x < 128) merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
             if (next) {
                 if (!(ok = wait_mma(bar, phase, a.meta))) break;  // GEMM1(t+1) done
-                fwd_e1<FMT>(tP, s1, b1, smem, cg, f);
+                fwd_e1<FMT>(tP, s1L, b1L, smem, cg, f);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncthreads();
@@ -555,10 +587,12 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 // ---------------------------------------------------------------------------
 // backward: dh_i = sum_j u_j (.) W_ij ;  s_e = sum_f W'_e,f u_i,f h_j,f
 // ---------------------------------------------------------------------------
-// backward epilogue 1 for this warp's 32 edges: a = ssp(p), b = ssp'(p) p'  (p = s1 P + b1, p' = s1 P')
+// backward epilogue 1 for this warp's 32 edges: a = sp2(p), b = ssp'(x) dx/dd, with
+// p = x log2e = s1 log2e P + b1 log2e and dx/dd = s1 2ln2 P' (P' from the scaled
+// Gaussian-derivative operand).  ssp'(x) = 1 / (1 + e^-x) shares 2^-|p| with sp2.
 template <int FMT>
-__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1, float b1, uint8_t* smem, uint32_t col0,
-                                       int f)
+__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* smem,
+                                       uint32_t col0, int f)
 {
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -568,10 +602,13 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1, floa
         tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-            float sv, gv;
-            ssp_and_grad(fmaf(s1, r[q], b1), sv, gv);
-            r[q] = sv;
-            rd[q] = gv * s1 * rd[q];
+            const float p = fmaf(s1L, r[q], b1L);
+            const float t = ex2_mufu(-fabsf(p));
+            const float y = 1.0f + t;
+            const float inv = rcp_mufu(y);
+            const float sg = p >= 0.0f ? inv : t * inv;       // logistic(x)
+            r[q] = fmaxf(p, 0.0f) + lg2_mufu(y);
+            rd[q] = sg * (s1d * rd[q]);
         }
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
@@ -626,7 +663,10 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     const uint32_t id = idesc_f16(128, TILE_E, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, TILE_E, FMT, 1);
 
-    const float s1 = a.s1[f], b1 = a.b1[f], s2 = a.s2[f], b2 = a.b2[f];
+    const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF, s1d = a.s1[f] * (2.0f * LN2F);
+    const float s2 = a.s2[f], s2L = a.s2[f] * LN2F, b2s = a.b2s[f];
+    const float* h_f = a.h + f;
+    const float* u_f = a.u + f;
     int cur = r0;
     float acc = 0.f;
     uint32_t phase = 0;
@@ -655,7 +695,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         }
         ok = wait_mma(bar, phase, a.meta);
         if (ok) {
-            bwd_e1<FMT>(tP, tPd, s1, b1, smem, col0, f);
+            bwd_e1<FMT>(tP, tPd, s1L, b1L, s1d, smem, col0, f);
             fence_proxy_async_smem();
             tc_fence_before();
             __syncthreads();
@@ -673,8 +713,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             const long long t0 = e0 + (long long)t * TILE_E;
             const int eb = (int)col0;
             float uv[16], hv[16];
-            gather<16>(a.u, tm, eb, f, uv);
-            gather<16>(a.h, tm, eb, f, hv);
+            gather<16>(u_f, tm, eb, uv);
+            gather<16>(h_f, tm, eb, hv);
             if (!(ok = wait_mma(bar, phase, a.meta))) break;            // GEMM2(t) done
             if (next) {
                 // Gaussians of the next tile into the (now dead) ssp(p) region; its metadata is staged
@@ -693,91 +733,107 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                     mma_commit(bar);
                 }
             }
-            // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 Q + b2, z' = s2 Q')
+            // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 ln2 Q + b2s, z' = s2 Q')
             {
                 const bool active = eb < ne;
                 const ChunkInfo ci = tm->c[cg];
-                // one or two rows in the chunk (the usual case): predicated first/last-row sums;
-                // otherwise the serial segmented sum with a row change test per edge
-                const float u_first = active ? __ldg(a.u + (size_t)ci.rfirst * FP + f) : 0.f;
-                const float u_last = active ? __ldg(a.u + (size_t)ci.rlast * FP + f) : 0.f;
-                float sf = 0.f, sl = 0.f;
-                ChunkSeg c{0, 0, 0.f, 0.f};
-                if (active && ci.other) seg_begin(c, tm, eb);
-                float u_row = u_first;
-    #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    if (hh == 1) {
-                        gather<16>(a.u, tm, eb + 16, f, uv);
-                        gather<16>(a.h, tm, eb + 16, f, hv);
-                    }
-                    float r[16], rd[16];
-                    tmem_ld16(tQ + hh * 16, r);
-                    tmem_ld16(tQd + hh * 16, rd);
-                    tmem_ld_wait();
-                    if (!ci.other) {
-    #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const int qq = hh * 16 + q;
-                            const EdgeMeta m = tm->e[eb + qq];
-                            float tval = 0.f;
-                            if (m.col >= 0) {
-                                const float z = fmaf(s2, r[q], b2);
-                                const float wd = fmaf(m.dfc, z, m.fc * s2 * rd[q]);
-                                const bool first = (ci.firstmask >> qq) & 1u;
-                                const float dt = m.fc * z * uv[q];
-                                sf += first ? dt : 0.f;
-                                sl += first ? 0.f : dt;
-                                tval = wd * (first ? u_first : u_last) * hv[q];
-                            }
-                            rd[q] = tval;
-                        }
-                    } else {
-    #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const int e = eb + hh * 16 + q;
-                            float tval = 0.f;
-                            if (e < ne) {
-                                const EdgeMeta m = tm->e[e];
-                                if (m.row != c.lrow) {
-                                    seg_row(c, m.row, a.out, f);
-                                    u_row = __ldg(a.u + (size_t)m.row * FP + f);
-                                }
-                                if (m.col >= 0) {
-                                    const float z = fmaf(s2, r[q], b2);
-                                    const float wd = fmaf(m.dfc, z, m.fc * s2 * rd[q]);
-                                    c.acc = fmaf(m.fc * z, uv[q], c.acc);
-                                    tval = wd * u_row * hv[q];
-                                }
-                            }
-                            rd[q] = tval;
-                        }
-                    }
-                    // transpose-reduce the 16 per-edge values over the warp's 32 features:
-                    // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
-    #pragma unroll
-                    for (int sh = 16; sh >= 2; sh >>= 1) {
-                        const bool upper = (lane & sh) != 0;
-    #pragma unroll
-                        for (int k = 0; k < sh / 2; ++k) {
-                            float send = upper ? rd[k] : rd[k + sh / 2];
-                            float keep = upper ? rd[k + sh / 2] : rd[k];
-                            rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
-                        }
-                    }
-                    rd[0] += __shfl_xor_sync(0xffffffffu, rd[0], 1);
-                    if ((lane & 1) == 0) ps_s[qd * TILE_E + eb + hh * 16 + (lane >> 1)] = rd[0];
-                }
+                // 1: one row in the chunk; 2: two rows (the first a prefix); 3: the general
+                // serial segmented sum with a row change test per edge
+                const int kind = !active ? 0 : ci.other ? 3 : (ci.rfirst == ci.rlast ? 1 : 2);
                 float pf = 0.f, pl = 0.f;
-                if (active) {
-                    if (!ci.other) {
-                        if (ci.rfirst == ci.rlast) {
-                            pf = sf + sl;
-                        } else {
-                            pf = sf;
-                            pl = sl;
-                            for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
+                if (kind != 0) {
+                    const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
+                    const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
+                    float sf = 0.f, sl = 0.f;
+                    ChunkSeg c{0, 0, 0.f, 0.f};
+                    if (kind == 3) seg_begin(c, tm, eb);
+                    float u_row = u_first;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (hh == 1) {
+                            gather<16>(u_f, tm, eb + 16, uv);
+                            gather<16>(h_f, tm, eb + 16, hv);
                         }
+                        float r[16], rd[16];
+                        tmem_ld16(tQ + hh * 16, r);
+                        tmem_ld16(tQd + hh * 16, rd);
+                        tmem_ld_wait();
+                        const float* fcp = tm->fc + eb + hh * 16;
+                        const float* dfcp = tm->dfc + eb + hh * 16;
+                        if (kind == 1) {
+#pragma unroll
+                            for (int g = 0; g < 16; g += 4) {
+                                float fc[4], dfc[4];
+                                load_edges<4>(fcp, g, fc);
+                                load_edges<4>(dfcp, g, dfc);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const int q = g + i;
+                                    const float z = fmaf(s2L, r[q], b2s);
+                                    sf = fmaf(fc[i] * z, uv[q], sf);
+                                    const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
+                                    rd[q] = wd * (u_first * hv[q]);
+                                }
+                            }
+                        } else if (kind == 2) {
+#pragma unroll
+                            for (int g = 0; g < 16; g += 4) {
+                                float fc[4], dfc[4];
+                                load_edges<4>(fcp, g, fc);
+                                load_edges<4>(dfcp, g, dfc);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const int q = g + i;
+                                    const float z = fmaf(s2L, r[q], b2s);
+                                    const float dt = fc[i] * z * uv[q];
+                                    const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
+                                    sf += first ? dt : 0.f;
+                                    sl += first ? 0.f : dt;
+                                    const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
+                                    rd[q] = wd * ((first ? u_first : u_last) * hv[q]);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 16; ++q) {
+                                const int e = eb + hh * 16 + q;
+                                float tval = 0.f;
+                                if (e < ne) {
+                                    const int row = tm->row[e];
+                                    if (row != c.lrow) {
+                                        seg_row(c, row, a.out, f);
+                                        u_row = __ldg(u_f + (size_t)row * FP);
+                                    }
+                                    const float fcq = fcp[q], dfcq = dfcp[q];
+                                    const float z = fmaf(s2L, r[q], b2s);
+                                    const float wd = fmaf(dfcq, z, fcq * (s2 * rd[q]));
+                                    c.acc = fmaf(fcq * z, uv[q], c.acc);
+                                    tval = wd * (u_row * hv[q]);
+                                }
+                                rd[q] = tval;
+                            }
+                        }
+                        // transpose-reduce the 16 per-edge values over the warp's 32 features:
+                        // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
+#pragma unroll
+                        for (int sh = 16; sh >= 2; sh >>= 1) {
+                            const bool upper = (lane & sh) != 0;
+#pragma unroll
+                            for (int k = 0; k < sh / 2; ++k) {
+                                float send = upper ? rd[k] : rd[k + sh / 2];
+                                float keep = upper ? rd[k + sh / 2] : rd[k];
+                                rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+                            }
+                        }
+                        rd[0] += __shfl_xor_sync(0xffffffffu, rd[0], 1);
+                        if ((lane & 1) == 0) ps_s[qd * TILE_E + eb + hh * 16 + (lane >> 1)] = rd[0];
+                    }
+                    if (kind == 1) {
+                        pf = sf;
+                    } else if (kind == 2) {
+                        pf = sf;
+                        pl = sl;
+                        for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
                     } else if (c.lrow == c.rfirst) {
                         pf = c.acc;
                     } else {
@@ -804,7 +860,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                 cur_g = nxt_g;
                 cur_so = nxt_so;
                 if (!(ok = wait_mma(bar, phase, a.meta))) break;        // GEMM1(t+1) done
-                bwd_e1<FMT>(tP, tPd, s1, b1, smem, col0, f);
+                bwd_e1<FMT>(tP, tPd, s1L, b1L, s1d, smem, col0, f);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncthreads();
@@ -927,14 +983,12 @@ static MPArgs make_args(schnet_ctx* c, int layer)
     a.inv_rc = 1.0f / c->cfg.cutoff;
     a.mu0 = c->mu0;
     a.dmu = c->dmu;
-    a.inv2s2 = 1.0f / (2.0f * c->cfg.rbf_sigma * c->cfg.rbf_sigma);
-    a.invs2 = 1.0f / (c->cfg.rbf_sigma * c->cfg.rbf_sigma);
-    a.K = c->K;
+    a.ngc = (float)(-1.4426950408889634 / (2.0 * (double)c->cfg.rbf_sigma * (double)c->cfg.rbf_sigma));
     a.img = w.img + (size_t)layer * LAYER_IMG;
     a.s1 = w.s1 + layer * FP;
     a.s2 = w.s2 + layer * FP;
     a.b1 = w.b1 + layer * FP;
-    a.b2 = w.b2 + layer * FP;
+    a.b2s = w.b2s + layer * FP;
     a.h = w.h + (size_t)layer * c->N * FP;
     a.u = w.m;
     a.out = nullptr;

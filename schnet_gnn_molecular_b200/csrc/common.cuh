@@ -50,6 +50,36 @@ __device__ __forceinline__ float sigmoidf(float x)
     return x >= 0.0f ? r : t * r;
 }
 
+// Single MUFU operations (PTX ex2.approx / lg2.approx / rcp.approx, denormals flushed).
+constexpr float LOG2EF = 1.44269504088896340736f;
+
+__device__ __forceinline__ float ex2_mufu(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_mufu(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_mufu(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Softplus in base 2: for p = x log2(e), sp2(p) = log2(1 + 2^p) = log2(1 + e^x),
+// so that ssp(x) = ln2 (sp2(p) - 1).  Written as max(p, 0) + log2(1 + 2^-|p|):
+// no overflow for any p, and 1 + 2^-|p| lies in [1, 2].
+__device__ __forceinline__ float sp2(float p)
+{
+    return fmaxf(p, 0.0f) + lg2_mufu(1.0f + ex2_mufu(-fabsf(p)));
+}
+
 // ssp(x) and ssp'(x) sharing one exponential
 __device__ __forceinline__ void ssp_and_grad(float x, float& s, float& g)
 {

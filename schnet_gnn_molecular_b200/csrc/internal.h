@@ -30,7 +30,8 @@ struct Workspace {
     DevMeta* meta;
     // packed weights
     uint8_t* img;                 // [L][LAYER_IMG]
-    float *s1, *s2, *b1, *b2;     // [L][FP]
+    float *s1, *s2, *b1;          // [L][FP] filter channel scales, first-layer bias
+    float* b2s;                   // [L][FP] second-layer bias minus ln2 s2 sum_k W2^[k][f] (base-2 softplus shift)
     float *emb;                   // [T][FP]
     float *Win, *Wo1, *Wo2;       // [L][FP][FP]  (row-major [in][out])
     float *WinT, *Wo1T, *Wo2T;    // [L][FP][FP]  (transposed: [out][in])

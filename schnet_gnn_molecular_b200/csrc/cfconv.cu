@@ -1,7 +1,8 @@
 // Fused continuous-filter convolution on the sm_100a tensor cores.
 //
-// One kernel per interaction and direction does, for 128-edge tiles of a CTA's
-// contiguous CSR rows:
+// One kernel per interaction and direction does, for tiles of a CTA's contiguous
+// CSR rows (forward: 128 edges; backward: 64 edges, whose derivative rows fill
+// the other half of the GEMM's N = 128):
 //   flash radial basis  (FlashSchNet paper-curation summary, How): distance,
 //     Gaussian expansion and cosine envelope computed once per edge into
 //     shared memory, never to HBM;
@@ -19,7 +20,21 @@
 // Tile orientation: the GEMMs are computed transposed, D[f][e] = W^T[f][k] B[e][k],
 // so TMEM lane = output feature and TMEM column = edge.  Each epilogue thread
 // then owns one feature of every edge in the tile, the per-row reduction is a
-// running sum in one register, and the h_j gathers are 512-byte coalesced rows.
+// running sum in one register, and the h_j gathers are 128-byte coalesced rows.
+// The weights (A) are re-read from shared memory by every MMA, so every MMA
+// has N = 128 to keep that re-read at half of the shared-memory bandwidth the
+// tensor core draws: the backward kernel stacks each edge's value and
+// derivative operands into one B tile instead of issuing two N = 64 GEMMs.
+//
+// Ping-pong: the CTA's 16 warps form two math groups of 8 warps.  Group g takes
+// tiles g, g+2, g+4, ... of the CTA's edge run, each with its own TMEM columns,
+// shared-memory operand buffers, named barrier and MMA mbarrier; the two groups
+// share only the filter weights (read-only) and the tensor core.  While one
+// group waits for its GEMMs or its gathers, the other issues.  The CSR segment
+// sums cross tile boundaries through a carry (current row, partial sum per
+// feature) handed from tile to tile in order by an mbarrier token.  Group 1
+// starts once group 0's first GEMM1 has completed, so that the groups settle
+// half a tile apart rather than in step.
 #include "internal.h"
 
 namespace schnet {
@@ -38,6 +53,7 @@ struct MPArgs {
     float rc, inv_rc;
     float mu0, dmu;       // Gaussian centres mu_k = mu0 + k dmu
     float ngc;            // -log2(e) / (2 sigma^2): e_k = 2^(ngc (d - mu_k)^2)
+    int K;                // Gaussians (columns K .. KP-1 are padding)
     const uint8_t* img;   // this layer's packed W1^T / W2^T images
     const float *s1, *s2, *b1;  // this layer's channel scales and first-layer bias [FP]
     const float* b2s;     // second-layer bias folded with the base-2 softplus shift [FP]
@@ -48,33 +64,25 @@ struct MPArgs {
     int accumulate_s;
 };
 
-constexpr int NT = 512;   // threads per CTA: 16 warps, four per TMEM lane quadrant
+constexpr int NT = 512;                  // threads per CTA: two math groups of 8 warps
+constexpr int GT = 256;                  // threads per math group
+constexpr int MN = 128;                  // GEMM N of every MMA
+constexpr int TE_F = 128;                // forward: edges per tile
+constexpr int TE_B = 64;                 // backward: edges per tile (B rows 64..127 hold their derivatives)
 
 // shared-memory map (bytes)
-constexpr uint32_t SM_W1 = 0;                          // W1^T hi, lo   2 x 16 KB
-constexpr uint32_t SM_W2 = 32768;                      // W2^T hi, lo   2 x 32 KB
-constexpr uint32_t SM_X = 98304;                       // fwd: rbf hi/lo (32 KB) ; bwd: rbf, rbf' then a (64 KB)
-constexpr uint32_t SM_FWD_A = 131072;                  // fwd: a hi/lo (64 KB)
-constexpr uint32_t SM_BWD_Y = 163840;                  // bwd: ssp'(p) p' hi/lo (64 KB); partial sums after GEMM2
-constexpr uint32_t SM_META_FWD = 196608;
-constexpr uint32_t SM_META_BWD = 229376;
-constexpr uint32_t TILEMETA_BYTES = 2048 + 64;         // per-edge records + per-chunk row summary
-constexpr uint32_t PART_BYTES = 2 * 4 * 128 * 4;       // first/last-row partial per chunk and feature
-// forward: two metadata buffers (tile t and the next tile are live together)
-constexpr uint32_t SMEM_FWD = SM_META_FWD + 2 * TILEMETA_BYTES + PART_BYTES + 16;
-constexpr uint32_t SMEM_BWD = SM_META_BWD + TILEMETA_BYTES + 16;
-static_assert(SMEM_BWD <= 232448, "backward shared memory exceeds the per-block limit");
-
-constexpr uint32_t RBF_TERM = TILE_E * KP * 2;   // 16 KB: one 16-bit term of a [128 x 64] tile
-constexpr uint32_t ACT_TERM = TILE_E * FP * 2;   // 32 KB: one 16-bit term of a [128 x 128] tile
+constexpr uint32_t SM_W1 = 0;            // W1^T hi, lo   2 x 16 KB  (shared by both groups)
+constexpr uint32_t SM_W2 = 32768;        // W2^T hi, lo   2 x 32 KB
+constexpr uint32_t SM_OP = 98304;        // per-group operand regions
+constexpr uint32_t RBF_TERM = MN * KP * 2;   // 16 KB: one 16-bit term of a [128 x 64] GEMM1 B tile
+constexpr uint32_t ACT_TERM = MN * FP * 2;   // 32 KB: one 16-bit term of a [128 x 128] GEMM2 B tile
+// Per group: GEMM2's B operand hi/lo (64 KB); GEMM1's B operand hi/lo (32 KB)
+// overlays its start; after GEMM2 the region is dead and holds the partial sums.
+constexpr uint32_t OP_BYTES = 2 * ACT_TERM;
+constexpr uint32_t CARRY_BYTES = FP * 4 + 16;                // carried partial per feature + row (x2)
+constexpr uint32_t BAR_BYTES = 64;
 constexpr uint32_t WAIT_POLLS = 1u << 22;
 
-struct EdgeMeta {          // one 16-byte record per edge of the tile
-    int32_t row;
-    int32_t col;           // -1: padding or d >= r_c (masked)
-    float fc;
-    float dfc;
-};
 // Row summary of one 32-edge chunk, written once per tile by warp votes in
 // stage R: first and last row, which edges belong to the first row, and
 // whether any third row occurs (then the general segmented path is taken).
@@ -88,21 +96,69 @@ struct ChunkInfo {
 // reads four consecutive edges with one 16-byte shared load.  A masked edge
 // (d >= r_c, or d = 0) keeps a valid column index and gets f_c = f_c' = 0, so
 // it contributes exactly zero without a branch; padding edges past the end of
-// the run get row = INT_MAX, column 0 and f_c = f_c' = 0.
+// the run get column 0 and f_c = f_c' = 0.  Row indices stay in global memory
+// (only chunks that hold three or more rows read them).
+template <int TE, bool BWD>
 struct TileMeta {
-    int32_t row[TILE_E];
-    int32_t col[TILE_E];
-    float fc[TILE_E];
-    float dfc[TILE_E];
-    ChunkInfo c[TILE_E / 32];
+    int32_t col[TE];
+    float fc[TE];
+    float dfc[BWD ? TE : 4];
+    ChunkInfo c[TE / 32];
 };
-static_assert(sizeof(TileMeta) == TILEMETA_BYTES, "tile metadata layout");
+
+template <int TE, bool BWD> constexpr uint32_t sm_meta() { return SM_OP + 2 * OP_BYTES; }
+template <int TE, bool BWD> constexpr uint32_t sm_carry() { return sm_meta<TE, BWD>() + 2 * sizeof(TileMeta<TE, BWD>); }
+template <int TE, bool BWD> constexpr uint32_t sm_bar() { return sm_carry<TE, BWD>() + CARRY_BYTES; }
+template <int TE, bool BWD> constexpr uint32_t smem_bytes() { return sm_bar<TE, BWD>() + BAR_BYTES; }
+// barrier block: [0] group 0 MMA commits, [1] group 1 MMA commits, [2] merge token,
+// [3] group 1 start (u64 each); then the TMEM base (u32), each group's MMA phase to
+// drain on an error exit (u32 x2) and each group's "commit outstanding" flag (u32 x2)
+static_assert(smem_bytes<TE_F, false>() <= 232448, "forward shared memory exceeds the per-block limit");
+static_assert(smem_bytes<TE_B, true>() <= 232448, "backward shared memory exceeds the per-block limit");
+static_assert(sizeof(TileMeta<TE_F, false>) % 16 == 0 && sizeof(TileMeta<TE_B, true>) % 16 == 0, "meta alignment");
+
+// Segment-sum state carried from one tile to the next (in tile order, across
+// the two groups): the open row and its partial sum per feature.  The row is
+// double-buffered by tile parity, so a slow reader of tile t-1's row never
+// races the writer of tile t's.
+struct Carry {
+    float acc[FP];
+    int32_t cur[2];
+    int32_t pad[2];
+};
+static_assert(sizeof(Carry) == CARRY_BYTES, "carry layout");
 
 __device__ __forceinline__ void copy_weights(uint8_t* smem, const uint8_t* __restrict__ img)
 {
     const uint4* src = reinterpret_cast<const uint4*>(img);
     uint4* dst = reinterpret_cast<uint4*>(smem + SM_W1);
     for (int i = threadIdx.x; i < (int)(LAYER_IMG / 16); i += blockDim.x) dst[i] = __ldg(src + i);
+}
+
+// named barrier of math group g (ids 1 and 2; id 0 is __syncthreads)
+__device__ __forceinline__ void group_sync(int g)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(GT) : "memory");
+}
+
+// OR of a predicate over math group g (a barrier of the group's 256 threads)
+__device__ __forceinline__ bool group_or(int g, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(1 + g), "n"(GT)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // two fp32 values -> packed 16-bit hi pair and lo (residual) pair
@@ -138,6 +194,12 @@ __device__ __forceinline__ void store8(uint8_t* hi_base, uint8_t* lo_base, uint3
     *reinterpret_cast<uint4*>(lo_base + off) = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+__device__ __forceinline__ void store8_zero(uint8_t* hi_base, uint8_t* lo_base, uint32_t off)
+{
+    *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(lo_base + off) = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // 32 lanes x 16 columns of TMEM -> 16 registers per thread
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
 {
@@ -150,7 +212,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
         : "r"(taddr));
 }
 
-// Endpoints of edge (threadIdx.x mod 128) of a tile, loaded one tile ahead so the
+// Endpoints of edge (group thread mod TE) of a tile, loaded one tile ahead so the
 // dependent loads (edge -> atom -> position) overlap the previous tile's work.
 struct EdgePre {
     int i, j;
@@ -159,8 +221,8 @@ struct EdgePre {
     float sold;    // backward: s_e accumulated by the later interactions so far
 };
 
-template <bool BWD = false>
-__device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, int ne)
+template <int TE, bool BWD>
+__device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, int ne, int mt)
 {
     EdgePre p;
     p.i = 0;
@@ -168,13 +230,13 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
     p.pi = p.pj = make_float4(0.f, 0.f, 0.f, 0.f);
     p.gidx = 0;
     p.sold = 0.f;
-    const int t = threadIdx.x & (TILE_E - 1);
+    const int t = mt & (TE - 1);
     if (t < ne) {
         p.i = __ldg(a.crow + e0 + t);
         p.j = __ldg(a.ccol + e0 + t);
         p.pi = __ldg(a.pos4 + p.i);
         p.pj = __ldg(a.pos4 + p.j);
-        if (BWD && threadIdx.x < TILE_E) {
+        if (BWD && mt < TE) {
             p.gidx = __ldg(a.cidx + e0 + t);
             if (a.accumulate_s) p.sold = a.s_edge[p.gidx];
         }
@@ -182,17 +244,21 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
     return p;
 }
 
-// Stage R: four threads per edge (one per 16 Gaussians): distance (minimum
-// image), cutoff mask, Gaussian expansion (and its d-derivative when BWD)
-// written as hi/lo 16-bit K-major B operands.  The derivative operand holds
-// (d e_k / d d) / (2 ln 2); the backward epilogue folds the factor back in.
-// Gaussian columns past K meet zero weight rows, and masked or padding edges
-// have f_c = f_c' = 0, so neither needs a mask here (both stay finite).
-template <int FMT, bool BWD>
-__device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMeta* tmeta, const EdgePre& ep, int ne)
+// Stage R: GT / TE threads per edge, each for KP / (GT / TE) Gaussians: distance
+// (minimum image), cutoff mask, Gaussian expansion written as hi/lo 16-bit
+// K-major B rows; in the backward tile row TE + e holds the d-derivative of
+// edge e's Gaussians, scaled by 1 / (2 ln 2) (the epilogue folds the factor
+// back in).  Gaussian columns K .. KP-1 meet zero weight rows and are stored
+// as zeros without evaluating them; masked or padding edges have
+// f_c = f_c' = 0, so their Gaussians need no mask (they stay finite).
+template <int FMT, bool BWD, int TE>
+__device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* op, TileMeta<TE, BWD>* tmeta, const EdgePre& ep,
+                                          int ne, int mt)
 {
-    const int e = threadIdx.x & (TILE_E - 1);
-    const int kq = threadIdx.x >> 7;
+    constexpr int TPE = GT / TE;         // threads per edge
+    constexpr int KPT = KP / TPE;        // Gaussians per thread
+    const int e = mt & (TE - 1);
+    const int kq = mt / TE;              // warp-uniform
     float d = 0.f;
     bool valid = false;
     if (e < ne) {
@@ -209,12 +275,11 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMe
             dfc = -0.5f * 3.14159265358979f * a.inv_rc * sn;
         }
         const int row = e < ne ? ep.i : 0x7fffffff;
-        tmeta->row[e] = row;
         tmeta->col[e] = e < ne ? ep.j : 0;
         tmeta->fc[e] = fc;
         if (BWD) tmeta->dfc[e] = dfc;
         // warp w of this quarter holds edges 32w .. 32w+31: summarise the chunk's rows
-        const int lane = threadIdx.x & 31, w = e >> 5;
+        const int lane = mt & 31, w = e >> 5;
         const int nv = min(max(ne - 32 * w, 0), 32);
         const int rfirst = __shfl_sync(0xffffffffu, row, 0);
         const int rlast = __shfl_sync(0xffffffffu, row, nv > 0 ? nv - 1 : 0);
@@ -222,14 +287,19 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMe
         const int oth = __any_sync(0xffffffffu, e < ne && row != rfirst && row != rlast);
         if (lane == 0) tmeta->c[w] = ChunkInfo{rfirst, rlast, fm, oth};
     }
-    uint8_t* b_hi = smem + SM_X;
-    uint8_t* b_lo = b_hi + RBF_TERM;
-    uint8_t* p_hi = smem + SM_X + 2 * RBF_TERM;   // derivative tile (backward)
-    uint8_t* p_lo = p_hi + RBF_TERM;
-    const float dm = d - fmaf((float)(kq * 16), a.dmu, a.mu0);   // d - mu of this thread's first Gaussian
+    uint8_t* b_hi = op;
+    uint8_t* b_lo = op + RBF_TERM;
+    const float dm = d - fmaf((float)(kq * KPT), a.dmu, a.mu0);   // d - mu of this thread's first Gaussian
 #pragma unroll
-    for (int g = 0; g < 2; ++g) {
-        const int kg = kq * 2 + g;
+    for (int g = 0; g < KPT / 8; ++g) {
+        const int kg = kq * (KPT / 8) + g;
+        const uint32_t off = kmajor_off(e, kg * 8, MN);
+        const uint32_t offd = kmajor_off(TE + e, kg * 8, MN);
+        if (kg * 8 >= a.K) {                 // padding columns (warp-uniform)
+            store8_zero(b_hi, b_lo, off);
+            if (BWD) store8_zero(b_hi, b_lo, offd);
+            continue;
+        }
         float gv[8], dv[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -239,52 +309,69 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* smem, TileMe
             gv[q] = gg;
             dv[q] = t * gg;
         }
-        const uint32_t off = kmajor_off(e, kg * 8, TILE_E);
         store8<FMT>(b_hi, b_lo, off, gv);
-        if (BWD) store8<FMT>(p_hi, p_lo, off, dv);
+        if (BWD) store8<FMT>(b_hi, b_lo, offd, dv);
     }
 }
 
-// Issue D (+)= W^T * B over `ksteps` K-steps of 16 with the hi/lo split.
+// Issue D (+)= W^T * B over `ksteps` K-steps of 16 with the hi/lo split
+// (A: 128 feature rows, B: MN = 128 rows; no-swizzle core matrices).
 template <int NW>
 __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_base, uint32_t a_term, uint32_t b_base,
                                            uint32_t b_term, int ksteps, uint32_t idesc)
 {
     for (int ks = 0; ks < ksteps; ++ks) {
-        uint32_t koff = (uint32_t)ks * 2u * (uint32_t)(FP * 16);   // 2 core matrices of 8 along K
+        const uint32_t koff = (uint32_t)ks * 2u * (uint32_t)(FP * 16);   // 2 core matrices of 8 along K
         uint64_t a_hi = smem_desc(a_base + koff, FP * 16, 128);
         uint64_t a_lo = smem_desc(a_base + a_term + koff, FP * 16, 128);
-        uint64_t b_hi = smem_desc(b_base + koff, TILE_E * 16, 128);
-        uint64_t b_lo = smem_desc(b_base + b_term + koff, TILE_E * 16, 128);
+        uint64_t b_hi = smem_desc(b_base + koff, MN * 16, 128);
+        uint64_t b_lo = smem_desc(b_base + b_term + koff, MN * 16, 128);
         mma_f16(d_tmem, a_hi, b_hi, idesc, ks > 0 ? 1u : 0u);
         if (NW == 2) mma_f16(d_tmem, a_lo, b_hi, idesc, 1u);
         mma_f16(d_tmem, a_hi, b_lo, idesc, 1u);
     }
 }
 
-// Wait for the tensor-core commit; returns false (uniformly) on timeout.
-__device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, DevMeta* meta)
+// Wait for group g's tensor-core commit; returns false (uniformly over the
+// group) on timeout, leaving `phase` at the commit still outstanding.  The
+// group's first warp polls, the others wait at the group barrier.
+__device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, DevMeta* meta, int g, int mt)
 {
     bool ok = true;
-    if ((threadIdx.x >> 5) == 0) ok = mbar_wait_bounded(bar, phase, WAIT_POLLS);   // the others sleep below
-    phase ^= 1u;
-    int bad = __syncthreads_or(!ok);
-    if (bad) {
-        if (threadIdx.x == 0) set_flag(meta, SCHNET_FLAG_TIMEOUT);
+    if ((mt >> 5) == 0) ok = mbar_wait_bounded(bar, phase, WAIT_POLLS);
+    if (group_or(g, !ok)) {
+        if (mt == 0) set_flag(meta, SCHNET_FLAG_TIMEOUT);
         return false;
     }
+    phase ^= 1u;
     tc_fence_after();
+    return true;
+}
+
+// Group-uniform bounded wait for phase `parity` of mbarrier `bar` (no wait when
+// !need).  Threads with `acquire` repeat the test after the decision, which
+// gives each of them its own acquire of what was released before the arrival.
+__device__ __forceinline__ bool wait_group(uint64_t* bar, uint32_t parity, bool need, bool acquire, DevMeta* meta,
+                                           int g, int mt)
+{
+    bool ok = true;
+    if (need && (mt >> 5) == 0) ok = mbar_wait_bounded(bar, parity, WAIT_POLLS);
+    if (group_or(g, !ok)) {
+        if (mt == 0) set_flag(meta, SCHNET_FLAG_TIMEOUT);
+        return false;
+    }
+    if (need && acquire && (mt >> 5) != 0) (void)mbar_try_wait(bar, parity);
     return true;
 }
 
 // x_j,f (one feature per thread, src_f = x + f) for N consecutive edges starting at e;
 // the column indices come four at a time from the tile's column array
 template <int N>
-__device__ __forceinline__ void gather(const float* __restrict__ src_f, const TileMeta* tm, int e, float (&dst)[N])
+__device__ __forceinline__ void gather(const float* __restrict__ src_f, const int32_t* col, int e, float (&dst)[N])
 {
 #pragma unroll
     for (int q = 0; q < N; q += 4) {
-        const int4 j = *reinterpret_cast<const int4*>(tm->col + e + q);
+        const int4 j = *reinterpret_cast<const int4*>(col + e + q);
         dst[q] = __ldg(src_f + (size_t)j.x * FP);
         dst[q + 1] = __ldg(src_f + (size_t)j.y * FP);
         dst[q + 2] = __ldg(src_f + (size_t)j.z * FP);
@@ -315,10 +402,10 @@ struct ChunkSeg {
     float acc, pf;
 };
 
-__device__ __forceinline__ void seg_begin(ChunkSeg& c, const TileMeta* tm, int eb)
+__device__ __forceinline__ void seg_begin(ChunkSeg& c, int rfirst)
 {
-    c.rfirst = tm->row[eb];
-    c.lrow = c.rfirst;
+    c.rfirst = rfirst;
+    c.lrow = rfirst;
     c.acc = 0.f;
     c.pf = 0.f;
 }
@@ -334,17 +421,17 @@ __device__ __forceinline__ void seg_row(ChunkSeg& c, int row, float* __restrict_
     }
 }
 
-// In-order merge of the four chunks' partials (threads 0..127, feature f).
-__device__ __forceinline__ void merge_chunks(const TileMeta* tm, const float* pf, const float* pl, int ne, int f,
+// In-order merge of a tile's chunk partials into the carried row (threads of
+// the group with feature f = group thread index < 128): rows the carry leaves
+// are complete and written out, with zeros for edge-less rows in between.
+template <int NCH>
+__device__ __forceinline__ void merge_chunks(const ChunkInfo* ci, const float* pf, const float* pl, int ne, int f,
                                              float* __restrict__ out, int& cur, float& acc)
 {
-#pragma unroll 1
-    for (int c = 0; c < TILE_E / 32; ++c) {
-        const int eb = c * 32;
-        if (eb >= ne) break;
-        const int last = min(eb + 31, ne - 1);
-        const int rfirst = tm->c[c].rfirst, rlast = tm->c[c].rlast;
-        (void)last;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        if (c * 32 >= ne) break;
+        const int rfirst = ci[c].rfirst, rlast = ci[c].rlast;
         const float v = pf[c * 128 + f];
         if (rfirst == cur) {
             acc += v;
@@ -362,6 +449,25 @@ __device__ __forceinline__ void merge_chunks(const TileMeta* tm, const float* pf
     }
 }
 
+// Merge step of tile t by its group: wait for tile t-1's merge, fold this
+// tile's partials into the carry, hand the carry on.  Returns false on timeout.
+template <int NCH>
+__device__ __forceinline__ bool merge_tile(Carry* cy, uint64_t* tok, const ChunkInfo* ci, const float* pf,
+                                           const float* pl, int ne, int t, float* __restrict__ out, DevMeta* meta,
+                                           int g, int mt)
+{
+    if (!wait_group(tok, (uint32_t)((t - 1) & 1), t > 0, mt < 128, meta, g, mt)) return false;
+    if (mt < 128) {
+        int cur = cy->cur[(t + 1) & 1];      // written by tile t-1 (or the initial row)
+        float acc = cy->acc[mt];
+        merge_chunks<NCH>(ci, pf, pl, ne, mt, out, cur, acc);
+        cy->acc[mt] = acc;
+        if (mt == 0) cy->cur[t & 1] = cur;
+        mbar_arrive(tok);
+    }
+    return true;
+}
+
 // pairwise sum of N values (fixed order)
 template <int N>
 __device__ __forceinline__ float tree_sum(float (&v)[N])
@@ -376,12 +482,13 @@ __device__ __forceinline__ float tree_sum(float (&v)[N])
 // Reduce a chunk's per-edge terms t[q] (edge eb + q) to the first-row and
 // last-row partials.  One or two rows: branch-free predicated sums (edge-less
 // rows strictly between them are written as zeros).  Three or more rows: the
-// serial segmented sum writes the inner rows out.
+// serial segmented sum (rows read from the tile's global row list) writes the
+// inner rows out.
 template <int N>
-__device__ __forceinline__ void chunk_partials(const TileMeta* tm, int cidx, int eb, int ne, float (&t)[N],
-                                               float* __restrict__ out, int f, float& pf, float& pl)
+__device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_t* __restrict__ rows_g, int eb,
+                                               int ne, float (&t)[N], float* __restrict__ out, int f, float& pf,
+                                               float& pl)
 {
-    const ChunkInfo ci = tm->c[cidx];
     if (!ci.other) {
         if (ci.rfirst == ci.rlast) {
             pf = tree_sum<N>(t);
@@ -400,23 +507,75 @@ __device__ __forceinline__ void chunk_partials(const TileMeta* tm, int cidx, int
         }
         return;
     }
-    ChunkSeg c{0, 0, 0.f, 0.f};
-    seg_begin(c, tm, eb);
+    ChunkSeg c;
+    seg_begin(c, ci.rfirst);
 #pragma unroll
     for (int q = 0; q < N; ++q) {
         const int e = eb + q;
         if (e >= ne) break;
-        seg_row(c, tm->row[e], out, f);
+        seg_row(c, __ldg(rows_g + e), out, f);
         c.acc += t[q];
     }
     if (c.lrow == c.rfirst) { pf = c.acc; pl = 0.f; } else { pf = c.pf; pl = c.acc; }
 }
 
-// forward epilogue 1 for this warp's 32 edges: a = sp2(s1 log2e P + b1 log2e) -> MN-major
-// B operand (the base-2 softplus; ssp = ln2 (a - 1), with ln2 and the shift folded
+// Common prologue of both kernels: TMEM allocation, mbarriers, weights into
+// shared memory, the initial carry.  Returns the TMEM base address.
+__device__ __forceinline__ uint32_t kernel_setup(uint8_t* smem, const MPArgs& a, uint32_t* tslot, uint64_t* bars,
+                                                 Carry* cy, int r0, uint32_t ncols)
+{
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
+        tmem_alloc(tslot, ncols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);      // group 0 MMA commits
+        mbar_init(&bars[1], 1);      // group 1 MMA commits
+        mbar_init(&bars[2], 128);    // merge token: the 128 merging threads of a tile
+        mbar_init(&bars[3], 1);      // group 1 start
+        fence_mbar_init();
+        cy->cur[1] = r0;             // tile 0 reads the carry of "tile -1"
+    }
+    if (threadIdx.x < FP) cy->acc[threadIdx.x] = 0.f;
+    copy_weights(smem, a.img);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *tslot;
+}
+
+// Common epilogue: the carried row is complete; rows after it without edges are zero.
+__device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r1, float* __restrict__ out, bool ok,
+                                              uint64_t* bars, const uint32_t* phases, const uint32_t* pending,
+                                              uint32_t tmem, uint32_t ncols)
+{
+    const int warp = threadIdx.x >> 5;
+    if (ok) {
+        if (threadIdx.x < FP) {
+            const int cur = cy->cur[(ntiles + 1) & 1];
+            out[(size_t)cur * FP + threadIdx.x] = cy->acc[threadIdx.x];
+            for (int rr = cur + 1; rr < r1; ++rr) out[(size_t)rr * FP + threadIdx.x] = 0.f;
+        }
+    } else if ((threadIdx.x & (GT - 1)) == 0) {
+        // drain: give the group's in-flight MMAs a bounded chance to retire before freeing TMEM
+        const int g = threadIdx.x / GT;
+        if (pending[g]) mbar_wait_bounded(&bars[g], phases[g], WAIT_POLLS);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, ncols);
+    }
+}
+
+// forward epilogue 1 for 32 edges: a = sp2(s1 log2e P + b1 log2e) -> MN-major B
+// operand (the base-2 softplus; ssp = ln2 (a - 1), with ln2 and the shift folded
 // into the second layer's scale and bias)
 template <int FMT>
-__device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_t* smem, int cg, int f)
+__device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_t* op, int e0, int f)
 {
     float r[32];
     tmem_ld32(tP, r);
@@ -425,26 +584,30 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
     for (int q = 0; q < 32; ++q) r[q] = sp2(fmaf(s1L, r[q], b1L));
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-        const uint32_t off = mnmajor_off(cg * 32 + g * 8, f, TILE_E);
-        store8<FMT>(smem + SM_FWD_A, smem + SM_FWD_A + ACT_TERM, off, r + g * 8);
+        const uint32_t off = mnmajor_off(e0 + g * 8, f, MN);
+        store8<FMT>(op, op + ACT_TERM, off, r + g * 8);
     }
 }
 
-// forward epilogue 2 for this warp's chunk: W = f_c (s2 ln2 Q + b2s), terms h_j W, chunk partials
-__device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta* tm, int cg, int ne, float s2L, float b2s,
-                                       const float (&hv)[32], float* __restrict__ out, int f, float& pf, float& pl)
+// forward epilogue 2 for chunk cc: W = f_c (s2 ln2 Q + b2s), terms h_j W, chunk partials
+template <int TE>
+__device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* tm, const int32_t* rows_g, int cc,
+                                       int ne, float s2L, float b2s, const float (&hv)[32], float* __restrict__ out,
+                                       int f, float& pf, float& pl)
 {
     float r[32];
     tmem_ld32(tQ, r);
     tmem_ld_wait();
-    const int eb = cg * 32;
+    const int eb = cc * 32;
     pf = pl = 0.f;
     if (eb >= ne) return;
     float fc[32];
     load_edges<32>(tm->fc, eb, fc);
 #pragma unroll
-    for (int q = 0; q < 32; ++q) r[q] = fc[q] * fmaf(s2L, r[q], b2s) * hv[q];
-    chunk_partials<32>(tm, cg, eb, ne, r, out, f, pf, pl);
+    for (int q = 0; q < 32; ++q) r[q] = fc[q] * fmaf(s2L, r[q], b2s);
+#pragma unroll
+    for (int q = 0; q < 32; ++q) r[q] *= hv[q];
+    chunk_partials<32>(tm->c[cc], rows_g, eb, ne, r, out, f, pf, pl);
 }
 
 // ---------------------------------------------------------------------------
@@ -453,135 +616,108 @@ __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta* tm, int cg, 
 template <int FMT, int NW>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {
+    constexpr int TE = TE_F;
+    constexpr int NCH = TE / 32;
+    using Meta = TileMeta<TE, false>;
     extern __shared__ __align__(1024) uint8_t smem[];
-    auto tmb = [&](int t) { return reinterpret_cast<TileMeta*>(smem + SM_META_FWD + (t & 1) * TILEMETA_BYTES); };
-    float* pf_s = reinterpret_cast<float*>(smem + SM_META_FWD + 2 * TILEMETA_BYTES);
-    float* pl_s = pf_s + 4 * 128;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_FWD + 2 * TILEMETA_BYTES + PART_BYTES);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_FWD + 2 * TILEMETA_BYTES + PART_BYTES + 8);
+    Carry* cy = reinterpret_cast<Carry*>(smem + sm_carry<TE, false>());
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sm_bar<TE, false>());
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+    uint32_t* phases_s = tslot + 1;
+    uint32_t* pend_s = tslot + 3;
 
     if (a.meta->n_edges > a.cap) return;
     const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
     if (r0 >= r1) return;
     const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qd = warp & 3, cg = warp >> 2;        // TMEM lane quadrant, 32-edge column chunk
+    const int g = warp >> 3;                        // math group
+    const int mt = threadIdx.x & (GT - 1);          // thread within the group
+    const int qd = warp & 3, ch = (warp >> 2) & 1;  // TMEM lane quadrant, 64-edge half of the tile
     const int f = qd * 32 + lane;                   // this thread's output feature
 
-    if (warp == 0) {
-        tmem_alloc(tslot, 256);
-        tmem_relinquish();
-    }
-    if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-    }
-    copy_weights(smem, a.img);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tslot;
+    const uint32_t tmem = kernel_setup(smem, a, tslot, bars, cy, r0, 512);
+    uint8_t* op = smem + SM_OP + g * OP_BYTES;
+    Meta* tm = reinterpret_cast<Meta*>(smem + sm_meta<TE, false>() + g * sizeof(Meta));
+    float* pf_s = reinterpret_cast<float*>(op);     // after GEMM2: [chunk][feature] partials
+    float* pl_s = pf_s + NCH * 128;
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    const uint32_t tP = tmem + lane_off + cg * 32, tQ = tmem + 128 + lane_off + cg * 32;
+    const uint32_t dP = tmem + g * 256, dQ = dP + 128;          // accumulators: P, then Q, 128 columns each
+    const uint32_t tP = dP + lane_off + ch * 64, tQ = dQ + lane_off + ch * 64;
+    const uint32_t sop = smem_u32(op);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t id = idesc_f16(128, TILE_E, FMT, 0);
-    const uint32_t id_mn = idesc_f16(128, TILE_E, FMT, 1);
-
+    const uint32_t id = idesc_f16(128, MN, FMT, 0);
+    const uint32_t id_mn = idesc_f16(128, MN, FMT, 1);
     const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF;
     const float s2L = a.s2[f] * LN2F, b2s = a.b2s[f];
     const float* h_f = a.h + f;
-    int cur = r0;          // carried row and partial sum (threads 0..127, feature = threadIdx.x)
-    float acc = 0.f;
-    uint32_t phase = 0;
-    bool ok = true;
-    const int ntiles = (int)((e1 - e0 + TILE_E - 1) / TILE_E);
-    auto tile_ne = [&](int t) { return (int)min((long long)TILE_E, e1 - e0 - (long long)t * TILE_E); };
 
-    // Software pipeline: tile t's GEMM2 runs while stage R of tile t+1 fills the
-    // Gaussian operand; tile t's epilogue 2 runs while GEMM1 of tile t+1 runs.
-    if (ntiles > 0) {
-        EdgePre ep = prefetch_edge(a, e0, tile_ne(0));
-        stage_rbf<FMT, false>(a, smem, tmb(0), ep, tile_ne(0));
-        if (ntiles > 1) ep = prefetch_edge(a, e0 + TILE_E, tile_ne(1));
+    uint32_t phase = 0, pending = 0;   // pending: a commit of this group not yet waited for
+    bool ok = true, go_sent = false;
+    const int ntiles = (int)((e1 - e0 + TE - 1) / TE);
+    auto tile_ne = [&](int t) { return (int)min((long long)TE, e1 - e0 - (long long)t * TE); };
+
+    EdgePre ep;
+    if (g < ntiles) {
+        ep = prefetch_edge<TE, false>(a, e0 + (long long)g * TE, tile_ne(g), mt);
+        if (g == 1) ok = wait_group(&bars[3], 0u, true, false, a.meta, g, mt);   // start half a tile behind
+    }
+    for (int t = g; t < ntiles && ok; t += 2) {
+        const int ne = tile_ne(t);
+        const int32_t* rows_g = a.crow + e0 + (long long)t * TE;
+        // stage R: Gaussians of this tile into the group's operand region
+        stage_rbf<FMT, false, TE>(a, op, tm, ep, ne, mt);
+        if (t + 2 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(t + 2) * TE, tile_ne(t + 2), mt);
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
-        if (threadIdx.x == 0) {
+        group_sync(g);
+        if (mt == 0) {
             tc_fence_after();
-            issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
-            mma_commit(bar);
+            issue_gemm<NW>(dP, sbase + SM_W1, (uint32_t)W1_IMG, sop, RBF_TERM, KP / 16, id);
+            mma_commit(&bars[g]);
         }
-        ok = wait_mma(bar, phase, a.meta);
-        if (ok) {
-            fwd_e1<FMT>(tP, s1L, b1L, smem, cg, f);
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                tc_fence_after();
-                issue_gemm<NW>(tmem + 128, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_FWD_A, ACT_TERM, FP / 16,
-                               id_mn);
-                mma_commit(bar);
-            }
+        pending = 1;
+        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM1 done
+        pending = 0;
+        if (g == 0 && !go_sent) {
+            if (mt == 0) mbar_arrive(&bars[3]);
+            go_sent = true;
         }
-        for (int t = 0; t < ntiles && ok; ++t) {
-            const int ne = tile_ne(t);
-            const bool next = t + 1 < ntiles;
-            TileMeta* tm = tmb(t);
-            // (GEMM2 of tile t in flight) Gaussians of the next tile, then this chunk's h_j rows
-            if (next) {
-                stage_rbf<FMT, false>(a, smem, tmb(t + 1), ep, tile_ne(t + 1));
-                fence_proxy_async_smem();
-                if (t + 2 < ntiles) ep = prefetch_edge(a, e0 + (long long)(t + 2) * TILE_E, tile_ne(t + 2));
-            }
-            float hv[32];
-            gather<32>(h_f, tm, cg * 32, hv);
-            if (!(ok = wait_mma(bar, phase, a.meta))) break;      // GEMM2(t) done; next tile's operand ready
-            if (next && threadIdx.x == 0) {
-                issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
-                mma_commit(bar);
-            }
-            // (GEMM1 of tile t+1 in flight) epilogue 2 and the in-order merge of tile t
+#pragma unroll 1
+        for (int c2 = 0; c2 < 2; ++c2) fwd_e1<FMT>(tP + c2 * 32, s1L, b1L, op, ch * 64 + c2 * 32, f);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        group_sync(g);
+        if (mt == 0) {
+            tc_fence_after();
+            issue_gemm<NW>(dQ, sbase + SM_W2, (uint32_t)W2_IMG, sop, ACT_TERM, FP / 16, id_mn);
+            mma_commit(&bars[g]);
+        }
+        pending = 1;
+        float hv[32];
+        gather<32>(h_f, tm->col, ch * 64, hv);                          // under GEMM2
+        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2 done
+        pending = 0;
+#pragma unroll 1
+        for (int c2 = 0; c2 < 2; ++c2) {
+            const int cc = ch * 2 + c2;
+            if (c2 == 1) gather<32>(h_f, tm->col, cc * 32, hv);
             float pf, pl;
-            fwd_e2(tQ, tm, cg, ne, s2L, b2s, hv, a.out, f, pf, pl);
-            pf_s[cg * 128 + f] = pf;
-            pl_s[cg * 128 + f] = pl;
-            __syncthreads();
-            if (threadIdx.x < 128) merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
-            if (next) {
-                if (!(ok = wait_mma(bar, phase, a.meta))) break;  // GEMM1(t+1) done
-                fwd_e1<FMT>(tP, s1L, b1L, smem, cg, f);
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncthreads();
-                if (threadIdx.x == 0) {
-                    tc_fence_after();
-                    issue_gemm<NW>(tmem + 128, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_FWD_A, ACT_TERM,
-                                   FP / 16, id_mn);
-                    mma_commit(bar);
-                }
-            } else {
-                __syncthreads();
-            }
+            fwd_e2<TE>(tQ + c2 * 32, tm, rows_g, cc, ne, s2L, b2s, hv, a.out, f, pf, pl);
+            pf_s[cc * 128 + f] = pf;
+            pl_s[cc * 128 + f] = pl;
         }
+        group_sync(g);
+        if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
+        group_sync(g);          // merge done with tm and the partials before the next stage R
     }
-
-    if (ok) {
-        if (threadIdx.x < 128) {
-            a.out[(size_t)cur * FP + threadIdx.x] = acc;
-            for (int rr = cur + 1; rr < r1; ++rr) a.out[(size_t)rr * FP + threadIdx.x] = 0.f;
-        }
-    } else {
-        // drain: give in-flight MMAs a bounded chance to retire before freeing TMEM
-        mbar_wait_bounded(bar, phase, WAIT_POLLS);
+    if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
+    if (mt == 0) {
+        phases_s[g] = phase;
+        pend_s[g] = ok ? 0u : pending;
     }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 256);
-    }
+    const bool all_ok = __syncthreads_or(!ok) == 0;
+    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
@@ -589,10 +725,11 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 // ---------------------------------------------------------------------------
 // backward epilogue 1 for this warp's 32 edges: a = sp2(p), b = ssp'(x) dx/dd, with
 // p = x log2e = s1 log2e P + b1 log2e and dx/dd = s1 2ln2 P' (P' from the scaled
-// Gaussian-derivative operand).  ssp'(x) = 1 / (1 + e^-x) shares 2^-|p| with sp2.
-template <int FMT>
-__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* smem,
-                                       uint32_t col0, int f)
+// Gaussian-derivative rows).  ssp'(x) = 1 / (1 + e^-x) shares 2^-|p| with sp2.
+// a goes to B rows e, b to B rows TE + e of GEMM2's operand.
+template <int FMT, int TE>
+__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* op,
+                                       int col0, int f)
 {
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -612,9 +749,9 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
         }
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-            const uint32_t off = mnmajor_off(col0 + hh * 16 + g * 8, f, TILE_E);
-            store8<FMT>(smem + SM_X, smem + SM_X + ACT_TERM, off, r + g * 8);
-            store8<FMT>(smem + SM_BWD_Y, smem + SM_BWD_Y + ACT_TERM, off, rd + g * 8);
+            const int e = col0 + hh * 16 + g * 8;
+            store8<FMT>(op, op + ACT_TERM, mnmajor_off(e, f, MN), r + g * 8);
+            store8<FMT>(op, op + ACT_TERM, mnmajor_off(TE + e, f, MN), rd + g * 8);
         }
     }
 }
@@ -622,276 +759,220 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
 template <int FMT, int NW>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
+    constexpr int TE = TE_B;
+    constexpr int NCH = TE / 32;
+    using Meta = TileMeta<TE, true>;
     extern __shared__ __align__(1024) uint8_t smem[];
-    TileMeta* tm = reinterpret_cast<TileMeta*>(smem + SM_META_BWD);
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + SM_META_BWD + TILEMETA_BYTES);
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + SM_META_BWD + TILEMETA_BYTES + 8);
-    // after GEMM2 the ssp'(p)p' tile is dead: its space holds the partial sums and,
-    // behind them, the next tile's metadata until the merge has finished with tm
-    float* pf_s = reinterpret_cast<float*>(smem + SM_BWD_Y);
-    float* pl_s = pf_s + 4 * 128;
-    float* ps_s = pl_s + 4 * 128;   // [quadrant][edge] per-edge partial of s_e
-    TileMeta* tm_next = reinterpret_cast<TileMeta*>(smem + SM_BWD_Y + 8192);
+    Carry* cy = reinterpret_cast<Carry*>(smem + sm_carry<TE, true>());
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sm_bar<TE, true>());
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+    uint32_t* phases_s = tslot + 1;
+    uint32_t* pend_s = tslot + 3;
 
     if (a.meta->n_edges > a.cap) return;
     const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
     if (r0 >= r1) return;
     const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qd = warp & 3, cg = warp >> 2;
+    const int g = warp >> 3;
+    const int mt = threadIdx.x & (GT - 1);
+    const int qd = warp & 3, ch = (warp >> 2) & 1;  // TMEM lane quadrant, 32-edge chunk of the tile
     const int f = qd * 32 + lane;
 
-    if (warp == 0) {
-        tmem_alloc(tslot, 512);
-        tmem_relinquish();
-    }
-    if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-    }
-    copy_weights(smem, a.img);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tslot;
+    const uint32_t tmem = kernel_setup(smem, a, tslot, bars, cy, r0, 512);
+    uint8_t* op = smem + SM_OP + g * OP_BYTES;
+    Meta* tm = reinterpret_cast<Meta*>(smem + sm_meta<TE, true>() + g * sizeof(Meta));
+    float* pf_s = reinterpret_cast<float*>(op);     // after GEMM2: [chunk][feature] partials
+    float* pl_s = pf_s + NCH * 128;
+    float* ps_s = pl_s + NCH * 128;                 // [quadrant][edge] partial of s_e
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    const uint32_t col0 = cg * 32;
-    const uint32_t tP = tmem + lane_off + col0, tPd = tmem + 128 + lane_off + col0;
-    const uint32_t tQ = tmem + 256 + lane_off + col0, tQd = tmem + 384 + lane_off + col0;
+    const int col0 = ch * 32;
+    // accumulators (columns): [P | P'] at tb, [Q | Q'] at tb + 128 (64 each)
+    const uint32_t tb = tmem + g * 256;
+    const uint32_t tP = tb + lane_off + col0, tPd = tP + 64, tQ = tP + 128, tQd = tP + 192;
+    const uint32_t sop = smem_u32(op);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t id = idesc_f16(128, TILE_E, FMT, 0);
-    const uint32_t id_mn = idesc_f16(128, TILE_E, FMT, 1);
-
+    const uint32_t id = idesc_f16(128, MN, FMT, 0);
+    const uint32_t id_mn = idesc_f16(128, MN, FMT, 1);
     const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF, s1d = a.s1[f] * (2.0f * LN2F);
     const float s2 = a.s2[f], s2L = a.s2[f] * LN2F, b2s = a.b2s[f];
     const float* h_f = a.h + f;
     const float* u_f = a.u + f;
-    int cur = r0;
-    float acc = 0.f;
-    uint32_t phase = 0;
-    bool ok = true;
-    const int ntiles = (int)((e1 - e0 + TILE_E - 1) / TILE_E);
-    auto tile_ne = [&](int t) { return (int)min((long long)TILE_E, e1 - e0 - (long long)t * TILE_E); };
-    int cur_g = 0, nxt_g = 0;           // threads < 128: s_e slot of edge threadIdx.x (this / next tile)
-    float cur_so = 0.f, nxt_so = 0.f;
 
-    // Software pipeline: epilogue 2 of tile t runs while GEMM1 of tile t+1 runs.
-    if (ntiles > 0) {
-        EdgePre ep = prefetch_edge<true>(a, e0, tile_ne(0));
-        stage_rbf<FMT, true>(a, smem, tm, ep, tile_ne(0));
-        cur_g = ep.gidx;
-        cur_so = ep.sold;
-        if (ntiles > 1) ep = prefetch_edge<true>(a, e0 + TILE_E, tile_ne(1));
+    uint32_t phase = 0, pending = 0;   // pending: a commit of this group not yet waited for
+    bool ok = true, go_sent = false;
+    const int ntiles = (int)((e1 - e0 + TE - 1) / TE);
+    auto tile_ne = [&](int t) { return (int)min((long long)TE, e1 - e0 - (long long)t * TE); };
+
+    EdgePre ep;
+    if (g < ntiles) {
+        ep = prefetch_edge<TE, true>(a, e0 + (long long)g * TE, tile_ne(g), mt);
+        if (g == 1) ok = wait_group(&bars[3], 0u, true, false, a.meta, g, mt);   // start half a tile behind
+    }
+    for (int t = g; t < ntiles && ok; t += 2) {
+        const int ne = tile_ne(t);
+        const int32_t* rows_g = a.crow + e0 + (long long)t * TE;
+        stage_rbf<FMT, true, TE>(a, op, tm, ep, ne, mt);
+        const int my_g = ep.gidx;           // group threads < TE: s_e slot of edge mt of this tile
+        const float my_so = ep.sold;
+        if (t + 2 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(t + 2) * TE, tile_ne(t + 2), mt);
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
-        if (threadIdx.x == 0) {
+        group_sync(g);
+        if (mt == 0) {
             tc_fence_after();
-            issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
-            issue_gemm<NW>(tmem + 128, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X + 2 * RBF_TERM, RBF_TERM,
-                           KP / 16, id);
-            mma_commit(bar);
+            issue_gemm<NW>(tb, sbase + SM_W1, (uint32_t)W1_IMG, sop, RBF_TERM, KP / 16, id);
+            mma_commit(&bars[g]);
         }
-        ok = wait_mma(bar, phase, a.meta);
-        if (ok) {
-            bwd_e1<FMT>(tP, tPd, s1L, b1L, s1d, smem, col0, f);
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                tc_fence_after();
-                issue_gemm<NW>(tmem + 256, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_X, ACT_TERM, FP / 16, id_mn);
-                issue_gemm<NW>(tmem + 384, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_BWD_Y, ACT_TERM, FP / 16,
-                               id_mn);
-                mma_commit(bar);
-            }
+        pending = 1;
+        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM1 done
+        pending = 0;
+        if (g == 0 && !go_sent) {
+            if (mt == 0) mbar_arrive(&bars[3]);
+            go_sent = true;
         }
-        for (int t = 0; t < ntiles && ok; ++t) {
-            const int ne = tile_ne(t);
-            const bool next = t + 1 < ntiles;
-            const long long t0 = e0 + (long long)t * TILE_E;
-            const int eb = (int)col0;
-            float uv[16], hv[16];
-            gather<16>(u_f, tm, eb, uv);
-            gather<16>(h_f, tm, eb, hv);
-            if (!(ok = wait_mma(bar, phase, a.meta))) break;            // GEMM2(t) done
-            if (next) {
-                // Gaussians of the next tile into the (now dead) ssp(p) region; its metadata is staged
-                stage_rbf<FMT, true>(a, smem, tm_next, ep, tile_ne(t + 1));
-                nxt_g = ep.gidx;
-                nxt_so = ep.sold;
-                if (t + 2 < ntiles) ep = prefetch_edge<true>(a, e0 + (long long)(t + 2) * TILE_E, tile_ne(t + 2));
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncthreads();
-                if (threadIdx.x == 0) {
-                    tc_fence_after();
-                    issue_gemm<NW>(tmem, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X, RBF_TERM, KP / 16, id);
-                    issue_gemm<NW>(tmem + 128, sbase + SM_W1, (uint32_t)W1_IMG, sbase + SM_X + 2 * RBF_TERM,
-                                   RBF_TERM, KP / 16, id);
-                    mma_commit(bar);
-                }
-            }
-            // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 ln2 Q + b2s, z' = s2 Q')
-            {
-                const bool active = eb < ne;
-                const ChunkInfo ci = tm->c[cg];
-                // 1: one row in the chunk; 2: two rows (the first a prefix); 3: the general
-                // serial segmented sum with a row change test per edge
-                const int kind = !active ? 0 : ci.other ? 3 : (ci.rfirst == ci.rlast ? 1 : 2);
-                float pf = 0.f, pl = 0.f;
-                if (kind != 0) {
-                    const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
-                    const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
-                    float sf = 0.f, sl = 0.f;
-                    ChunkSeg c{0, 0, 0.f, 0.f};
-                    if (kind == 3) seg_begin(c, tm, eb);
-                    float u_row = u_first;
+        bwd_e1<FMT, TE>(tP, tPd, s1L, b1L, s1d, op, col0, f);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        group_sync(g);
+        if (mt == 0) {
+            tc_fence_after();
+            issue_gemm<NW>(tb + 128, sbase + SM_W2, (uint32_t)W2_IMG, sop, ACT_TERM, FP / 16, id_mn);
+            mma_commit(&bars[g]);
+        }
+        pending = 1;
+        const int eb = col0;
+        float uv[16], hv[16];
+        gather<16>(u_f, tm->col, eb, uv);                                // under GEMM2
+        gather<16>(h_f, tm->col, eb, hv);
+        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2 done
+        pending = 0;
+        // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 ln2 Q + b2s, z' = s2 Q')
+        {
+            const bool active = eb < ne;
+            const ChunkInfo ci = tm->c[ch];
+            // 1: one row in the chunk; 2: two rows (the first a prefix); 3: the general
+            // serial segmented sum with a row change test per edge
+            const int kind = !active ? 0 : ci.other ? 3 : (ci.rfirst == ci.rlast ? 1 : 2);
+            float pf = 0.f, pl = 0.f;
+            if (kind != 0) {
+                const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
+                const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
+                float sf = 0.f, sl = 0.f;
+                ChunkSeg c;
+                seg_begin(c, ci.rfirst);
+                float u_row = u_first;
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        if (hh == 1) {
-                            gather<16>(u_f, tm, eb + 16, uv);
-                            gather<16>(h_f, tm, eb + 16, hv);
-                        }
-                        float r[16], rd[16];
-                        tmem_ld16(tQ + hh * 16, r);
-                        tmem_ld16(tQd + hh * 16, rd);
-                        tmem_ld_wait();
-                        const float* fcp = tm->fc + eb + hh * 16;
-                        const float* dfcp = tm->dfc + eb + hh * 16;
-                        if (kind == 1) {
-#pragma unroll
-                            for (int g = 0; g < 16; g += 4) {
-                                float fc[4], dfc[4];
-                                load_edges<4>(fcp, g, fc);
-                                load_edges<4>(dfcp, g, dfc);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const int q = g + i;
-                                    const float z = fmaf(s2L, r[q], b2s);
-                                    sf = fmaf(fc[i] * z, uv[q], sf);
-                                    const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
-                                    rd[q] = wd * (u_first * hv[q]);
-                                }
-                            }
-                        } else if (kind == 2) {
-#pragma unroll
-                            for (int g = 0; g < 16; g += 4) {
-                                float fc[4], dfc[4];
-                                load_edges<4>(fcp, g, fc);
-                                load_edges<4>(dfcp, g, dfc);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const int q = g + i;
-                                    const float z = fmaf(s2L, r[q], b2s);
-                                    const float dt = fc[i] * z * uv[q];
-                                    const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
-                                    sf += first ? dt : 0.f;
-                                    sl += first ? 0.f : dt;
-                                    const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
-                                    rd[q] = wd * ((first ? u_first : u_last) * hv[q]);
-                                }
-                            }
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 16; ++q) {
-                                const int e = eb + hh * 16 + q;
-                                float tval = 0.f;
-                                if (e < ne) {
-                                    const int row = tm->row[e];
-                                    if (row != c.lrow) {
-                                        seg_row(c, row, a.out, f);
-                                        u_row = __ldg(u_f + (size_t)row * FP);
-                                    }
-                                    const float fcq = fcp[q], dfcq = dfcp[q];
-                                    const float z = fmaf(s2L, r[q], b2s);
-                                    const float wd = fmaf(dfcq, z, fcq * (s2 * rd[q]));
-                                    c.acc = fmaf(fcq * z, uv[q], c.acc);
-                                    tval = wd * (u_row * hv[q]);
-                                }
-                                rd[q] = tval;
-                            }
-                        }
-                        // transpose-reduce the 16 per-edge values over the warp's 32 features:
-                        // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
-#pragma unroll
-                        for (int sh = 16; sh >= 2; sh >>= 1) {
-                            const bool upper = (lane & sh) != 0;
-#pragma unroll
-                            for (int k = 0; k < sh / 2; ++k) {
-                                float send = upper ? rd[k] : rd[k + sh / 2];
-                                float keep = upper ? rd[k + sh / 2] : rd[k];
-                                rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
-                            }
-                        }
-                        rd[0] += __shfl_xor_sync(0xffffffffu, rd[0], 1);
-                        if ((lane & 1) == 0) ps_s[qd * TILE_E + eb + hh * 16 + (lane >> 1)] = rd[0];
+                for (int hh = 0; hh < 2; ++hh) {
+                    if (hh == 1) {
+                        gather<16>(u_f, tm->col, eb + 16, uv);
+                        gather<16>(h_f, tm->col, eb + 16, hv);
                     }
+                    float r[16], rd[16];
+                    tmem_ld16(tQ + hh * 16, r);
+                    tmem_ld16(tQd + hh * 16, rd);
+                    tmem_ld_wait();
+                    const float* fcp = tm->fc + eb + hh * 16;
+                    const float* dfcp = tm->dfc + eb + hh * 16;
                     if (kind == 1) {
-                        pf = sf;
+#pragma unroll
+                        for (int gq = 0; gq < 16; gq += 4) {
+                            float fc[4], dfc[4];
+                            load_edges<4>(fcp, gq, fc);
+                            load_edges<4>(dfcp, gq, dfc);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int q = gq + i;
+                                const float z = fmaf(s2L, r[q], b2s);
+                                sf = fmaf(fc[i] * z, uv[q], sf);
+                                const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
+                                rd[q] = wd * (u_first * hv[q]);
+                            }
+                        }
                     } else if (kind == 2) {
-                        pf = sf;
-                        pl = sl;
-                        for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
-                    } else if (c.lrow == c.rfirst) {
-                        pf = c.acc;
+#pragma unroll
+                        for (int gq = 0; gq < 16; gq += 4) {
+                            float fc[4], dfc[4];
+                            load_edges<4>(fcp, gq, fc);
+                            load_edges<4>(dfcp, gq, dfc);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int q = gq + i;
+                                const float z = fmaf(s2L, r[q], b2s);
+                                const float dt = fc[i] * z * uv[q];
+                                const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
+                                sf += first ? dt : 0.f;
+                                sl += first ? 0.f : dt;
+                                const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
+                                rd[q] = wd * ((first ? u_first : u_last) * hv[q]);
+                            }
+                        }
                     } else {
-                        pf = c.pf;
-                        pl = c.acc;
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const int e = eb + hh * 16 + q;
+                            float tval = 0.f;
+                            if (e < ne) {
+                                const int row = __ldg(rows_g + e);
+                                if (row != c.lrow) {
+                                    seg_row(c, row, a.out, f);
+                                    u_row = __ldg(u_f + (size_t)row * FP);
+                                }
+                                const float fcq = fcp[q], dfcq = dfcp[q];
+                                const float z = fmaf(s2L, r[q], b2s);
+                                const float wd = fmaf(dfcq, z, fcq * (s2 * rd[q]));
+                                c.acc = fmaf(fcq * z, uv[q], c.acc);
+                                tval = wd * (u_row * hv[q]);
+                            }
+                            rd[q] = tval;
+                        }
                     }
+                    // transpose-reduce the 16 per-edge values over the warp's 32 features:
+                    // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
+#pragma unroll
+                    for (int sh = 16; sh >= 2; sh >>= 1) {
+                        const bool upper = (lane & sh) != 0;
+#pragma unroll
+                        for (int k = 0; k < sh / 2; ++k) {
+                            float send = upper ? rd[k] : rd[k + sh / 2];
+                            float keep = upper ? rd[k + sh / 2] : rd[k];
+                            rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+                        }
+                    }
+                    rd[0] += __shfl_xor_sync(0xffffffffu, rd[0], 1);
+                    if ((lane & 1) == 0) ps_s[qd * TE + eb + hh * 16 + (lane >> 1)] = rd[0];
                 }
-                pf_s[cg * 128 + f] = pf;
-                pl_s[cg * 128 + f] = pl;
-            }
-            __syncthreads();
-            if (threadIdx.x < 128) {
-                merge_chunks(tm, pf_s, pl_s, ne, threadIdx.x, a.out, cur, acc);
-                if ((int)threadIdx.x < ne) {
-                    const int q = threadIdx.x;
-                    const float sv = ps_s[q] + ps_s[TILE_E + q] + ps_s[2 * TILE_E + q] + ps_s[3 * TILE_E + q];
-                    a.s_edge[cur_g] = a.accumulate_s ? cur_so + sv : sv;
+                if (kind == 1) {
+                    pf = sf;
+                } else if (kind == 2) {
+                    pf = sf;
+                    pl = sl;
+                    for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
+                } else if (c.lrow == c.rfirst) {
+                    pf = c.acc;
+                } else {
+                    pf = c.pf;
+                    pl = c.acc;
                 }
             }
-            if (next) {
-                __syncthreads();                                        // merge done with tm
-                for (int i = threadIdx.x; i < (int)(sizeof(TileMeta) / 4); i += NT)
-                    reinterpret_cast<uint32_t*>(tm)[i] = reinterpret_cast<const uint32_t*>(tm_next)[i];
-                cur_g = nxt_g;
-                cur_so = nxt_so;
-                if (!(ok = wait_mma(bar, phase, a.meta))) break;        // GEMM1(t+1) done
-                bwd_e1<FMT>(tP, tPd, s1L, b1L, s1d, smem, col0, f);
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncthreads();
-                if (threadIdx.x == 0) {
-                    tc_fence_after();
-                    issue_gemm<NW>(tmem + 256, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_X, ACT_TERM, FP / 16,
-                                   id_mn);
-                    issue_gemm<NW>(tmem + 384, sbase + SM_W2, (uint32_t)W2_IMG, sbase + SM_BWD_Y, ACT_TERM, FP / 16,
-                                   id_mn);
-                    mma_commit(bar);
-                }
-            } else {
-                __syncthreads();
-            }
+            pf_s[ch * 128 + f] = pf;
+            pl_s[ch * 128 + f] = pl;
         }
-    }
-
-    if (ok) {
-        if (threadIdx.x < 128) {
-            a.out[(size_t)cur * FP + threadIdx.x] = acc;
-            for (int rr = cur + 1; rr < r1; ++rr) a.out[(size_t)rr * FP + threadIdx.x] = 0.f;
+        group_sync(g);
+        if (mt < ne) {
+            const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];
+            a.s_edge[my_g] = a.accumulate_s ? my_so + sv : sv;
         }
-    } else {
-        mbar_wait_bounded(bar, phase, WAIT_POLLS);
+        if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
+        group_sync(g);          // merge and s_e done with tm and the partials before the next stage R
     }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
+    if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
+    if (mt == 0) {
+        phases_s[g] = phase;
+        pend_s[g] = ok ? 0u : pending;
     }
+    const bool all_ok = __syncthreads_or(!ok) == 0;
+    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
@@ -983,6 +1064,7 @@ static MPArgs make_args(schnet_ctx* c, int layer)
     a.inv_rc = 1.0f / c->cfg.cutoff;
     a.mu0 = c->mu0;
     a.dmu = c->dmu;
+    a.K = c->K;
     a.ngc = (float)(-1.4426950408889634 / (2.0 * (double)c->cfg.rbf_sigma * (double)c->cfg.rbf_sigma));
     a.img = w.img + (size_t)layer * LAYER_IMG;
     a.s1 = w.s1 + layer * FP;
@@ -1001,9 +1083,10 @@ template <int FMT, int NW>
 static cudaError_t set_attrs()
 {
     cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_FWD);
+                                         (int)smem_bytes<TE_F, false>());
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BWD);
+    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_bytes<TE_B, true>());
 }
 
 cudaError_t cfconv_init_attributes()
@@ -1019,11 +1102,11 @@ cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
     MPArgs a = make_args(c, layer);
     a.out = c->ws.m;
     if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_fwd<0, 2><<<c->ncta, NT, SMEM_FWD, c->s>>>(a);
+        k_cfconv_fwd<0, 2><<<c->ncta, NT, smem_bytes<TE_F, false>(), c->s>>>(a);
     else if (c->weight_fmt == 0)
-        k_cfconv_fwd<0, 1><<<c->ncta, NT, SMEM_FWD, c->s>>>(a);
+        k_cfconv_fwd<0, 1><<<c->ncta, NT, smem_bytes<TE_F, false>(), c->s>>>(a);
     else
-        k_cfconv_fwd<1, 1><<<c->ncta, NT, SMEM_FWD, c->s>>>(a);
+        k_cfconv_fwd<1, 1><<<c->ncta, NT, smem_bytes<TE_F, false>(), c->s>>>(a);
     c->launches += 1;
     return cudaGetLastError();
 }
@@ -1034,11 +1117,11 @@ cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s)
     a.out = c->ws.dh;
     a.accumulate_s = accumulate_s;
     if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_bwd<0, 2><<<c->ncta, NT, SMEM_BWD, c->s>>>(a);
+        k_cfconv_bwd<0, 2><<<c->ncta, NT, smem_bytes<TE_B, true>(), c->s>>>(a);
     else if (c->weight_fmt == 0)
-        k_cfconv_bwd<0, 1><<<c->ncta, NT, SMEM_BWD, c->s>>>(a);
+        k_cfconv_bwd<0, 1><<<c->ncta, NT, smem_bytes<TE_B, true>(), c->s>>>(a);
     else
-        k_cfconv_bwd<1, 1><<<c->ncta, NT, SMEM_BWD, c->s>>>(a);
+        k_cfconv_bwd<1, 1><<<c->ncta, NT, smem_bytes<TE_B, true>(), c->s>>>(a);
     c->launches += 1;
     return cudaGetLastError();
 }

@@ -70,16 +70,19 @@ constexpr int MN = 128;                  // GEMM N of every MMA
 constexpr int TE_F = 128;                // forward: edges per tile
 constexpr int TE_B = 64;                 // backward: edges per tile (B rows 64..127 hold their derivatives)
 
+// TMEM columns (512 allocated): each group's accumulator (P, then Q over it), and
+// the filter weights as the MMAs' A operand, one row (output channel) per lane,
+// two 16-bit K elements per 32-bit column.
+constexpr uint32_t TM_ACC = 128;         // group g: columns g*128 .. g*128+127
+constexpr uint32_t TM_W1H = 256, TM_W1L = 288, TM_W2H = 320, TM_W2L = 384;
+
 // shared-memory map (bytes)
-constexpr uint32_t SM_W1 = 0;            // W1^T hi, lo   2 x 16 KB  (shared by both groups)
-constexpr uint32_t SM_W2 = 32768;        // W2^T hi, lo   2 x 32 KB
-constexpr uint32_t SM_OP = 98304;        // per-group operand regions
 constexpr uint32_t RBF_TERM = MN * KP * 2;   // 16 KB: one 16-bit term of a [128 x 64] GEMM1 B tile
 constexpr uint32_t ACT_TERM = MN * FP * 2;   // 32 KB: one 16-bit term of a [128 x 128] GEMM2 B tile
-// Per group: GEMM2's B operand hi/lo (64 KB); GEMM1's B operand hi/lo (32 KB)
-// overlays its start; after GEMM2 the region is dead and holds the partial sums.
-constexpr uint32_t OP_BYTES = 2 * ACT_TERM;
-constexpr uint32_t CARRY_BYTES = FP * 4 + 16;                // carried partial per feature + row (x2)
+constexpr uint32_t SM_RBF = 0;               // group g: GEMM1 B operand hi/lo at g * 32 KB
+constexpr uint32_t SM_ACT = 65536;           // group g: GEMM2 B operand hi/lo at 64 KB + g * 64 KB;
+                                             //   after GEMM2 it holds the epilogue's partial sums
+constexpr uint32_t CARRY_BYTES = FP * 4 + 16;  // carried partial per feature + row (x2)
 constexpr uint32_t BAR_BYTES = 64;
 constexpr uint32_t WAIT_POLLS = 1u << 22;
 
@@ -106,8 +109,10 @@ struct TileMeta {
     ChunkInfo c[TE / 32];
 };
 
-template <int TE, bool BWD> constexpr uint32_t sm_meta() { return SM_OP + 2 * OP_BYTES; }
-template <int TE, bool BWD> constexpr uint32_t sm_carry() { return sm_meta<TE, BWD>() + 2 * sizeof(TileMeta<TE, BWD>); }
+// metadata: [group][buffer] (double-buffered per group: stage R of tile t+2
+// fills one while the epilogue and merge of tile t read the other)
+template <int TE, bool BWD> constexpr uint32_t sm_meta() { return SM_ACT + 2 * 2 * ACT_TERM; }
+template <int TE, bool BWD> constexpr uint32_t sm_carry() { return sm_meta<TE, BWD>() + 4 * sizeof(TileMeta<TE, BWD>); }
 template <int TE, bool BWD> constexpr uint32_t sm_bar() { return sm_carry<TE, BWD>() + CARRY_BYTES; }
 template <int TE, bool BWD> constexpr uint32_t smem_bytes() { return sm_bar<TE, BWD>() + BAR_BYTES; }
 // barrier block: [0] group 0 MMA commits, [1] group 1 MMA commits, [2] merge token,
@@ -116,6 +121,7 @@ template <int TE, bool BWD> constexpr uint32_t smem_bytes() { return sm_bar<TE, 
 static_assert(smem_bytes<TE_F, false>() <= 232448, "forward shared memory exceeds the per-block limit");
 static_assert(smem_bytes<TE_B, true>() <= 232448, "backward shared memory exceeds the per-block limit");
 static_assert(sizeof(TileMeta<TE_F, false>) % 16 == 0 && sizeof(TileMeta<TE_B, true>) % 16 == 0, "meta alignment");
+static_assert(2 * RBF_TERM * 2 <= SM_ACT, "GEMM1 operands");
 
 // Segment-sum state carried from one tile to the next (in tile order, across
 // the two groups): the open row and its partial sum per feature.  The row is
@@ -127,13 +133,6 @@ struct Carry {
     int32_t pad[2];
 };
 static_assert(sizeof(Carry) == CARRY_BYTES, "carry layout");
-
-__device__ __forceinline__ void copy_weights(uint8_t* smem, const uint8_t* __restrict__ img)
-{
-    const uint4* src = reinterpret_cast<const uint4*>(img);
-    uint4* dst = reinterpret_cast<uint4*>(smem + SM_W1);
-    for (int i = threadIdx.x; i < (int)(LAYER_IMG / 16); i += blockDim.x) dst[i] = __ldg(src + i);
-}
 
 // named barrier of math group g (ids 1 and 2; id 0 is __syncthreads)
 __device__ __forceinline__ void group_sync(int g)
@@ -159,6 +158,50 @@ __device__ __forceinline__ bool group_or(int g, bool v)
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar)
 {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16 (A read from tensor memory)
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this warp's 32 lanes <- 32 registers per thread
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+// Row f of one packed weight term (the K-major core-matrix image: K elements
+// 8kg .. 8kg+7 of row f are the 16 bytes at kg * 2048 + f * 16) into 32 TMEM
+// columns starting at `col` (K elements 64 * half .. 64 * half + 63).
+__device__ __forceinline__ void weights_to_tmem(uint32_t taddr_lane, uint32_t col, const uint8_t* __restrict__ term,
+                                                int f, int half)
+{
+    uint32_t v[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(term + (size_t)(half * 8 + q) * (FP * 16) + f * 16));
+        v[4 * q] = x.x;
+        v[4 * q + 1] = x.y;
+        v[4 * q + 2] = x.z;
+        v[4 * q + 3] = x.w;
+    }
+    tmem_st32(taddr_lane + col + half * 32, v);
 }
 
 // two fp32 values -> packed 16-bit hi pair and lo (residual) pair
@@ -212,7 +255,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
         : "r"(taddr));
 }
 
-// Endpoints of edge (group thread mod TE) of a tile, loaded one tile ahead so the
+// Endpoints of edge (group thread mod TE) of a tile, loaded a tile ahead so the
 // dependent loads (edge -> atom -> position) overlap the previous tile's work.
 struct EdgePre {
     int i, j;
@@ -252,7 +295,7 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
 // as zeros without evaluating them; masked or padding edges have
 // f_c = f_c' = 0, so their Gaussians need no mask (they stay finite).
 template <int FMT, bool BWD, int TE>
-__device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* op, TileMeta<TE, BWD>* tmeta, const EdgePre& ep,
+__device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMeta<TE, BWD>* tmeta, const EdgePre& ep,
                                           int ne, int mt)
 {
     constexpr int TPE = GT / TE;         // threads per edge
@@ -287,8 +330,8 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* op, TileMeta
         const int oth = __any_sync(0xffffffffu, e < ne && row != rfirst && row != rlast);
         if (lane == 0) tmeta->c[w] = ChunkInfo{rfirst, rlast, fm, oth};
     }
-    uint8_t* b_hi = op;
-    uint8_t* b_lo = op + RBF_TERM;
+    uint8_t* b_hi = rbf;
+    uint8_t* b_lo = rbf + RBF_TERM;
     const float dm = d - fmaf((float)(kq * KPT), a.dmu, a.mu0);   // d - mu of this thread's first Gaussian
 #pragma unroll
     for (int g = 0; g < KPT / 8; ++g) {
@@ -315,20 +358,19 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* op, TileMeta
 }
 
 // Issue D (+)= W^T * B over `ksteps` K-steps of 16 with the hi/lo split
-// (A: 128 feature rows, B: MN = 128 rows; no-swizzle core matrices).
+// (A: the weight term in TMEM, 8 columns per K-step; B: MN = 128 rows in
+// shared memory, no-swizzle core matrices).
 template <int NW>
-__device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_base, uint32_t a_term, uint32_t b_base,
+__device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_hi_t, uint32_t a_lo_t, uint32_t b_base,
                                            uint32_t b_term, int ksteps, uint32_t idesc)
 {
     for (int ks = 0; ks < ksteps; ++ks) {
-        const uint32_t koff = (uint32_t)ks * 2u * (uint32_t)(FP * 16);   // 2 core matrices of 8 along K
-        uint64_t a_hi = smem_desc(a_base + koff, FP * 16, 128);
-        uint64_t a_lo = smem_desc(a_base + a_term + koff, FP * 16, 128);
-        uint64_t b_hi = smem_desc(b_base + koff, MN * 16, 128);
-        uint64_t b_lo = smem_desc(b_base + b_term + koff, MN * 16, 128);
-        mma_f16(d_tmem, a_hi, b_hi, idesc, ks > 0 ? 1u : 0u);
-        if (NW == 2) mma_f16(d_tmem, a_lo, b_hi, idesc, 1u);
-        mma_f16(d_tmem, a_hi, b_lo, idesc, 1u);
+        const uint32_t koff = (uint32_t)ks * 2u * (uint32_t)(MN * 16);   // 2 core matrices of 8 along K
+        const uint64_t b_hi = smem_desc(b_base + koff, MN * 16, 128);
+        const uint64_t b_lo = smem_desc(b_base + b_term + koff, MN * 16, 128);
+        mma_f16_ts(d_tmem, a_hi_t + ks * 8, b_hi, idesc, ks > 0 ? 1u : 0u);
+        if (NW == 2) mma_f16_ts(d_tmem, a_lo_t + ks * 8, b_hi, idesc, 1u);
+        mma_f16_ts(d_tmem, a_hi_t + ks * 8, b_lo, idesc, 1u);
     }
 }
 
@@ -519,14 +561,14 @@ __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_
     if (c.lrow == c.rfirst) { pf = c.acc; pl = 0.f; } else { pf = c.pf; pl = c.acc; }
 }
 
-// Common prologue of both kernels: TMEM allocation, mbarriers, weights into
-// shared memory, the initial carry.  Returns the TMEM base address.
-__device__ __forceinline__ uint32_t kernel_setup(uint8_t* smem, const MPArgs& a, uint32_t* tslot, uint64_t* bars,
-                                                 Carry* cy, int r0, uint32_t ncols)
+// Common prologue of both kernels: TMEM allocation, mbarriers, the filter
+// weights into TMEM (warps 0-3, one output channel per lane), the initial
+// carry.  Returns the TMEM base address.
+__device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslot, uint64_t* bars, Carry* cy, int r0)
 {
     const int warp = threadIdx.x >> 5;
     if (warp == 0) {
-        tmem_alloc(tslot, ncols);
+        tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     if (threadIdx.x == 0) {
@@ -538,18 +580,31 @@ __device__ __forceinline__ uint32_t kernel_setup(uint8_t* smem, const MPArgs& a,
         cy->cur[1] = r0;             // tile 0 reads the carry of "tile -1"
     }
     if (threadIdx.x < FP) cy->acc[threadIdx.x] = 0.f;
-    copy_weights(smem, a.img);
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    return *tslot;
+    const uint32_t tmem = *tslot;
+    if (warp < 4) {
+        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+        const int f = threadIdx.x;
+        weights_to_tmem(tl, TM_W1H, a.img, f, 0);
+        weights_to_tmem(tl, TM_W1L, a.img + W1_IMG, f, 0);
+        weights_to_tmem(tl, TM_W2H, a.img + 2 * W1_IMG, f, 0);
+        weights_to_tmem(tl, TM_W2H, a.img + 2 * W1_IMG, f, 1);
+        weights_to_tmem(tl, TM_W2L, a.img + 2 * W1_IMG + W2_IMG, f, 0);
+        weights_to_tmem(tl, TM_W2L, a.img + 2 * W1_IMG + W2_IMG, f, 1);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return tmem;
 }
 
 // Common epilogue: the carried row is complete; rows after it without edges are zero.
 __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r1, float* __restrict__ out, bool ok,
                                               uint64_t* bars, const uint32_t* phases, const uint32_t* pending,
-                                              uint32_t tmem, uint32_t ncols)
+                                              uint32_t tmem)
 {
     const int warp = threadIdx.x >> 5;
     if (ok) {
@@ -567,7 +622,7 @@ __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, ncols);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -575,7 +630,7 @@ __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r
 // operand (the base-2 softplus; ssp = ln2 (a - 1), with ln2 and the shift folded
 // into the second layer's scale and bias)
 template <int FMT>
-__device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_t* op, int e0, int f)
+__device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_t* act, int e0, int f)
 {
     float r[32];
     tmem_ld32(tP, r);
@@ -585,7 +640,7 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         const uint32_t off = mnmajor_off(e0 + g * 8, f, MN);
-        store8<FMT>(op, op + ACT_TERM, off, r + g * 8);
+        store8<FMT>(act, act + ACT_TERM, off, r + g * 8);
     }
 }
 
@@ -610,9 +665,21 @@ __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* t
     chunk_partials<32>(tm->c[cc], rows_g, eb, ne, r, out, f, pf, pl);
 }
 
+// Issue GEMM1 of a tile (group g): D = W1^T [B rows of the group's GEMM1 operand]
+template <int NW>
+__device__ __forceinline__ void issue_gemm1(uint32_t tmem, uint32_t dacc, uint32_t srbf, uint32_t id, uint64_t* bar)
+{
+    tc_fence_after();
+    issue_gemm<NW>(dacc, tmem + TM_W1H, tmem + TM_W1L, srbf, RBF_TERM, KP / 16, id);
+    mma_commit(bar);
+}
+
 // ---------------------------------------------------------------------------
 // forward: m_i = sum_j h_j (.) W(d_ij)
 // ---------------------------------------------------------------------------
+// Per group and tile t: [GEMM1(t) in flight] E1 -> issue GEMM2 -> stage R of
+// t+2 (into the group's own GEMM1 operand and second metadata buffer) and the
+// first gather under GEMM2 -> E2 -> issue GEMM1(t+2) -> merge under GEMM1(t+2).
 template <int FMT, int NW>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {
@@ -636,16 +703,15 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     const int qd = warp & 3, ch = (warp >> 2) & 1;  // TMEM lane quadrant, 64-edge half of the tile
     const int f = qd * 32 + lane;                   // this thread's output feature
 
-    const uint32_t tmem = kernel_setup(smem, a, tslot, bars, cy, r0, 512);
-    uint8_t* op = smem + SM_OP + g * OP_BYTES;
-    Meta* tm = reinterpret_cast<Meta*>(smem + sm_meta<TE, false>() + g * sizeof(Meta));
-    float* pf_s = reinterpret_cast<float*>(op);     // after GEMM2: [chunk][feature] partials
+    const uint32_t tmem = kernel_setup(a, tslot, bars, cy, r0);
+    uint8_t* rbf = smem + SM_RBF + g * 2 * RBF_TERM;
+    uint8_t* act = smem + SM_ACT + g * 2 * ACT_TERM;
+    Meta* tmb = reinterpret_cast<Meta*>(smem + sm_meta<TE, false>() + g * 2 * sizeof(Meta));
+    float* pf_s = reinterpret_cast<float*>(act);    // after GEMM2: [chunk][feature] partials
     float* pl_s = pf_s + NCH * 128;
-    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-    const uint32_t dP = tmem + g * 256, dQ = dP + 128;          // accumulators: P, then Q, 128 columns each
-    const uint32_t tP = dP + lane_off + ch * 64, tQ = dQ + lane_off + ch * 64;
-    const uint32_t sop = smem_u32(op);
-    const uint32_t sbase = smem_u32(smem);
+    const uint32_t dacc = tmem + g * TM_ACC;        // P, then Q over it (128 columns)
+    const uint32_t tA = dacc + ((uint32_t)(qd * 32) << 16) + ch * 64;
+    const uint32_t srbf = smem_u32(rbf), sact = smem_u32(act);
     const uint32_t id = idesc_f16(128, MN, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, MN, FMT, 1);
     const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF;
@@ -659,57 +725,64 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 
     EdgePre ep;
     if (g < ntiles) {
-        ep = prefetch_edge<TE, false>(a, e0 + (long long)g * TE, tile_ne(g), mt);
         if (g == 1) ok = wait_group(&bars[3], 0u, true, false, a.meta, g, mt);   // start half a tile behind
-    }
-    for (int t = g; t < ntiles && ok; t += 2) {
-        const int ne = tile_ne(t);
-        const int32_t* rows_g = a.crow + e0 + (long long)t * TE;
-        // stage R: Gaussians of this tile into the group's operand region
-        stage_rbf<FMT, false, TE>(a, op, tm, ep, ne, mt);
-        if (t + 2 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(t + 2) * TE, tile_ne(t + 2), mt);
+        ep = prefetch_edge<TE, false>(a, e0 + (long long)g * TE, tile_ne(g), mt);
+        stage_rbf<FMT, false, TE>(a, rbf, tmb, ep, tile_ne(g), mt);
+        if (g + 2 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(g + 2) * TE, tile_ne(g + 2), mt);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
-        if (mt == 0) {
-            tc_fence_after();
-            issue_gemm<NW>(dP, sbase + SM_W1, (uint32_t)W1_IMG, sop, RBF_TERM, KP / 16, id);
-            mma_commit(&bars[g]);
-        }
-        pending = 1;
-        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM1 done
+        if (ok && mt == 0) issue_gemm1<NW>(tmem, dacc, srbf, id, &bars[g]);
+        pending = ok ? 1 : 0;
+    }
+    int buf = 0;
+    for (int t = g; t < ntiles && ok; t += 2, buf ^= 1) {
+        const int ne = tile_ne(t);
+        const bool next = t + 2 < ntiles;
+        Meta* tm = tmb + buf;
+        const int32_t* rows_g = a.crow + e0 + (long long)t * TE;
+        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM1(t) done
         pending = 0;
         if (g == 0 && !go_sent) {
             if (mt == 0) mbar_arrive(&bars[3]);
             go_sent = true;
         }
 #pragma unroll 1
-        for (int c2 = 0; c2 < 2; ++c2) fwd_e1<FMT>(tP + c2 * 32, s1L, b1L, op, ch * 64 + c2 * 32, f);
+        for (int c2 = 0; c2 < 2; ++c2) fwd_e1<FMT>(tA + c2 * 32, s1L, b1L, act, ch * 64 + c2 * 32, f);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
         if (mt == 0) {
             tc_fence_after();
-            issue_gemm<NW>(dQ, sbase + SM_W2, (uint32_t)W2_IMG, sop, ACT_TERM, FP / 16, id_mn);
+            issue_gemm<NW>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, FP / 16, id_mn);
             mma_commit(&bars[g]);
         }
         pending = 1;
+        // under GEMM2: stage R of tile t+2 and the first gather of this tile
+        if (next) {
+            stage_rbf<FMT, false, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), mt);
+            if (t + 4 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(t + 4) * TE, tile_ne(t + 4), mt);
+            fence_proxy_async_smem();
+        }
         float hv[32];
-        gather<32>(h_f, tm->col, ch * 64, hv);                          // under GEMM2
-        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2 done
+        gather<32>(h_f, tm->col, ch * 64, hv);
+        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2(t) done
         pending = 0;
 #pragma unroll 1
         for (int c2 = 0; c2 < 2; ++c2) {
             const int cc = ch * 2 + c2;
             if (c2 == 1) gather<32>(h_f, tm->col, cc * 32, hv);
             float pf, pl;
-            fwd_e2<TE>(tQ + c2 * 32, tm, rows_g, cc, ne, s2L, b2s, hv, a.out, f, pf, pl);
+            fwd_e2<TE>(tA + c2 * 32, tm, rows_g, cc, ne, s2L, b2s, hv, a.out, f, pf, pl);
             pf_s[cc * 128 + f] = pf;
             pl_s[cc * 128 + f] = pl;
         }
-        group_sync(g);
+        tc_fence_before();
+        group_sync(g);          // Q read out; partials and the next tile's Gaussians in place
+        if (next && mt == 0) issue_gemm1<NW>(tmem, dacc, srbf, id, &bars[g]);
+        if (next) pending = 1;
         if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
-        group_sync(g);          // merge done with tm and the partials before the next stage R
+        group_sync(g);          // merge done with the partials before E1 of the next tile overwrites them
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
     if (mt == 0) {
@@ -717,7 +790,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         pend_s[g] = ok ? 0u : pending;
     }
     const bool all_ok = __syncthreads_or(!ok) == 0;
-    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, 512);
+    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem);
 }
 
 // ---------------------------------------------------------------------------
@@ -728,7 +801,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 // Gaussian-derivative rows).  ssp'(x) = 1 / (1 + e^-x) shares 2^-|p| with sp2.
 // a goes to B rows e, b to B rows TE + e of GEMM2's operand.
 template <int FMT, int TE>
-__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* op,
+__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* act,
                                        int col0, int f)
 {
 #pragma unroll
@@ -750,8 +823,8 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
             const int e = col0 + hh * 16 + g * 8;
-            store8<FMT>(op, op + ACT_TERM, mnmajor_off(e, f, MN), r + g * 8);
-            store8<FMT>(op, op + ACT_TERM, mnmajor_off(TE + e, f, MN), rd + g * 8);
+            store8<FMT>(act, act + ACT_TERM, mnmajor_off(e, f, MN), r + g * 8);
+            store8<FMT>(act, act + ACT_TERM, mnmajor_off(TE + e, f, MN), rd + g * 8);
         }
     }
 }
@@ -779,19 +852,18 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     const int qd = warp & 3, ch = (warp >> 2) & 1;  // TMEM lane quadrant, 32-edge chunk of the tile
     const int f = qd * 32 + lane;
 
-    const uint32_t tmem = kernel_setup(smem, a, tslot, bars, cy, r0, 512);
-    uint8_t* op = smem + SM_OP + g * OP_BYTES;
-    Meta* tm = reinterpret_cast<Meta*>(smem + sm_meta<TE, true>() + g * sizeof(Meta));
-    float* pf_s = reinterpret_cast<float*>(op);     // after GEMM2: [chunk][feature] partials
+    const uint32_t tmem = kernel_setup(a, tslot, bars, cy, r0);
+    uint8_t* rbf = smem + SM_RBF + g * 2 * RBF_TERM;
+    uint8_t* act = smem + SM_ACT + g * 2 * ACT_TERM;
+    Meta* tmb = reinterpret_cast<Meta*>(smem + sm_meta<TE, true>() + g * 2 * sizeof(Meta));
+    float* pf_s = reinterpret_cast<float*>(act);    // after GEMM2: [chunk][feature] partials
     float* pl_s = pf_s + NCH * 128;
     float* ps_s = pl_s + NCH * 128;                 // [quadrant][edge] partial of s_e
-    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     const int col0 = ch * 32;
-    // accumulators (columns): [P | P'] at tb, [Q | Q'] at tb + 128 (64 each)
-    const uint32_t tb = tmem + g * 256;
-    const uint32_t tP = tb + lane_off + col0, tPd = tP + 64, tQ = tP + 128, tQd = tP + 192;
-    const uint32_t sop = smem_u32(op);
-    const uint32_t sbase = smem_u32(smem);
+    // accumulator columns: [P | P'] (64 each), then [Q | Q'] over them
+    const uint32_t dacc = tmem + g * TM_ACC;
+    const uint32_t tP = dacc + ((uint32_t)(qd * 32) << 16) + col0, tPd = tP + 64;
+    const uint32_t srbf = smem_u32(rbf), sact = smem_u32(act);
     const uint32_t id = idesc_f16(128, MN, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, MN, FMT, 1);
     const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF, s1d = a.s1[f] * (2.0f * LN2F);
@@ -805,47 +877,58 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     auto tile_ne = [&](int t) { return (int)min((long long)TE, e1 - e0 - (long long)t * TE); };
 
     EdgePre ep;
+    int my_g = 0, nx_g = 0;        // group threads < TE: s_e slot of edge mt (this tile / tile t+2)
+    float my_so = 0.f, nx_so = 0.f;
     if (g < ntiles) {
-        ep = prefetch_edge<TE, true>(a, e0 + (long long)g * TE, tile_ne(g), mt);
         if (g == 1) ok = wait_group(&bars[3], 0u, true, false, a.meta, g, mt);   // start half a tile behind
-    }
-    for (int t = g; t < ntiles && ok; t += 2) {
-        const int ne = tile_ne(t);
-        const int32_t* rows_g = a.crow + e0 + (long long)t * TE;
-        stage_rbf<FMT, true, TE>(a, op, tm, ep, ne, mt);
-        const int my_g = ep.gidx;           // group threads < TE: s_e slot of edge mt of this tile
-        const float my_so = ep.sold;
-        if (t + 2 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(t + 2) * TE, tile_ne(t + 2), mt);
+        ep = prefetch_edge<TE, true>(a, e0 + (long long)g * TE, tile_ne(g), mt);
+        stage_rbf<FMT, true, TE>(a, rbf, tmb, ep, tile_ne(g), mt);
+        nx_g = ep.gidx;
+        nx_so = ep.sold;
+        if (g + 2 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(g + 2) * TE, tile_ne(g + 2), mt);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
-        if (mt == 0) {
-            tc_fence_after();
-            issue_gemm<NW>(tb, sbase + SM_W1, (uint32_t)W1_IMG, sop, RBF_TERM, KP / 16, id);
-            mma_commit(&bars[g]);
-        }
-        pending = 1;
-        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM1 done
+        if (ok && mt == 0) issue_gemm1<NW>(tmem, dacc, srbf, id, &bars[g]);
+        pending = ok ? 1 : 0;
+    }
+    int buf = 0;
+    for (int t = g; t < ntiles && ok; t += 2, buf ^= 1) {
+        const int ne = tile_ne(t);
+        const bool next = t + 2 < ntiles;
+        Meta* tm = tmb + buf;
+        const int32_t* rows_g = a.crow + e0 + (long long)t * TE;
+        my_g = nx_g;
+        my_so = nx_so;
+        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM1(t) done
         pending = 0;
         if (g == 0 && !go_sent) {
             if (mt == 0) mbar_arrive(&bars[3]);
             go_sent = true;
         }
-        bwd_e1<FMT, TE>(tP, tPd, s1L, b1L, s1d, op, col0, f);
+        bwd_e1<FMT, TE>(tP, tPd, s1L, b1L, s1d, act, col0, f);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
         if (mt == 0) {
             tc_fence_after();
-            issue_gemm<NW>(tb + 128, sbase + SM_W2, (uint32_t)W2_IMG, sop, ACT_TERM, FP / 16, id_mn);
+            issue_gemm<NW>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, FP / 16, id_mn);
             mma_commit(&bars[g]);
         }
         pending = 1;
+        // under GEMM2: stage R of tile t+2 and the first gathers of this tile
+        if (next) {
+            stage_rbf<FMT, true, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), mt);
+            nx_g = ep.gidx;
+            nx_so = ep.sold;
+            if (t + 4 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(t + 4) * TE, tile_ne(t + 4), mt);
+            fence_proxy_async_smem();
+        }
         const int eb = col0;
         float uv[16], hv[16];
-        gather<16>(u_f, tm->col, eb, uv);                                // under GEMM2
+        gather<16>(u_f, tm->col, eb, uv);
         gather<16>(h_f, tm->col, eb, hv);
-        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2 done
+        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2(t) done
         pending = 0;
         // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 ln2 Q + b2s, z' = s2 Q')
         {
@@ -869,8 +952,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                         gather<16>(h_f, tm->col, eb + 16, hv);
                     }
                     float r[16], rd[16];
-                    tmem_ld16(tQ + hh * 16, r);
-                    tmem_ld16(tQd + hh * 16, rd);
+                    tmem_ld16(tP + hh * 16, r);          // Q
+                    tmem_ld16(tPd + hh * 16, rd);        // Q'
                     tmem_ld_wait();
                     const float* fcp = tm->fc + eb + hh * 16;
                     const float* dfcp = tm->dfc + eb + hh * 16;
@@ -958,13 +1041,16 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             pf_s[ch * 128 + f] = pf;
             pl_s[ch * 128 + f] = pl;
         }
-        group_sync(g);
+        tc_fence_before();
+        group_sync(g);          // Q, Q' read out; partials and the next tile's Gaussians in place
+        if (next && mt == 0) issue_gemm1<NW>(tmem, dacc, srbf, id, &bars[g]);
+        if (next) pending = 1;
         if (mt < ne) {
             const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];
             a.s_edge[my_g] = a.accumulate_s ? my_so + sv : sv;
         }
         if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
-        group_sync(g);          // merge and s_e done with tm and the partials before the next stage R
+        group_sync(g);          // merge and s_e done with the partials before E1 of the next tile overwrites them
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
     if (mt == 0) {
@@ -972,7 +1058,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         pend_s[g] = ok ? 0u : pending;
     }
     const bool all_ok = __syncthreads_or(!ok) == 0;
-    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, 512);
+    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem);
 }
 
 // ---------------------------------------------------------------------------

@@ -135,11 +135,9 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.s1 = cv.take<float>(L * FP); w.s2 = cv.take<float>(L * FP);
     w.b1 = cv.take<float>(L * FP); w.b2s = cv.take<float>(L * FP);
     w.emb = cv.take<float>((size_t)d.T * FP);
-    w.Win = cv.take<float>(L * FP * FP); w.Wo1 = cv.take<float>(L * FP * FP); w.Wo2 = cv.take<float>(L * FP * FP);
-    w.WinT = cv.take<float>(L * FP * FP); w.Wo1T = cv.take<float>(L * FP * FP);
-    w.Wo2T = cv.take<float>(L * FP * FP);
+    w.aw_img = cv.take<uint8_t>((size_t)(6 * L + 2) * AW_IMG);
+    w.aw_sc = cv.take<float>((size_t)(6 * L + 2) * FP);
     w.bo1 = cv.take<float>(L * FP); w.bo2 = cv.take<float>(L * FP);
-    w.R1 = cv.take<float>(FP * HP); w.R1T = cv.take<float>(HP * FP);
     w.c1 = cv.take<float>(HP); w.R2 = cv.take<float>(HP); w.c2 = cv.take<float>(4);
     w.rep_off = cv.take<int32_t>(R + 1);
     w.atom_rep = cv.take<int32_t>(N);
@@ -199,6 +197,33 @@ void pack_operand(const float* W, int kin, int fout, int KD, const std::vector<d
             hi[idx] = h;
             lo[idx] = l;
         }
+}
+
+// An atom-wise dense layer as a tensor-core A operand for D[r][atom] = sum_k A[r][k] X[atom][k]:
+// A[r][k] = W[k][r] (transposed use, y = x W) or W[r][k] (y = g W^T), W row-major [nrow][ncol],
+// zero outside.  Each row r is divided by its max-abs s_r (1 for a zero row), stored as fp16
+// hi + lo terms in the K-major core-matrix layout; s_r goes to sc[r].
+void pack_aw(const float* W, int nrow, int ncol, bool transposed, uint8_t* img, float* sc)
+{
+    uint16_t* hi = reinterpret_cast<uint16_t*>(img);
+    uint16_t* lo = reinterpret_cast<uint16_t*>(img + AW_IMG / 2);
+    auto A = [&](int r, int k) -> double {
+        if (transposed) return (k < nrow && r < ncol) ? (double)W[(size_t)k * ncol + r] : 0.0;
+        return (r < nrow && k < ncol) ? (double)W[(size_t)r * ncol + k] : 0.0;
+    };
+    for (int r = 0; r < FP; ++r) {
+        double m = 0.0;
+        for (int k = 0; k < FP; ++k) m = std::max(m, std::fabs(A(r, k)));
+        const float s = m > 0.0 ? (float)m : 1.0f;
+        sc[r] = s;
+        for (int k = 0; k < FP; ++k) {
+            const double v = A(r, k) / (double)s;
+            const uint16_t h = to16(v, 0);
+            const size_t idx = kmajor_off(r, k, FP) / 2;
+            hi[idx] = h;
+            lo[idx] = to16(v - from16(h, 0), 0);
+        }
+    }
 }
 
 std::vector<double> channel_scales(const float* W, int kin, int fout)
@@ -262,17 +287,14 @@ void build_weight_blob(const schnet_ctx* c, const schnet_weights* wt, uint8_t* w
             H(w.bo1)[l * FP + f] = f < F ? wt->bo1[l * F + f] : 0.f;
             H(w.bo2)[l * FP + f] = f < F ? wt->bo2[l * F + f] : 0.f;
         }
-        const size_t o = (size_t)l * FP * FP, oi = (size_t)l * F * F;
-        pad_mat(wt->W_in + oi, F, F, H(w.Win) + o, FP, FP, false);
-        pad_mat(wt->Wo1 + oi, F, F, H(w.Wo1) + o, FP, FP, false);
-        pad_mat(wt->Wo2 + oi, F, F, H(w.Wo2) + o, FP, FP, false);
-        pad_mat(wt->W_in + oi, F, F, H(w.WinT) + o, FP, FP, true);
-        pad_mat(wt->Wo1 + oi, F, F, H(w.Wo1T) + o, FP, FP, true);
-        pad_mat(wt->Wo2 + oi, F, F, H(w.Wo2T) + o, FP, FP, true);
+        const size_t oi = (size_t)l * F * F;
+        const float* mats[6] = {wt->Wo1 + oi, wt->Wo2 + oi, wt->W_in + oi, wt->W_in + oi, wt->Wo2 + oi, wt->Wo1 + oi};
+        for (int j = 0; j < 6; ++j)
+            pack_aw(mats[j], F, F, j < 3, H(w.aw_img) + (size_t)(6 * l + j) * AW_IMG, H(w.aw_sc) + (size_t)(6 * l + j) * FP);
     }
+    pack_aw(wt->R1, F, Hh, true, H(w.aw_img) + (size_t)(6 * L) * AW_IMG, H(w.aw_sc) + (size_t)(6 * L) * FP);
+    pack_aw(wt->R1, F, Hh, false, H(w.aw_img) + (size_t)(6 * L + 1) * AW_IMG, H(w.aw_sc) + (size_t)(6 * L + 1) * FP);
     pad_mat(wt->emb, c->T, F, H(w.emb), c->T, FP, false);
-    pad_mat(wt->R1, F, Hh, H(w.R1), FP, HP, false);
-    pad_mat(wt->R1, F, Hh, H(w.R1T), HP, FP, true);
     for (int k = 0; k < HP; ++k) {
         H(w.c1)[k] = k < Hh ? wt->c1[k] : 0.f;
         H(w.R2)[k] = k < Hh ? wt->R2[k] : 0.f;

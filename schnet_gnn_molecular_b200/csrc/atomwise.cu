@@ -1,6 +1,6 @@
-// Atom-wise parts of SchNet: embedding, the interaction's in/out dense layers
-// with the residual update, the per-atom readout, their backward pass, and the
-// per-replica sums.  Rows are atoms; 64 atoms per CTA, fp32 throughout.
+// Atom-wise parts of SchNet on the sm_100a tensor cores: embedding, the
+// interaction's in/out dense layers with the residual update, the per-atom
+// readout, their backward pass, and the per-replica sums.
 //
 // Model reading (FlashSchNet paper-curation summary, How / Figure 2 caption:
 // positions and embeddings pass through interaction blocks; readout per atom
@@ -8,268 +8,285 @@
 // eps = ssp(x R1 + c1) R2 + c2.  Backward (chain rule, by hand):
 //   g^L = (ssp'(pr) (.) R2) R1^T;  u = ((g Wo2^T) (.) ssp'(q)) Wo1^T;
 //   g^l = g^{l+1} + dh W_in^T.
+//
+// Each launch is a persistent kernel over tiles of 128 atoms that chains up to
+// three dense layers.  Every layer is one transposed GEMM on tcgen05,
+// D[o][atom] = A[o][k] X[atom][k]: the weights A (one output channel per lane,
+// channel-scaled, hi/lo 16-bit terms) sit in TMEM for the whole launch, the
+// activations X are staged in shared memory as hi/lo 16-bit terms after a
+// power-of-two scaling of the whole tile (so small gradients keep their
+// relative precision), and the accumulator D (128 TMEM columns) is read back
+// one feature per thread, 32 atoms per thread, for the elementwise epilogue.
+// 3 MMAs per K-step (hi*hi + lo_w*hi + hi*lo_x), fp32 accumulation.
+#include <algorithm>
+
 #include "internal.h"
 
 namespace schnet {
 
-constexpr int AT = 64;           // atoms per CTA
-constexpr int AW_THREADS = 256;
+constexpr int AWT = 512;                      // 16 warps: TMEM lane quadrant = warp % 4, atom chunk = warp / 4
+constexpr int ATILE = 128;                    // atoms per tile (GEMM N)
+constexpr uint32_t AW_BTERM = ATILE * FP * 2; // 32 KB: one 16-bit term of the [128 atoms x 128] B tile
+constexpr uint32_t AW_SMEM = 2 * AW_BTERM + 128 + 64;   // B hi/lo, per-warp maxima, mbarrier + TMEM slot
+constexpr uint32_t AW_POLLS = 1u << 22;
+constexpr uint32_t AW_ACC = 0;                // TMEM columns 0..127: accumulator
+constexpr uint32_t AW_SLOT = 128;             // TMEM columns 128 + 128 s: weight slot s (hi 64, lo 64)
+
+enum { AW_FIRST = 0, AW_FWD = 1, AW_TOP = 2, AW_BWD = 3 };
 
 struct AWArgs {
-    int N, T, L, layer;
+    int N, T, ntiles;
+    int ngemm;                    // dense layers chained in this launch (1..3)
+    int last;                     // AW_FWD: readout instead of the next layer's h
     const int32_t* types;
-    const float *emb, *Win, *Wo1, *Wo2, *WinT, *Wo1T, *Wo2T, *bo1, *bo2, *R1, *R1T, *c1, *R2, *c2;
-    float *x, *h, *q, *m, *g, *dh, *pr, *eps;
+    const uint8_t* img[3];        // the layers' packed A images (hi term, then lo term)
+    const float* sc[3];           // their per-row scales [FP]
+    const float *emb, *bo1, *bo2, *c1, *R2, *c2;
+    float *x, *h_out, *q, *m, *g, *dh, *pr, *eps;
+    const float* q_in;            // backward: q of the layer whose u is formed
     DevMeta* meta;
 };
 
-// C[64][NC] = A[64][KD] * B[KD][NC]; thread layout: 8 row groups x 32 column
-// lanes; each thread owns rows rg*8..+7 and columns lane + 32 j.
-template <int KD, int NC>
-__device__ __forceinline__ void gemm64(const float* __restrict__ sA, const float* __restrict__ sB,
-                                       float (&acc)[8][NC / 32])
+// per-tile power-of-two scale: maps the tile's largest |value| into [2^14, 2^15)
+__device__ __forceinline__ float tile_scale(const float (&v)[32], float* wmax, float& inv)
 {
-    const int lane = threadIdx.x & 31, rg = threadIdx.x >> 5;
+    float mx = 0.f;
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+    for (int q = 0; q < 32; ++q) mx = fmaxf(mx, fabsf(v[q]));
 #pragma unroll
-        for (int j = 0; j < NC / 32; ++j) acc[r][j] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < KD; ++k) {
-        float b[NC / 32];
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    __syncthreads();                                  // previous readers of wmax are done
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = 0.f;
 #pragma unroll
-        for (int j = 0; j < NC / 32; ++j) b[j] = sB[k * NC + lane + 32 * j];
+    for (int w = 0; w < AWT / 32; ++w) mx = fmaxf(mx, wmax[w]);
+    int e = 0;
+    const int ex = (int)((__float_as_uint(mx) >> 23) & 255u);
+    if (ex > 0 && ex < 255) e = 14 - (ex - 127);      // 2^(ex-127) <= mx < 2^(ex-126)
+    e = max(-120, min(120, e));
+    inv = __uint_as_float((uint32_t)(127 - e) << 23);
+    return __uint_as_float((uint32_t)(127 + e) << 23);
+}
+
+// stage 32 values (feature f = K index, atoms 32c .. 32c+31 = B rows) as hi/lo MN-major B
+__device__ __forceinline__ void stage_b(uint8_t* B, const float (&v)[32], float s, int c, int f)
+{
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            float a = sA[(rg * 8 + r) * KD + k];
+    for (int g = 0; g < 4; ++g) {
+        float w[8];
 #pragma unroll
-            for (int j = 0; j < NC / 32; ++j) acc[r][j] = fmaf(a, b[j], acc[r][j]);
+        for (int q = 0; q < 8; ++q) w[q] = v[g * 8 + q] * s;
+        store8<0>(B, B + AW_BTERM, mnmajor_off(c * 32 + g * 8, f, ATILE), w);
+    }
+}
+
+// one layer: D = A_slot * B^T, then the accumulator row of this thread (32 atoms)
+__device__ __forceinline__ bool aw_gemm(uint32_t tmem, int slot, uint32_t sB, uint64_t* bar, uint32_t& phase,
+                                        DevMeta* meta, uint32_t tD, float (&d)[32])
+{
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_f16(128, ATILE, 0, 1);
+        const uint32_t ahi = tmem + AW_SLOT + 128 * slot, alo = ahi + 64;
+        for (int ks = 0; ks < FP / 16; ++ks) {
+            const uint32_t koff = (uint32_t)ks * 2u * (uint32_t)(ATILE * 16);
+            const uint64_t bhi = smem_desc(sB + koff, ATILE * 16, 128);
+            const uint64_t blo = smem_desc(sB + AW_BTERM + koff, ATILE * 16, 128);
+            mma_f16_ts(tmem + AW_ACC, ahi + ks * 8, bhi, id, ks > 0 ? 1u : 0u);
+            mma_f16_ts(tmem + AW_ACC, alo + ks * 8, bhi, id, 1u);
+            mma_f16_ts(tmem + AW_ACC, ahi + ks * 8, blo, id, 1u);
         }
+        mma_commit(bar);
     }
-}
-
-__device__ __forceinline__ void load_mat(float* __restrict__ dst, const float* __restrict__ src, int n)
-{
-    const float4* s = reinterpret_cast<const float4*>(src);
-    float4* d = reinterpret_cast<float4*>(dst);
-    for (int i = threadIdx.x; i < n / 4; i += blockDim.x) d[i] = __ldg(s + i);
-}
-
-// load rows [i0, i0+64) of a [N][W] array into smem (zeros past N)
-template <int W>
-__device__ __forceinline__ void load_rows(float* __restrict__ dst, const float* __restrict__ src, int i0, int N)
-{
-    for (int idx = threadIdx.x; idx < AT * W / 4; idx += blockDim.x) {
-        int r = idx / (W / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i0 + r < N) v = __ldg(reinterpret_cast<const float4*>(src + (size_t)(i0 + r) * W) + idx % (W / 4));
-        reinterpret_cast<float4*>(dst)[idx] = v;
+    bool ok = true;
+    if ((threadIdx.x >> 5) == 0) ok = mbar_wait_bounded(bar, phase, AW_POLLS);
+    if (__syncthreads_or(!ok)) {
+        if (threadIdx.x == 0) set_flag(meta, SCHNET_FLAG_TIMEOUT);
+        return false;
     }
+    phase ^= 1u;
+    tc_fence_after();
+    tmem_ld32(tD, d);
+    tmem_ld_wait();
+    return true;
 }
 
-#define AW_SMEM_FLOATS (FP * FP + 2 * AT * FP)
-
-// x = emb[z]; h0 = x W_in[0]
-__global__ void __launch_bounds__(AW_THREADS) k_aw_first(AWArgs a)
+template <int MODE>
+__global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
 {
-    extern __shared__ float sm[];
-    float *sW = sm, *sX = sm + FP * FP;
-    const int i0 = blockIdx.x * AT;
-    const int lane = threadIdx.x & 31, rg = threadIdx.x >> 5;
-    for (int idx = threadIdx.x; idx < AT * FP; idx += blockDim.x) {
-        int r = idx / FP, f = idx % FP, i = i0 + r;
-        float v = 0.f;
-        if (i < a.N) {
-            int z = a.types[i];
-            if (z < 0 || z >= a.T) {
-                if (f == 0) set_flag(a.meta, SCHNET_FLAG_BADTYPE);
-                z = 0;
+    extern __shared__ __align__(1024) uint8_t sm[];
+    uint8_t* B = sm;
+    float* wmax = reinterpret_cast<float*>(sm + 2 * AW_BTERM);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 2 * AW_BTERM + 128);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qd = warp & 3, c = warp >> 2;
+    const int f = qd * 32 + lane;                    // this thread's feature (output row / next K index)
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
+    // weights: warp c of quadrant qd loads (term c >> 1, half c & 1) of every slot
+    for (int s = 0; s < a.ngemm; ++s)
+        weights_to_tmem(lane_base, AW_SLOT + 128 * s + (c >> 1) * 64, a.img[s] + (c >> 1) * AW_BTERM, f, c & 1);
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    const uint32_t sB = smem_u32(B);
+    const uint32_t tD = lane_base + AW_ACC + c * 32;
+    float sc[3];
+#pragma unroll
+    for (int s = 0; s < 3; ++s) sc[s] = s < a.ngemm ? a.sc[s][f] : 0.f;
+    uint32_t phase = 0;
+    bool ok = true;
+
+    for (int tile = blockIdx.x; tile < a.ntiles && ok; tile += gridDim.x) {
+        const int i0 = tile * ATILE + c * 32;       // this thread's first atom
+        float v[32], d[32];
+        float s, inv;
+        auto row_ok = [&](int q) { return i0 + q < a.N; };
+        auto at = [&](int q, int w) { return (size_t)(i0 + q) * w + f; };
+        // ---- input of the first layer
+        if (MODE == AW_FIRST) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                float xv = 0.f;
+                if (row_ok(q)) {
+                    int z = __ldg(a.types + i0 + q);
+                    if (z < 0 || z >= a.T) {
+                        if (f == 0) set_flag(a.meta, SCHNET_FLAG_BADTYPE);
+                        z = 0;
+                    }
+                    xv = __ldg(a.emb + (size_t)z * FP + f);
+                    a.x[at(q, FP)] = xv;
+                }
+                v[q] = xv;
             }
-            v = a.emb[z * FP + f];
-            a.x[(size_t)i * FP + f] = v;
+        } else if (MODE == AW_FWD) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] = row_ok(q) ? __ldg(a.m + at(q, FP)) : 0.f;
+        } else if (MODE == AW_TOP) {
+            // y = ssp'(pr) (.) R2 over the readout's hidden units (K = HP, zero beyond)
+            const float r2 = f < HP ? __ldg(a.R2 + f) : 0.f;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] = (f < HP && row_ok(q)) ? sigmoidf(__ldg(a.pr + at(q, HP))) * r2 : 0.f;
+        } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] = row_ok(q) ? __ldg(a.dh + at(q, FP)) : 0.f;
         }
-        sX[idx] = v;
-    }
-    load_mat(sW, a.Win, FP * FP);
-    __syncthreads();
-    float acc[8][4];
-    gemm64<FP, FP>(sX, sW, acc);
+        s = tile_scale(v, wmax, inv);
+        stage_b(B, v, s, c, f);
+        if (!(ok = aw_gemm(tmem, 0, sB, bar, phase, a.meta, tD, d))) break;
+        const float k0 = sc[0] * inv;
+        if (MODE == AW_FIRST) {
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        int i = i0 + rg * 8 + r;
-        if (i < a.N)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) a.h[(size_t)i * FP + lane + 32 * j] = acc[r][j];
-    }
-}
-
-// after the filter convolution of layer l:
-//   q = m Wo1 + bo1; x += ssp(q) Wo2 + bo2; then h_{l+1} = x W_in or the readout.
-__global__ void __launch_bounds__(AW_THREADS) k_aw_fwd(AWArgs a)
-{
-    extern __shared__ float sm[];
-    float *sW = sm, *sX = sm + FP * FP, *sY = sX + AT * FP;
-    const int l = a.layer, i0 = blockIdx.x * AT;
-    const int lane = threadIdx.x & 31, rg = threadIdx.x >> 5;
-    float* ql = a.q + (size_t)l * a.N * FP;
-    load_rows<FP>(sX, a.m, i0, a.N);
-    load_mat(sW, a.Wo1 + (size_t)l * FP * FP, FP * FP);
-    __syncthreads();
-    float acc[8][4];
-    gemm64<FP, FP>(sX, sW, acc);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        int row = rg * 8 + r, i = i0 + row;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int f = lane + 32 * j;
-            float qv = acc[r][j] + a.bo1[l * FP + f];
-            if (i < a.N) ql[(size_t)i * FP + f] = qv;
-            sY[row * FP + f] = ssp(qv);
+            for (int q = 0; q < 32; ++q)
+                if (row_ok(q)) a.h_out[at(q, FP)] = d[q] * k0;
+            continue;
         }
-    }
-    __syncthreads();
-    load_mat(sW, a.Wo2 + (size_t)l * FP * FP, FP * FP);
-    load_rows<FP>(sX, a.x, i0, a.N);
-    __syncthreads();
-    gemm64<FP, FP>(sY, sW, acc);
-    __syncthreads();
+        if (MODE == AW_FWD) {
+            // q = m Wo1 + bo1 ; a = ssp(q)
+            const float b = __ldg(a.bo1 + f);
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        int row = rg * 8 + r, i = i0 + row;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int f = lane + 32 * j;
-            float xv = sX[row * FP + f] + acc[r][j] + a.bo2[l * FP + f];
-            sX[row * FP + f] = xv;
-            if (i < a.N) a.x[(size_t)i * FP + f] = xv;
-        }
-    }
-    if (l + 1 < a.L) {
-        load_mat(sW, a.Win + (size_t)(l + 1) * FP * FP, FP * FP);
-        __syncthreads();
-        gemm64<FP, FP>(sX, sW, acc);
-        float* hn = a.h + (size_t)(l + 1) * a.N * FP;
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            int i = i0 + rg * 8 + r;
-            if (i < a.N)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) hn[(size_t)i * FP + lane + 32 * j] = acc[r][j];
-        }
-    } else {
-        // readout: pr = x R1 + c1 (HP columns); eps = sum_k ssp(pr_k) R2_k + c2
-        load_mat(sW, a.R1, FP * HP);
-        __syncthreads();
-        float acr[8][2];
-        gemm64<FP, HP>(sX, sW, acr);
-        const float c2 = a.c2[0];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            int i = i0 + rg * 8 + r;
-            float part = 0.f;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                int k = lane + 32 * j;
-                float p = acr[r][j] + a.c1[k];
-                if (i < a.N) a.pr[(size_t)i * HP + k] = p;
-                part += ssp(p) * a.R2[k];
+            for (int q = 0; q < 32; ++q) {
+                const float qv = fmaf(d[q], k0, b);
+                if (row_ok(q)) a.q[at(q, FP)] = qv;
+                v[q] = ssp(qv);
             }
+        } else if (MODE == AW_TOP) {
+            // g = y R1^T
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            if (lane == 0 && i < a.N) a.eps[i] = part + c2;
+            for (int q = 0; q < 32; ++q) {
+                v[q] = d[q] * k0;
+                if (row_ok(q)) a.g[at(q, FP)] = v[q];
+            }
+        } else {
+            // g += dh W_in^T
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                v[q] = row_ok(q) ? fmaf(d[q], k0, __ldg(a.g + at(q, FP))) : 0.f;
+                if (row_ok(q)) a.g[at(q, FP)] = v[q];
+            }
+        }
+        if (a.ngemm < 2) continue;
+        // ---- second layer
+        s = tile_scale(v, wmax, inv);
+        stage_b(B, v, s, c, f);
+        if (!(ok = aw_gemm(tmem, 1, sB, bar, phase, a.meta, tD, d))) break;
+        const float k1 = sc[1] * inv;
+        if (MODE == AW_FWD) {
+            // x += a Wo2 + bo2
+            const float b = __ldg(a.bo2 + f);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                float xv = 0.f;
+                if (row_ok(q)) {
+                    xv = a.x[at(q, FP)] + fmaf(d[q], k1, b);
+                    a.x[at(q, FP)] = xv;
+                }
+                v[q] = xv;
+            }
+        } else {
+            // t = (g Wo2^T) (.) ssp'(q)
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] = row_ok(q) ? d[q] * k1 * sigmoidf(__ldg(a.q_in + at(q, FP))) : 0.f;
+        }
+        // ---- third layer
+        s = tile_scale(v, wmax, inv);
+        stage_b(B, v, s, c, f);
+        if (!(ok = aw_gemm(tmem, 2, sB, bar, phase, a.meta, tD, d))) break;
+        const float k2 = sc[2] * inv;
+        if (MODE == AW_FWD && !a.last) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+                if (row_ok(q)) a.h_out[at(q, FP)] = d[q] * k2;
+        } else if (MODE == AW_FWD) {
+            // readout: pr = x R1 + c1 (rows f < HP); eps = sum_k ssp(pr_k) R2_k + c2, summed over
+            // the hidden units through shared memory (B is dead after the last GEMM)
+            float* S = reinterpret_cast<float*>(B);      // [HP][ATILE + 1]
+            if (f < HP) {
+                const float cb = __ldg(a.c1 + f), r2 = __ldg(a.R2 + f);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const float p = fmaf(d[q], k2, cb);
+                    if (row_ok(q)) a.pr[at(q, HP)] = p;
+                    S[f * (ATILE + 1) + c * 32 + q] = ssp(p) * r2;
+                }
+            }
+            __syncthreads();
+            if (threadIdx.x < ATILE) {
+                const int i = tile * ATILE + threadIdx.x;
+                float e = 0.f;
+                for (int k = 0; k < HP; ++k) e += S[k * (ATILE + 1) + threadIdx.x];
+                if (i < a.N) a.eps[i] = e + __ldg(a.c2);
+            }
+        } else {
+            // u = t Wo1^T, into m
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+                if (row_ok(q)) a.m[at(q, FP)] = d[q] * k2;
         }
     }
-}
-
-// u_{l} = ((g Wo2_l^T) (.) ssp'(q_l)) Wo1_l^T, with g held in sX; writes u into m.
-__device__ __forceinline__ void bwd_to_u(const AWArgs& a, int l, int i0, float* sW, float* sX, float* sY)
-{
-    const int lane = threadIdx.x & 31, rg = threadIdx.x >> 5;
-    const float* ql = a.q + (size_t)l * a.N * FP;
-    float acc[8][4];
+    // error exit: give an MMA still in flight a bounded chance to retire before freeing TMEM
+    if (!ok && threadIdx.x == 0) mbar_wait_bounded(bar, phase, AW_POLLS);
+    tc_fence_before();
     __syncthreads();
-    load_mat(sW, a.Wo2T + (size_t)l * FP * FP, FP * FP);
-    __syncthreads();
-    gemm64<FP, FP>(sX, sW, acc);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        int row = rg * 8 + r, i = i0 + row;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int f = lane + 32 * j;
-            float qv = i < a.N ? ql[(size_t)i * FP + f] : 0.f;
-            sY[row * FP + f] = acc[r][j] * sigmoidf(qv);
-        }
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
-    __syncthreads();
-    load_mat(sW, a.Wo1T + (size_t)l * FP * FP, FP * FP);
-    __syncthreads();
-    gemm64<FP, FP>(sY, sW, acc);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        int i = i0 + rg * 8 + r;
-        if (i < a.N)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) a.m[(size_t)i * FP + lane + 32 * j] = acc[r][j];
-    }
-}
-
-// g^L from the readout, then u_{L-1}
-__global__ void __launch_bounds__(AW_THREADS) k_aw_bwd_top(AWArgs a)
-{
-    extern __shared__ float sm[];
-    float *sW = sm, *sX = sm + FP * FP, *sY = sX + AT * FP;
-    const int i0 = blockIdx.x * AT;
-    const int lane = threadIdx.x & 31, rg = threadIdx.x >> 5;
-    // sY[64][HP] = ssp'(pr) (.) R2
-    for (int idx = threadIdx.x; idx < AT * HP; idx += blockDim.x) {
-        int r = idx / HP, k = idx % HP, i = i0 + r;
-        float v = 0.f;
-        if (i < a.N) v = sigmoidf(a.pr[(size_t)i * HP + k]) * a.R2[k];
-        sY[idx] = v;
-    }
-    load_mat(sW, a.R1T, HP * FP);
-    __syncthreads();
-    float acc[8][4];
-    gemm64<HP, FP>(sY, sW, acc);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        int row = rg * 8 + r, i = i0 + row;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int f = lane + 32 * j;
-            sX[row * FP + f] = acc[r][j];
-            if (i < a.N) a.g[(size_t)i * FP + f] = acc[r][j];
-        }
-    }
-    bwd_to_u(a, a.L - 1, i0, sW, sX, sY);
-}
-
-// g^l = g^{l+1} + dh_l W_in_l^T, then u_{l-1} when l > 0
-__global__ void __launch_bounds__(AW_THREADS) k_aw_bwd(AWArgs a)
-{
-    extern __shared__ float sm[];
-    float *sW = sm, *sX = sm + FP * FP, *sY = sX + AT * FP;
-    const int l = a.layer, i0 = blockIdx.x * AT;
-    const int lane = threadIdx.x & 31, rg = threadIdx.x >> 5;
-    load_rows<FP>(sY, a.dh, i0, a.N);
-    load_mat(sW, a.WinT + (size_t)l * FP * FP, FP * FP);
-    __syncthreads();
-    float acc[8][4];
-    gemm64<FP, FP>(sY, sW, acc);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        int row = rg * 8 + r, i = i0 + row;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            int f = lane + 32 * j;
-            float gv = acc[r][j] + (i < a.N ? a.g[(size_t)i * FP + f] : 0.f);
-            sX[row * FP + f] = gv;
-            if (i < a.N) a.g[(size_t)i * FP + f] = gv;
-        }
-    }
-    if (l > 0) bwd_to_u(a, l - 1, i0, sW, sX, sY);
 }
 
 // ---------------------------------------------------------------------------
@@ -305,58 +322,87 @@ __global__ void k_replica_sums(int R, const int32_t* __restrict__ chunk_rep, int
     if (!isfinite(s)) set_flag(meta, SCHNET_FLAG_NONFINITE);
 }
 
-static AWArgs aw_args(schnet_ctx* c, const int32_t* types, int layer)
+// images and scales of the atom-wise layers: per layer l, matrix id 6 l + j with
+// j = 0 Wo1^T, 1 Wo2^T, 2 W_in^T (forward), 3 W_in, 4 Wo2, 5 Wo1 (backward);
+// then 6 L = R1^T (readout), 6 L + 1 = R1 (readout backward)
+static AWArgs aw_args(schnet_ctx* c, const int32_t* types, int mode, int layer)
 {
     Workspace& w = c->ws;
-    AWArgs a;
-    a.N = c->N; a.T = c->T; a.L = c->L; a.layer = layer;
+    const int L = c->L;
+    AWArgs a{};
+    a.N = c->N;
+    a.T = c->T;
+    a.ntiles = (c->N + ATILE - 1) / ATILE;
     a.types = types;
-    a.emb = w.emb; a.Win = w.Win; a.Wo1 = w.Wo1; a.Wo2 = w.Wo2;
-    a.WinT = w.WinT; a.Wo1T = w.Wo1T; a.Wo2T = w.Wo2T;
-    a.bo1 = w.bo1; a.bo2 = w.bo2; a.R1 = w.R1; a.R1T = w.R1T; a.c1 = w.c1; a.R2 = w.R2; a.c2 = w.c2;
-    a.x = w.x; a.h = w.h; a.q = w.q; a.m = w.m; a.g = w.g; a.dh = w.dh; a.pr = w.pr; a.eps = w.eps;
-    a.meta = w.meta;
+    a.emb = w.emb; a.bo1 = w.bo1 + layer * FP; a.bo2 = w.bo2 + layer * FP;
+    a.c1 = w.c1; a.R2 = w.R2; a.c2 = w.c2;
+    a.x = w.x; a.q = w.q + (size_t)layer * c->N * FP; a.m = w.m; a.g = w.g; a.dh = w.dh; a.pr = w.pr;
+    a.eps = w.eps; a.meta = w.meta;
+    int ids[3] = {0, 0, 0};
+    if (mode == AW_FIRST) {
+        a.ngemm = 1; ids[0] = 2;
+        a.h_out = w.h;
+    } else if (mode == AW_FWD) {
+        a.ngemm = 3; ids[0] = 6 * layer; ids[1] = 6 * layer + 1;
+        a.last = layer + 1 == L;
+        ids[2] = a.last ? 6 * L : 6 * (layer + 1) + 2;
+        a.h_out = a.last ? nullptr : w.h + (size_t)(layer + 1) * c->N * FP;
+    } else if (mode == AW_TOP) {
+        a.ngemm = 3; ids[0] = 6 * L + 1; ids[1] = 6 * (L - 1) + 4; ids[2] = 6 * (L - 1) + 5;
+        a.q_in = w.q + (size_t)(L - 1) * c->N * FP;
+    } else {
+        a.ngemm = layer > 0 ? 3 : 1;
+        ids[0] = 6 * layer + 3;
+        if (layer > 0) {
+            ids[1] = 6 * (layer - 1) + 4; ids[2] = 6 * (layer - 1) + 5;
+            a.q_in = w.q + (size_t)(layer - 1) * c->N * FP;
+        }
+    }
+    for (int s = 0; s < 3; ++s) {
+        a.img[s] = w.aw_img + (size_t)ids[s] * AW_IMG;
+        a.sc[s] = w.aw_sc + (size_t)ids[s] * FP;
+    }
     return a;
 }
-
-constexpr size_t AW_SMEM = sizeof(float) * AW_SMEM_FLOATS;
 
 cudaError_t atomwise_init_attributes()
 {
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(k_aw_first, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM))) return e;
-    if ((e = cudaFuncSetAttribute(k_aw_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM))) return e;
-    if ((e = cudaFuncSetAttribute(k_aw_bwd_top, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM)))
+    if ((e = cudaFuncSetAttribute(k_atomwise<AW_FIRST>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM)))
         return e;
-    return cudaFuncSetAttribute(k_aw_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM);
+    if ((e = cudaFuncSetAttribute(k_atomwise<AW_FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM)))
+        return e;
+    if ((e = cudaFuncSetAttribute(k_atomwise<AW_TOP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM)))
+        return e;
+    return cudaFuncSetAttribute(k_atomwise<AW_BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM);
 }
 
-static int aw_blocks(schnet_ctx* c) { return (c->N + AT - 1) / AT; }
+static int aw_grid(schnet_ctx* c) { return std::min((c->N + ATILE - 1) / ATILE, c->nsm); }
 
 cudaError_t launch_aw_first(schnet_ctx* c, const int32_t* types)
 {
-    k_aw_first<<<aw_blocks(c), AW_THREADS, AW_SMEM, c->s>>>(aw_args(c, types, 0));
+    k_atomwise<AW_FIRST><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, types, AW_FIRST, 0));
     c->launches += 1;
     return cudaGetLastError();
 }
 
 cudaError_t launch_aw_fwd(schnet_ctx* c, int layer)
 {
-    k_aw_fwd<<<aw_blocks(c), AW_THREADS, AW_SMEM, c->s>>>(aw_args(c, nullptr, layer));
+    k_atomwise<AW_FWD><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, nullptr, AW_FWD, layer));
     c->launches += 1;
     return cudaGetLastError();
 }
 
 cudaError_t launch_aw_bwd_top(schnet_ctx* c)
 {
-    k_aw_bwd_top<<<aw_blocks(c), AW_THREADS, AW_SMEM, c->s>>>(aw_args(c, nullptr, c->L - 1));
+    k_atomwise<AW_TOP><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, nullptr, AW_TOP, c->L - 1));
     c->launches += 1;
     return cudaGetLastError();
 }
 
 cudaError_t launch_aw_bwd(schnet_ctx* c, int layer)
 {
-    k_aw_bwd<<<aw_blocks(c), AW_THREADS, AW_SMEM, c->s>>>(aw_args(c, nullptr, layer));
+    k_atomwise<AW_BWD><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, nullptr, AW_BWD, layer));
     c->launches += 1;
     return cudaGetLastError();
 }

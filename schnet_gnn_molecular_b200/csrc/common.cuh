@@ -283,4 +283,102 @@ struct Split<1> {
     }
 };
 
+// ---------------------------------------------------------------------------
+// tcgen05 helpers shared by the tensor-core kernels
+// ---------------------------------------------------------------------------
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16 (A read from tensor memory)
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this warp's 32 lanes <- 32 registers per thread
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+        "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+        "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+// Row f of one packed weight term (the K-major core-matrix image: K elements
+// 8kg .. 8kg+7 of row f are the 16 bytes at kg * 2048 + f * 16) into 32 TMEM
+// columns starting at `col` (K elements 64 * half .. 64 * half + 63).
+__device__ __forceinline__ void weights_to_tmem(uint32_t taddr_lane, uint32_t col, const uint8_t* __restrict__ term,
+                                                int f, int half)
+{
+    uint32_t v[32];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(term + (size_t)(half * 8 + q) * (FP * 16) + f * 16));
+        v[4 * q] = x.x;
+        v[4 * q + 1] = x.y;
+        v[4 * q + 2] = x.z;
+        v[4 * q + 3] = x.w;
+    }
+    tmem_st32(taddr_lane + col + half * 32, v);
+}
+
+// two fp32 values -> packed 16-bit hi pair and lo (residual) pair
+template <int FMT>
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo);
+template <>
+__device__ __forceinline__ void split2<0>(float x0, float x1, uint32_t& hi, uint32_t& lo)
+{
+    __half2 h = __floats2half2_rn(x0, x1);
+    float2 hf = __half22float2(h);
+    __half2 l = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<uint32_t*>(&h);
+    lo = *reinterpret_cast<uint32_t*>(&l);
+}
+template <>
+__device__ __forceinline__ void split2<1>(float x0, float x1, uint32_t& hi, uint32_t& lo)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    float2 hf = __bfloat1622float2(h);
+    __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<uint32_t*>(&h);
+    lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
+// 8 consecutive fp32 values -> one 16-byte hi store and one 16-byte lo store
+template <int FMT>
+__device__ __forceinline__ void store8(uint8_t* hi_base, uint8_t* lo_base, uint32_t off, const float* v)
+{
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) split2<FMT>(v[2 * q], v[2 * q + 1], h[q], l[q]);
+    *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4*>(lo_base + off) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void store8_zero(uint8_t* hi_base, uint8_t* lo_base, uint32_t off)
+{
+    *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(lo_base + off) = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// 32 lanes x 16 columns of TMEM -> 16 registers per thread
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])
+{
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+
 }  // namespace schnet

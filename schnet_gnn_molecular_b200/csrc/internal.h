@@ -25,6 +25,8 @@ constexpr int REDUCE_CHUNK = 4096;    // atoms per partial sum of a per-replica 
 constexpr size_t W1_IMG = (size_t)FP * KP * 2;   // one 16-bit term of W1^T (M=128 x K=64)
 constexpr size_t W2_IMG = (size_t)FP * FP * 2;   // one 16-bit term of W2^T (M=128 x K=128)
 constexpr size_t LAYER_IMG = 2 * W1_IMG + 2 * W2_IMG;  // hi + lo of both
+// One atom-wise dense layer as an A operand: [128 rows][K = 128], hi term then lo term.
+constexpr size_t AW_IMG = 2 * (size_t)FP * FP * 2;
 
 struct Workspace {
     DevMeta* meta;
@@ -33,10 +35,9 @@ struct Workspace {
     float *s1, *s2, *b1;          // [L][FP] filter channel scales, first-layer bias
     float* b2s;                   // [L][FP] second-layer bias minus ln2 s2 sum_k W2^[k][f] (base-2 softplus shift)
     float *emb;                   // [T][FP]
-    float *Win, *Wo1, *Wo2;       // [L][FP][FP]  (row-major [in][out])
-    float *WinT, *Wo1T, *Wo2T;    // [L][FP][FP]  (transposed: [out][in])
+    uint8_t* aw_img;              // [6 L + 2][AW_IMG] atom-wise layers as tensor-core A operands
+    float* aw_sc;                 // [6 L + 2][FP] their per-row scales
     float *bo1, *bo2;             // [L][FP]
-    float *R1, *R1T;              // [FP][HP], [HP][FP]
     float *c1, *R2;               // [HP]
     float *c2;                    // [1]
     // atoms

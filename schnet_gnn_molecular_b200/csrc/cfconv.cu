@@ -262,20 +262,23 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMet
     }
 }
 
-// Issue D (+)= W^T * B over `ksteps` K-steps of 16 with the hi/lo split
+// Issue D (+)= W^T * B over KSTEPS K-steps of 16 with the hi/lo split
 // (A: the weight term in TMEM, 8 columns per K-step; B: MN = 128 rows in
-// shared memory, no-swizzle core matrices).
-template <int NW>
+// shared memory, no-swizzle core matrices).  The two B descriptors are built
+// once; a K-step advances only their 14-bit start-address field (operand
+// regions lie below 256 KB, so the field cannot carry into the strides).
+template <int NW, int KSTEPS>
 __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_hi_t, uint32_t a_lo_t, uint32_t b_base,
-                                           uint32_t b_term, int ksteps, uint32_t idesc)
+                                           uint32_t b_term, uint32_t idesc)
 {
-    for (int ks = 0; ks < ksteps; ++ks) {
-        const uint32_t koff = (uint32_t)ks * 2u * (uint32_t)(MN * 16);   // 2 core matrices of 8 along K
-        const uint64_t b_hi = smem_desc(b_base + koff, MN * 16, 128);
-        const uint64_t b_lo = smem_desc(b_base + b_term + koff, MN * 16, 128);
-        mma_f16_ts(d_tmem, a_hi_t + ks * 8, b_hi, idesc, ks > 0 ? 1u : 0u);
-        if (NW == 2) mma_f16_ts(d_tmem, a_lo_t + ks * 8, b_hi, idesc, 1u);
-        mma_f16_ts(d_tmem, a_hi_t + ks * 8, b_lo, idesc, 1u);
+    const uint64_t bh0 = smem_desc(b_base, MN * 16, 128);
+    const uint64_t bl0 = smem_desc(b_base + b_term, MN * 16, 128);
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+        const uint64_t step = (uint64_t)((ks * 2 * MN * 16) >> 4);   // 2 core matrices of 8 along K
+        mma_f16_ts(d_tmem, a_hi_t + ks * 8, bh0 + step, idesc, ks > 0 ? 1u : 0u);
+        if (NW == 2) mma_f16_ts(d_tmem, a_lo_t + ks * 8, bh0 + step, idesc, 1u);
+        mma_f16_ts(d_tmem, a_hi_t + ks * 8, bl0 + step, idesc, 1u);
     }
 }
 
@@ -575,7 +578,7 @@ template <int NW>
 __device__ __forceinline__ void issue_gemm1(uint32_t tmem, uint32_t dacc, uint32_t srbf, uint32_t id, uint64_t* bar)
 {
     tc_fence_after();
-    issue_gemm<NW>(dacc, tmem + TM_W1H, tmem + TM_W1L, srbf, RBF_TERM, KP / 16, id);
+    issue_gemm<NW, KP / 16>(dacc, tmem + TM_W1H, tmem + TM_W1L, srbf, RBF_TERM, id);
     mma_commit(bar);
 }
 
@@ -659,7 +662,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         group_sync(g);
         if (mt == 0) {
             tc_fence_after();
-            issue_gemm<NW>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, FP / 16, id_mn);
+            issue_gemm<NW, FP / 16>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, id_mn);
             mma_commit(&bars[g]);
         }
         pending = 1;
@@ -817,7 +820,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         group_sync(g);
         if (mt == 0) {
             tc_fence_after();
-            issue_gemm<NW>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, FP / 16, id_mn);
+            issue_gemm<NW, FP / 16>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, id_mn);
             mma_commit(&bars[g]);
         }
         pending = 1;

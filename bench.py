@@ -201,6 +201,20 @@ def _edge_stats(model, pos, w):
     return int(len(col)), int((d < w.cutoff).sum())
 
 
+def _traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
+    the kernel source has changed since that capture (hash recorded beside the figure)."""
+    import hashlib
+    try:
+        d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        src = open(os.path.join(ROOT, d["source"]), "rb").read()
+        if hashlib.sha256(src).hexdigest()[:16] != d["source_sha256_16"]:
+            return None
+        return d.get(kernel)
+    except Exception:
+        return None
+
+
 def nat_status(st):
     from schnet_gnn_molecular_b200 import _native
     return _native.STATUS_NAMES.get(int(st), str(st))
@@ -275,13 +289,7 @@ def run_native(args):
         flops, kms = (flop_bwd, bwd_ms) if dominant == "cfconv_bwd" else (flop_fwd, fwd_ms)
         peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
         achieved = flops / (kms * 1e-3) / 1e12
-        traffic = None
-        tf = os.path.join(ROOT, "profiles", "traffic.json")
-        if os.path.exists(tf):
-            try:
-                traffic = json.load(open(tf)).get(dominant)
-            except Exception:
-                traffic = None
+        traffic = _traffic(dominant)
         roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 2),
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                     "peak_source": f"{src} dense bf16/fp16 sustained",

@@ -249,13 +249,24 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMet
             continue;
         }
         float gv[8], dv[8];
+        if (!BWD) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const float x = fmaf(-(float)(g * 8 + q), a.dmu, dm);
-            const float t = x * a.ngc;
-            const float gg = ex2_mufu(t * x);
-            gv[q] = gg;
-            dv[q] = t * gg;
+            for (int q = 0; q < 8; q += 2) {
+                const float2 x = fma2(make_float2(-(float)(g * 8 + q), -(float)(g * 8 + q + 1)), dup2(a.dmu), dup2(dm));
+                const float2 t = mul2(x, dup2(a.ngc));
+                const float2 e = mul2(t, x);
+                gv[q] = ex2_mufu(e.x);
+                gv[q + 1] = ex2_mufu(e.y);
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float x = fmaf(-(float)(g * 8 + q), a.dmu, dm);
+                const float t = x * a.ngc;
+                const float gg = ex2_mufu(t * x);
+                gv[q] = gg;
+                dv[q] = t * gg;
+            }
         }
         store8<FMT>(b_hi, b_lo, off, gv);
         if (BWD) store8<FMT>(b_hi, b_lo, offd, dv);
@@ -423,10 +434,14 @@ template <int N>
 __device__ __forceinline__ float tree_sum(float (&v)[N])
 {
 #pragma unroll
-    for (int w = N / 2; w >= 1; w >>= 1)
+    for (int w = N / 2; w >= 2; w >>= 1)
 #pragma unroll
-        for (int q = 0; q < w; ++q) v[q] += v[q + w];
-    return v[0];
+        for (int q = 0; q < w; q += 2) {
+            const float2 t = add2(make_float2(v[q], v[q + 1]), make_float2(v[q + w], v[q + w + 1]));
+            v[q] = t.x;
+            v[q + 1] = t.y;
+        }
+    return v[0] + v[1];
 }
 
 // Reduce a chunk's per-edge terms t[q] (edge eb + q) to the first-row and
@@ -544,7 +559,11 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
     tmem_ld32(tP, r);
     tmem_ld_wait();
 #pragma unroll
-    for (int q = 0; q < 32; ++q) r[q] = sp2(fmaf(s1L, r[q], b1L));
+    for (int q = 0; q < 32; q += 2) {
+        const float2 v = sp2x2(fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L)));
+        r[q] = v.x;
+        r[q + 1] = v.y;
+    }
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         const uint32_t off = mnmajor_off(e0 + g * 8, f, MN);
@@ -567,9 +586,12 @@ __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* t
     float fc[32];
     load_edges<32>(tm->fc, eb, fc);
 #pragma unroll
-    for (int q = 0; q < 32; ++q) r[q] = fc[q] * fmaf(s2L, r[q], b2s);
-#pragma unroll
-    for (int q = 0; q < 32; ++q) r[q] *= hv[q];
+    for (int q = 0; q < 32; q += 2) {
+        const float2 z = fma2(dup2(s2L), make_float2(r[q], r[q + 1]), dup2(b2s));
+        const float2 v = mul2(mul2(make_float2(fc[q], fc[q + 1]), z), make_float2(hv[q], hv[q + 1]));
+        r[q] = v.x;
+        r[q + 1] = v.y;
+    }
     chunk_partials<32>(tm->c[cc], rows_g, eb, ne, r, out, f, pf, pl);
 }
 

@@ -80,6 +80,20 @@ __device__ __forceinline__ float sp2(float p)
     return fmaxf(p, 0.0f) + lg2_mufu(1.0f + ex2_mufu(-fabsf(p)));
 }
 
+// Two-wide fp32 arithmetic (sm_100 packed FFMA2 / FMUL2 / FADD2: two lanes of
+// ordinary round-to-nearest single precision per instruction).
+__device__ __forceinline__ float2 dup2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// sp2 of two values: max(p, 0) + log2(1 + 2^-|p|)
+__device__ __forceinline__ float2 sp2x2(float2 p)
+{
+    const float2 y = add2(dup2(1.0f), make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y))));
+    return add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
+}
+
 // ssp(x) and ssp'(x) sharing one exponential
 __device__ __forceinline__ void ssp_and_grad(float x, float& s, float& g)
 {

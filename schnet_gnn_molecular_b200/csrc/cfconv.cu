@@ -745,7 +745,7 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
             const float p = fmaf(s1L, r[q], b1L);
             const float t = ex2_mufu(-fabsf(p));
             const float y = 1.0f + t;
-            const float inv = rcp_mufu(y);
+            const float inv = rcp_1to2(y);                    // y = 1 + 2^-|p| in [1, 2]
             const float sg = p >= 0.0f ? inv : t * inv;       // logistic(x)
             r[q] = fmaxf(p, 0.0f) + lg2_mufu(y);
             rd[q] = sg * (s1d * rd[q]);

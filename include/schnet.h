@@ -84,8 +84,19 @@ typedef enum {
  *         significant bits) and activations likewise: fp32-level accuracy on
  *         the 16-bit tensor-core path.
  *   FP16 / BF16: the scaled weights are rounded once to the 16-bit type
- *         (what is stored), activations still carried as hi + lo pairs. */
-typedef enum { SCHNET_WEIGHTS_FP32 = 0, SCHNET_WEIGHTS_FP16 = 1, SCHNET_WEIGHTS_BF16 = 2 } schnet_weight_dtype;
+ *         (what is stored), activations still carried as hi + lo pairs.
+ *   FP16_FAST: fp16 weights as FP16, and the filter network's activations
+ *         (Gaussians, their distance derivatives, the softplus outputs and
+ *         their tangents) rounded once to fp16 as well: one tensor-core
+ *         product per K-step instead of two (FP16) or three (FP32).  The
+ *         atom-wise layers and all accumulations stay fp32.  A speed mode,
+ *         held to the 16-bit tolerance (forces within 2e-3 of fp32). */
+typedef enum {
+    SCHNET_WEIGHTS_FP32 = 0,
+    SCHNET_WEIGHTS_FP16 = 1,
+    SCHNET_WEIGHTS_BF16 = 2,
+    SCHNET_WEIGHTS_FP16_FAST = 3
+} schnet_weight_dtype;
 
 typedef struct {
     int32_t n_types;          /* T  >= 1                                       */

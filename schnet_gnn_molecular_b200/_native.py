@@ -15,7 +15,7 @@ OK = 0
 STATUS_NAMES = {0: "OK", 1: "INVALID_ARG", 2: "CUDA", 3: "CAPACITY", 4: "SKIN", 5: "NONFINITE", 6: "BADTYPE",
                 7: "STATE", 8: "TIMEOUT", 9: "UNSUPPORTED"}
 FLAG_CAPACITY, FLAG_SKIN, FLAG_NONFINITE, FLAG_BADTYPE, FLAG_TIMEOUT = 0x1, 0x2, 0x4, 0x8, 0x10
-WEIGHT_DTYPES = {"fp32": 0, "fp16": 1, "bf16": 2}
+WEIGHT_DTYPES = {"fp32": 0, "fp16": 1, "bf16": 2, "fp16fast": 3}
 
 EXPORTED = ["schnet_workspace_bytes", "schnet_create", "schnet_build_neighbors", "schnet_energy_forces",
             "schnet_step", "schnet_step_host", "schnet_get_status", "schnet_last_error", "schnet_destroy",

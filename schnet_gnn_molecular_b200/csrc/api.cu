@@ -80,7 +80,7 @@ schnet_status validate(const schnet_config* c, std::string& why)
                 return SCHNET_ERR_UNSUPPORTED;
             }
     }
-    if (c->weight_dtype < 0 || c->weight_dtype > 2) { why = "weight_dtype"; return SCHNET_ERR_INVALID_ARG; }
+    if (c->weight_dtype < 0 || c->weight_dtype > 3) { why = "weight_dtype"; return SCHNET_ERR_INVALID_ARG; }
     if ((int64_t)c->n_atoms * FP > (int64_t)1 << 40) { why = "too many atoms"; return SCHNET_ERR_UNSUPPORTED; }
     return SCHNET_OK;
 }
@@ -561,6 +561,7 @@ schnet_status schnet_create(const schnet_config* cfg, const schnet_weights* wt, 
     c->N = d.N; c->R = d.R; c->T = d.T; c->F = d.F; c->K = d.K; c->L = d.L; c->H = d.F / 2;
     c->weight_fmt = cfg->weight_dtype == SCHNET_WEIGHTS_BF16 ? 1 : 0;
     c->n_wterms = cfg->weight_dtype == SCHNET_WEIGHTS_FP32 ? 2 : 1;
+    c->n_xterms = cfg->weight_dtype == SCHNET_WEIGHTS_FP16_FAST ? 1 : 2;
     c->cap = d.cap;
     c->ncell = d.ncell;
     c->nchunk = d.nchunk;

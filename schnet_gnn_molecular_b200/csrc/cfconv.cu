@@ -199,7 +199,7 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
 // back in).  Gaussian columns K .. KP-1 meet zero weight rows and are stored
 // as zeros without evaluating them; masked or padding edges have
 // f_c = f_c' = 0, so their Gaussians need no mask (they stay finite).
-template <int FMT, bool BWD, int TE>
+template <int FMT, int NX, bool BWD, int TE>
 __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMeta<TE, BWD>* tmeta, const EdgePre& ep,
                                           int ne, int mt)
 {
@@ -268,8 +268,8 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMet
                 dv[q] = t * gg;
             }
         }
-        store8<FMT>(b_hi, b_lo, off, gv);
-        if (BWD) store8<FMT>(b_hi, b_lo, offd, dv);
+        store8_act<FMT, NX>(b_hi, b_lo, off, gv);
+        if (BWD) store8_act<FMT, NX>(b_hi, b_lo, offd, dv);
     }
 }
 
@@ -278,7 +278,7 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMet
 // shared memory, no-swizzle core matrices).  The two B descriptors are built
 // once; a K-step advances only their 14-bit start-address field (operand
 // regions lie below 256 KB, so the field cannot carry into the strides).
-template <int NW, int KSTEPS>
+template <int NW, int NX, int KSTEPS>
 __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_hi_t, uint32_t a_lo_t, uint32_t b_base,
                                            uint32_t b_term, uint32_t idesc)
 {
@@ -289,7 +289,7 @@ __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_hi_t, uin
         const uint64_t step = (uint64_t)((ks * 2 * MN * 16) >> 4);   // 2 core matrices of 8 along K
         mma_f16_ts(d_tmem, a_hi_t + ks * 8, bh0 + step, idesc, ks > 0 ? 1u : 0u);
         if (NW == 2) mma_f16_ts(d_tmem, a_lo_t + ks * 8, bh0 + step, idesc, 1u);
-        mma_f16_ts(d_tmem, a_hi_t + ks * 8, bl0 + step, idesc, 1u);
+        if (NX == 2) mma_f16_ts(d_tmem, a_hi_t + ks * 8, bl0 + step, idesc, 1u);
     }
 }
 
@@ -552,7 +552,7 @@ __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r
 // forward epilogue 1 for 32 edges: a = sp2(s1 log2e P + b1 log2e) -> MN-major B
 // operand (the base-2 softplus; ssp = ln2 (a - 1), with ln2 and the shift folded
 // into the second layer's scale and bias)
-template <int FMT>
+template <int FMT, int NX>
 __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_t* act, int e0, int f)
 {
     float r[32];
@@ -567,7 +567,7 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
         const uint32_t off = mnmajor_off(e0 + g * 8, f, MN);
-        store8<FMT>(act, act + ACT_TERM, off, r + g * 8);
+        store8_act<FMT, NX>(act, act + ACT_TERM, off, r + g * 8);
     }
 }
 
@@ -596,11 +596,11 @@ __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* t
 }
 
 // Issue GEMM1 of a tile (group g): D = W1^T [B rows of the group's GEMM1 operand]
-template <int NW>
+template <int NW, int NX>
 __device__ __forceinline__ void issue_gemm1(uint32_t tmem, uint32_t dacc, uint32_t srbf, uint32_t id, uint64_t* bar)
 {
     tc_fence_after();
-    issue_gemm<NW, KP / 16>(dacc, tmem + TM_W1H, tmem + TM_W1L, srbf, RBF_TERM, id);
+    issue_gemm<NW, NX, KP / 16>(dacc, tmem + TM_W1H, tmem + TM_W1L, srbf, RBF_TERM, id);
     mma_commit(bar);
 }
 
@@ -610,7 +610,7 @@ __device__ __forceinline__ void issue_gemm1(uint32_t tmem, uint32_t dacc, uint32
 // Per group and tile t: [GEMM1(t) in flight] E1 -> issue GEMM2 -> stage R of
 // t+2 (into the group's own GEMM1 operand and second metadata buffer) and the
 // first gather under GEMM2 -> E2 -> issue GEMM1(t+2) -> merge under GEMM1(t+2).
-template <int FMT, int NW>
+template <int FMT, int NW, int NX>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {
     constexpr int TE = TE_F;
@@ -657,12 +657,12 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     if (g < ntiles) {
         if (g == 1) ok = wait_group(&bars[3], 0u, true, false, a.meta, g, mt);   // start half a tile behind
         ep = prefetch_edge<TE, false>(a, e0 + (long long)g * TE, tile_ne(g), mt);
-        stage_rbf<FMT, false, TE>(a, rbf, tmb, ep, tile_ne(g), mt);
+        stage_rbf<FMT, NX, false, TE>(a, rbf, tmb, ep, tile_ne(g), mt);
         if (g + 2 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(g + 2) * TE, tile_ne(g + 2), mt);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
-        if (ok && mt == 0) issue_gemm1<NW>(tmem, dacc, srbf, id, &bars[g]);
+        if (ok && mt == 0) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         pending = ok ? 1 : 0;
     }
     int buf = 0;
@@ -678,19 +678,19 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
             go_sent = true;
         }
 #pragma unroll 1
-        for (int c2 = 0; c2 < 2; ++c2) fwd_e1<FMT>(tA + c2 * 32, s1L, b1L, act, ch * 64 + c2 * 32, f);
+        for (int c2 = 0; c2 < 2; ++c2) fwd_e1<FMT, NX>(tA + c2 * 32, s1L, b1L, act, ch * 64 + c2 * 32, f);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
         if (mt == 0) {
             tc_fence_after();
-            issue_gemm<NW, FP / 16>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, id_mn);
+            issue_gemm<NW, NX, FP / 16>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, id_mn);
             mma_commit(&bars[g]);
         }
         pending = 1;
         // under GEMM2: stage R of tile t+2 and the first gather of this tile
         if (next) {
-            stage_rbf<FMT, false, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), mt);
+            stage_rbf<FMT, NX, false, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), mt);
             if (t + 4 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(t + 4) * TE, tile_ne(t + 4), mt);
             fence_proxy_async_smem();
         }
@@ -709,7 +709,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         }
         tc_fence_before();
         group_sync(g);          // Q read out; partials and the next tile's Gaussians in place
-        if (next && mt == 0) issue_gemm1<NW>(tmem, dacc, srbf, id, &bars[g]);
+        if (next && mt == 0) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
         if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
         group_sync(g);          // merge done with the partials before E1 of the next tile overwrites them
@@ -730,7 +730,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 // p = x log2e = s1 log2e P + b1 log2e and dx/dd = s1 2ln2 P' (P' from the scaled
 // Gaussian-derivative rows).  ssp'(x) = 1 / (1 + e^-x) shares 2^-|p| with sp2.
 // a goes to B rows e, b to B rows TE + e of GEMM2's operand.
-template <int FMT, int TE>
+template <int FMT, int NX, int TE>
 __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* act,
                                        int col0, int f)
 {
@@ -753,13 +753,13 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
             const int e = col0 + hh * 16 + g * 8;
-            store8<FMT>(act, act + ACT_TERM, mnmajor_off(e, f, MN), r + g * 8);
-            store8<FMT>(act, act + ACT_TERM, mnmajor_off(TE + e, f, MN), rd + g * 8);
+            store8_act<FMT, NX>(act, act + ACT_TERM, mnmajor_off(e, f, MN), r + g * 8);
+            store8_act<FMT, NX>(act, act + ACT_TERM, mnmajor_off(TE + e, f, MN), rd + g * 8);
         }
     }
 }
 
-template <int FMT, int NW>
+template <int FMT, int NW, int NX>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
     constexpr int TE = TE_B;
@@ -812,14 +812,14 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     if (g < ntiles) {
         if (g == 1) ok = wait_group(&bars[3], 0u, true, false, a.meta, g, mt);   // start half a tile behind
         ep = prefetch_edge<TE, true>(a, e0 + (long long)g * TE, tile_ne(g), mt);
-        stage_rbf<FMT, true, TE>(a, rbf, tmb, ep, tile_ne(g), mt);
+        stage_rbf<FMT, NX, true, TE>(a, rbf, tmb, ep, tile_ne(g), mt);
         nx_g = ep.gidx;
         nx_so = ep.sold;
         if (g + 2 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(g + 2) * TE, tile_ne(g + 2), mt);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
-        if (ok && mt == 0) issue_gemm1<NW>(tmem, dacc, srbf, id, &bars[g]);
+        if (ok && mt == 0) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         pending = ok ? 1 : 0;
     }
     int buf = 0;
@@ -836,19 +836,19 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             if (mt == 0) mbar_arrive(&bars[3]);
             go_sent = true;
         }
-        bwd_e1<FMT, TE>(tP, tPd, s1L, b1L, s1d, act, col0, f);
+        bwd_e1<FMT, NX, TE>(tP, tPd, s1L, b1L, s1d, act, col0, f);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
         if (mt == 0) {
             tc_fence_after();
-            issue_gemm<NW, FP / 16>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, id_mn);
+            issue_gemm<NW, NX, FP / 16>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, id_mn);
             mma_commit(&bars[g]);
         }
         pending = 1;
         // under GEMM2: stage R of tile t+2 and the first gathers of this tile
         if (next) {
-            stage_rbf<FMT, true, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), mt);
+            stage_rbf<FMT, NX, true, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), mt);
             nx_g = ep.gidx;
             nx_so = ep.sold;
             if (t + 4 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(t + 4) * TE, tile_ne(t + 4), mt);
@@ -973,7 +973,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         }
         tc_fence_before();
         group_sync(g);          // Q, Q' read out; partials and the next tile's Gaussians in place
-        if (next && mt == 0) issue_gemm1<NW>(tmem, dacc, srbf, id, &bars[g]);
+        if (next && mt == 0) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
         if (mt < ne) {
             const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];
@@ -1095,34 +1095,40 @@ static MPArgs make_args(schnet_ctx* c, int layer)
     return a;
 }
 
-template <int FMT, int NW>
+template <int FMT, int NW, int NX>
 static cudaError_t set_attrs()
 {
-    cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_bytes<TE_F, false>());
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_bytes<TE_B, true>());
 }
 
 cudaError_t cfconv_init_attributes()
 {
     cudaError_t e;
-    if ((e = set_attrs<0, 2>()) != cudaSuccess) return e;
-    if ((e = set_attrs<0, 1>()) != cudaSuccess) return e;
-    return set_attrs<1, 1>();
+    if ((e = set_attrs<0, 2, 2>()) != cudaSuccess) return e;
+    if ((e = set_attrs<0, 1, 2>()) != cudaSuccess) return e;
+    if ((e = set_attrs<1, 1, 2>()) != cudaSuccess) return e;
+    return set_attrs<0, 1, 1>();
 }
 
+// operand formats: fp32 weights (fp16 hi+lo weights and activations), fp16 or bf16
+// weights (one weight term, hi+lo activations), fp16 weights with fp16 activations
 cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
 {
     MPArgs a = make_args(c, layer);
     a.out = c->ws.m;
-    if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_fwd<0, 2><<<c->ncta, NT, smem_bytes<TE_F, false>(), c->s>>>(a);
+    const size_t sm = smem_bytes<TE_F, false>();
+    if (c->n_xterms == 1)
+        k_cfconv_fwd<0, 1, 1><<<c->ncta, NT, sm, c->s>>>(a);
+    else if (c->weight_fmt == 0 && c->n_wterms == 2)
+        k_cfconv_fwd<0, 2, 2><<<c->ncta, NT, sm, c->s>>>(a);
     else if (c->weight_fmt == 0)
-        k_cfconv_fwd<0, 1><<<c->ncta, NT, smem_bytes<TE_F, false>(), c->s>>>(a);
+        k_cfconv_fwd<0, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
     else
-        k_cfconv_fwd<1, 1><<<c->ncta, NT, smem_bytes<TE_F, false>(), c->s>>>(a);
+        k_cfconv_fwd<1, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
     c->launches += 1;
     return cudaGetLastError();
 }
@@ -1132,12 +1138,15 @@ cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s)
     MPArgs a = make_args(c, layer);
     a.out = c->ws.dh;
     a.accumulate_s = accumulate_s;
-    if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_bwd<0, 2><<<c->ncta, NT, smem_bytes<TE_B, true>(), c->s>>>(a);
+    const size_t sm = smem_bytes<TE_B, true>();
+    if (c->n_xterms == 1)
+        k_cfconv_bwd<0, 1, 1><<<c->ncta, NT, sm, c->s>>>(a);
+    else if (c->weight_fmt == 0 && c->n_wterms == 2)
+        k_cfconv_bwd<0, 2, 2><<<c->ncta, NT, sm, c->s>>>(a);
     else if (c->weight_fmt == 0)
-        k_cfconv_bwd<0, 1><<<c->ncta, NT, smem_bytes<TE_B, true>(), c->s>>>(a);
+        k_cfconv_bwd<0, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
     else
-        k_cfconv_bwd<1, 1><<<c->ncta, NT, smem_bytes<TE_B, true>(), c->s>>>(a);
+        k_cfconv_bwd<1, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
     c->launches += 1;
     return cudaGetLastError();
 }

@@ -388,6 +388,32 @@ __device__ __forceinline__ void store8(uint8_t* hi_base, uint8_t* lo_base, uint3
     *reinterpret_cast<uint4*>(lo_base + off) = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
+// 8 consecutive fp32 values -> one 16-byte store of their 16-bit rounding (no lo term)
+template <int FMT>
+__device__ __forceinline__ void store8_hi(uint8_t* hi_base, uint32_t off, const float* v)
+{
+    uint32_t h[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        if (FMT == 0) {
+            __half2 x = __floats2half2_rn(v[2 * q], v[2 * q + 1]);
+            h[q] = *reinterpret_cast<uint32_t*>(&x);
+        } else {
+            __nv_bfloat162 x = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+            h[q] = *reinterpret_cast<uint32_t*>(&x);
+        }
+    }
+    *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// activation operand: hi/lo pair (NX = 2) or the 16-bit rounding alone (NX = 1)
+template <int FMT, int NX>
+__device__ __forceinline__ void store8_act(uint8_t* hi_base, uint8_t* lo_base, uint32_t off, const float* v)
+{
+    if (NX == 2) store8<FMT>(hi_base, lo_base, off, v);
+    else store8_hi<FMT>(hi_base, off, v);
+}
+
 __device__ __forceinline__ void store8_zero(uint8_t* hi_base, uint8_t* lo_base, uint32_t off)
 {
     *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(0u, 0u, 0u, 0u);

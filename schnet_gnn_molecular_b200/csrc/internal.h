@@ -91,6 +91,7 @@ struct schnet_ctx {
     int N, R, T, F, K, L, H;
     int weight_fmt;                 // 0 fp16 operands, 1 bf16 operands
     int n_wterms;                   // 2 (fp32 storage: hi+lo) or 1
+    int n_xterms;                   // filter activations: 2 (hi+lo) or 1 (16-bit, the fast mode)
     int64_t cap;
     int nsm, ncta;                  // SMs; CTAs of the tensor-core kernels
     int ncell;                      // total cells reserved

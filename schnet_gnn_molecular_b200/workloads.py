@@ -41,7 +41,7 @@ class Workload:
     temperature: float = 300.0
     n_rebuild: int = 20
     steps: int = 1
-    weight_dtype: str = "fp32"  # "fp32" | "fp16" | "bf16"
+    weight_dtype: str = "fp32"  # "fp32" | "fp16" | "bf16" | "fp16fast" (fp16 weights and filter activations)
     seed: int = 0
     radius: float | None = None  # confinement radius for compact chains
     rg_target: float = 12.0
@@ -68,6 +68,7 @@ PROTEIN64 = Workload(name="cg_protein_64x269", n_replicas=64, beads=269, geometr
 
 PROTEIN64_FP16 = PROTEIN64.with_(name="cg_protein_64x269_fp16w", weight_dtype="fp16", seed=2000)
 PROTEIN64_BF16 = PROTEIN64.with_(name="cg_protein_64x269_bf16w", weight_dtype="bf16", seed=2000)
+PROTEIN64_FP16FAST = PROTEIN64.with_(name="cg_protein_64x269_fp16fast", weight_dtype="fp16fast", seed=2000)
 
 
 def sweep(n_replicas: int) -> Workload:
@@ -89,7 +90,7 @@ BOX1M = Workload(name="periodic_box_1M", n_replicas=1, beads=1_000_000, geometry
                  density=0.01, box=(1_000_000 / 0.01) ** (1.0 / 3.0), integrator="vv", gamma_per_ps=0.0,
                  steps=1000, seed=4000)
 
-ALL = {w.name: w for w in [TINY, PROTEIN64, PROTEIN64_FP16, PROTEIN64_BF16, BOX1M]}
+ALL = {w.name: w for w in [TINY, PROTEIN64, PROTEIN64_FP16, PROTEIN64_BF16, PROTEIN64_FP16FAST, BOX1M]}
 
 
 @lru_cache(maxsize=16)

@@ -12,6 +12,7 @@ ENERGY_RTOL = 1e-5          # float32 / tensor-core path vs float64 oracle, per 
 FORCE_RTOL = 1e-4           # relative Frobenius error of all forces
 FORCE_RTOL_16BIT = 2e-3     # 16-bit filter weights vs the fp32 oracle
 FORCE_RTOL_DEQUANT = 1e-4   # 16-bit filter weights vs the oracle on the same dequantized weights
+ENERGY_RTOL_16BIT = 2e-3    # fp16 fast mode (16-bit weights and filter activations) vs the fp32 oracle
 
 
 def oracle_model(w: workloads.Workload, weights: dict, dequant: str | None = None) -> oracle.Model:

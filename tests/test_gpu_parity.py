@@ -7,7 +7,8 @@ import pytest
 import torch
 
 import oracle
-from _helpers import (ENERGY_RTOL, FORCE_RTOL, FORCE_RTOL_16BIT, FORCE_RTOL_DEQUANT, energy_rel, oracle_model,
+from _helpers import (ENERGY_RTOL, ENERGY_RTOL_16BIT, FORCE_RTOL, FORCE_RTOL_16BIT, FORCE_RTOL_DEQUANT,
+                      energy_rel, oracle_model,
                       rel_frobenius)
 from schnet_gnn_molecular_b200 import api, inputs, workloads
 
@@ -113,6 +114,25 @@ def test_sixteen_bit_filter_weights(dtype):
     assert energy_rel(E, Eq, eps_q, ro) <= ENERGY_RTOL
     assert rel_frobenius(F, Fq) <= FORCE_RTOL_DEQUANT
     assert rel_frobenius(F, F32) <= FORCE_RTOL_16BIT
+
+
+def test_fp16_fast_mode():
+    # fp16 weights and fp16 filter activations (one tensor-core product per K-step):
+    # held to the 16-bit force bound against the fp32 oracle, and compared with the
+    # oracle on the same dequantized weights (the difference is the activation rounding)
+    w = SMALL_PROTEIN.with_(weight_dtype="fp16fast")
+    pos, types, weights, model = _setup(w, bias_scale=0.1)
+    E, F = _gpu_eval(model, pos, types)
+    x64 = pos.astype(np.float64)
+    ro = w.replica_offsets()
+    Eq, eps_q, Fq = oracle.energy_forces(oracle_model(w, weights, dequant="fp16"), x64, types, ro)
+    E32, eps32, F32 = oracle.energy_forces(oracle_model(w, weights), x64, types, ro)
+    print(f"[errors fp16fast] energy vs dequantized {energy_rel(E, Eq, eps_q, ro):.3e}, forces vs dequantized "
+          f"{rel_frobenius(F, Fq):.3e}, energy vs fp32 weights {energy_rel(E, E32, eps32, ro):.3e}, forces vs "
+          f"fp32 weights {rel_frobenius(F, F32):.3e}")
+    assert rel_frobenius(F, F32) <= FORCE_RTOL_16BIT
+    assert rel_frobenius(F, Fq) <= FORCE_RTOL_16BIT
+    assert energy_rel(E, E32, eps32, ro) <= ENERGY_RTOL_16BIT
 
 
 def test_isolated_atoms_and_empty_rows():

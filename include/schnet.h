@@ -150,8 +150,12 @@ SCHNET_API schnet_status schnet_create(const schnet_config *cfg, const schnet_we
  * j ascending) plus rev[e] = index of the reverse edge (j, i), i.e. the
  * transposed list; a cell list (cells >= r_c + skin) limits the candidates.
  * The list is kept on the device with its edge count; positions are
- * snapshotted for the skin check.  Overflow sets SCHNET_FLAG_CAPACITY and
- * leaves the list unusable until a build fits.  Errors: INVALID_ARG, CUDA. */
+ * snapshotted for the skin check.  Until the next build the context holds
+ * atoms internally in cell order (cells grouped by replica, ascending atom
+ * index inside a cell) so that atoms close in space are close in memory;
+ * every value it returns (forces, energies, the taps below) is in the
+ * caller's atom order.  Overflow sets SCHNET_FLAG_CAPACITY and leaves the
+ * list unusable until a build fits.  Errors: INVALID_ARG, CUDA. */
 SCHNET_API schnet_status schnet_build_neighbors(schnet_ctx *ctx, const float *d_pos);
 
 /* Energy per replica and forces at d_pos using the current list.
@@ -209,13 +213,17 @@ SCHNET_API const char *schnet_last_error(const schnet_ctx *ctx);
 /* Release the context (synchronizes; the workspace stays the caller's). */
 SCHNET_API schnet_status schnet_destroy(schnet_ctx *ctx);
 
-/* Test tap: synchronize and copy the current list to host arrays:
- * h_row_ptr int32 [N+1], h_col, h_rev int32 [cap]; *n_edges = edge count.
- * Any pointer may be NULL.  Errors: CAPACITY if cap is smaller than the list. */
+/* Test tap: synchronize and copy the current list, in the caller's atom order
+ * (row i lists j ascending, as schnet_build_neighbors defines it), to host
+ * arrays: h_row_ptr int32 [N+1], h_col, h_rev int32 [cap]; *n_edges = edge
+ * count.  Any pointer may be NULL.  The reordering uses scratch that the next
+ * evaluation rewrites anyway.  Errors: STATE (no list), CAPACITY if cap is
+ * smaller than the list. */
 SCHNET_API schnet_status schnet_get_neighbors(schnet_ctx *ctx, int32_t *h_row_ptr, int32_t *h_col, int32_t *h_rev,
                                    int64_t *n_edges, int64_t cap);
 
-/* Test tap: per-atom energies eps_i of the last evaluation, device float32 [N]. */
+/* Test tap: per-atom energies eps_i of the last evaluation, device float32 [N],
+ * caller's atom order.  Errors: INVALID_ARG, STATE (no list), CUDA. */
 SCHNET_API schnet_status schnet_get_atom_energies(schnet_ctx *ctx, float *d_eps);
 
 /* Kernel classes reported by schnet_profile_steps. */

@@ -146,6 +146,7 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     cv.off = align_up(cv.off, 256);
     if (wend) *wend = cv.off;
     w.pos4 = cv.take<float4>(N); w.ref4 = cv.take<float4>(N); w.frc4 = cv.take<float4>(N);
+    w.perm = cv.take<int32_t>(N); w.cell_slot = cv.take<int32_t>(N);
     w.row_ptr = cv.take<int32_t>(N + 1); w.rowcnt = cv.take<int32_t>(N + 1);
     w.col = cv.take<int32_t>(d.cap); w.coltmp = cv.take<int32_t>(d.cap);
     w.rev = cv.take<int32_t>(d.cap); w.erow = cv.take<int32_t>(d.cap);
@@ -394,7 +395,7 @@ cudaError_t enqueue_steps(schnet_ctx* c, int k, bool build_first, float* pos, fl
     cudaError_t e;
     if (build_first) {
         Timed t(c, SCHNET_KERNEL_NEIGHBORS);
-        if ((e = launch_build_neighbors(c)) != cudaSuccess) return e;
+        if ((e = launch_build_neighbors(c, pos)) != cudaSuccess) return e;
     }
     for (int s = 0; s < k; ++s) {
         {
@@ -457,9 +458,8 @@ schnet_status step_impl(schnet_ctx* c, float* pos, float* vel, const int32_t* ty
     double* ep = epot ? epot : c->ws.epot;
     double* ek = ekin ? ekin : c->ws.ekin;
     if (!p->resume || !c->forces_valid) {
-        c->have_list = false;            // fresh start: the build below replaces the list (no skin check)
-        CK(launch_pack_positions(c, pos));
-        CK(launch_build_neighbors(c));
+        c->have_list = false;            // fresh start: the build below replaces the list
+        CK(launch_build_neighbors(c, pos));
         c->have_list = true;
         CK(launch_energy_forces(c, types, ep, nullptr));
         c->since_build = p->n_rebuild;   // the first interval starts with a fresh build
@@ -611,9 +611,8 @@ schnet_status schnet_build_neighbors(schnet_ctx* c, const float* d_pos)
 {
     if (!c || !d_pos) return SCHNET_ERR_INVALID_ARG;
     join_in(c);
-    c->have_list = false;   // no skin check while packing for a build
-    CK(launch_pack_positions(c, d_pos));
-    CK(launch_build_neighbors(c));
+    c->have_list = false;
+    CK(launch_build_neighbors(c, d_pos));
     c->have_list = true;
     c->forces_valid = false;
     CK(join_out(c));
@@ -706,11 +705,12 @@ schnet_status schnet_get_neighbors(schnet_ctx* c, int32_t* h_row_ptr, int32_t* h
     CK(cudaStreamSynchronize(c->s));
     if (n_edges) *n_edges = hm.n_edges;
     if (hm.n_edges > c->cap) return fail(c, SCHNET_ERR_CAPACITY, "edge list overflowed its capacity");
-    if (h_row_ptr)
-        CK(cudaMemcpyAsync(h_row_ptr, c->ws.row_ptr, (c->N + 1) * sizeof(int32_t), cudaMemcpyDeviceToHost, c->s));
     if ((h_col || h_rev) && cap < hm.n_edges) return fail(c, SCHNET_ERR_CAPACITY, "host buffer too small");
-    if (h_col) CK(cudaMemcpyAsync(h_col, c->ws.col, hm.n_edges * sizeof(int32_t), cudaMemcpyDeviceToHost, c->s));
-    if (h_rev) CK(cudaMemcpyAsync(h_rev, c->ws.rev, hm.n_edges * sizeof(int32_t), cudaMemcpyDeviceToHost, c->s));
+    const int32_t *rp = nullptr, *col = nullptr, *rev = nullptr;
+    CK(launch_caller_order_list(c, &rp, &col, &rev));
+    if (h_row_ptr) CK(cudaMemcpyAsync(h_row_ptr, rp, (c->N + 1) * sizeof(int32_t), cudaMemcpyDeviceToHost, c->s));
+    if (h_col) CK(cudaMemcpyAsync(h_col, col, hm.n_edges * sizeof(int32_t), cudaMemcpyDeviceToHost, c->s));
+    if (h_rev) CK(cudaMemcpyAsync(h_rev, rev, hm.n_edges * sizeof(int32_t), cudaMemcpyDeviceToHost, c->s));
     CK(cudaStreamSynchronize(c->s));
     return SCHNET_OK;
 }
@@ -718,8 +718,9 @@ schnet_status schnet_get_neighbors(schnet_ctx* c, int32_t* h_row_ptr, int32_t* h
 schnet_status schnet_get_atom_energies(schnet_ctx* c, float* d_eps)
 {
     if (!c || !d_eps) return SCHNET_ERR_INVALID_ARG;
+    if (!c->have_list) return fail(c, SCHNET_ERR_STATE, "no neighbour list");
     join_in(c);
-    CK(cudaMemcpyAsync(d_eps, c->ws.eps, c->N * sizeof(float), cudaMemcpyDeviceToDevice, c->s));
+    CK(launch_scatter_atoms(c, c->ws.eps, d_eps));
     CK(join_out(c));
     return SCHNET_OK;
 }

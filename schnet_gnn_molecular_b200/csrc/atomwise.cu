@@ -38,7 +38,8 @@ struct AWArgs {
     int N, T, ntiles;
     int ngemm;                    // dense layers chained in this launch (1..3)
     int last;                     // AW_FWD: readout instead of the next layer's h
-    const int32_t* types;
+    const int32_t* types;         // caller order
+    const int32_t* perm;          // slot -> caller index
     const uint8_t* img[3];        // the layers' packed A images (hi term, then lo term)
     const float* sc[3];           // their per-row scales [FP]
     const float *emb, *bo1, *bo2, *c1, *R2, *c2;
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
             for (int q = 0; q < 32; ++q) {
                 float xv = 0.f;
                 if (row_ok(q)) {
-                    int z = __ldg(a.types + i0 + q);
+                    int z = __ldg(a.types + __ldg(a.perm + i0 + q));
                     if (z < 0 || z >= a.T) {
                         if (f == 0) set_flag(a.meta, SCHNET_FLAG_BADTYPE);
                         z = 0;
@@ -334,6 +335,7 @@ static AWArgs aw_args(schnet_ctx* c, const int32_t* types, int mode, int layer)
     a.T = c->T;
     a.ntiles = (c->N + ATILE - 1) / ATILE;
     a.types = types;
+    a.perm = w.perm;
     a.emb = w.emb; a.bo1 = w.bo1 + layer * FP; a.bo2 = w.bo2 + layer * FP;
     a.c1 = w.c1; a.R2 = w.R2; a.c2 = w.c2;
     a.x = w.x; a.q = w.q + (size_t)layer * c->N * FP; a.m = w.m; a.g = w.g; a.dh = w.dh; a.pr = w.pr;

@@ -8,6 +8,8 @@
 // segment sum over the CSR and its transpose map, no atomics (FlashSchNet
 // paper-curation summary, How: contention-free accumulation forward and
 // backward).
+// Rows are slots (atoms in cell order); perm maps a slot to the caller's
+// index, under which forces are stored for the integrator and the caller.
 // Integrator (the pages name Langevin / velocity-Verlet dynamics but give no
 // scheme): BAOAB of Leimkuhler & Matthews; gamma = 0 is velocity Verlet.
 // Noise: Philox4x32-10 (Salmon et al., SC'11) keyed by the seed, counter
@@ -21,8 +23,9 @@ constexpr double KB = 0.0019872041;       // kcal/mol/K
 
 __global__ void k_forces(int n, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
                          const int32_t* __restrict__ rev, const float* __restrict__ s_edge,
-                         const float4* __restrict__ pos4, const Box box, float rc, long long cap,
-                         DevMeta* meta, float4* __restrict__ frc4, float* __restrict__ out3)
+                         const float4* __restrict__ pos4, const int32_t* __restrict__ perm, const Box box,
+                         float rc, long long cap, DevMeta* meta, float4* __restrict__ frc4,
+                         float* __restrict__ out3)
 {
     if (meta->n_edges > cap) return;
     const int lane = threadIdx.x & 31;
@@ -52,11 +55,12 @@ __global__ void k_forces(int n, const int32_t* __restrict__ row_ptr, const int32
             fz += __shfl_xor_sync(0xffffffffu, fz, o);
         }
         if (lane == 0) {
-            frc4[i] = make_float4(fx, fy, fz, 0.f);
+            const int ic = perm[i];
+            frc4[ic] = make_float4(fx, fy, fz, 0.f);
             if (out3) {
-                out3[3 * i] = fx;
-                out3[3 * i + 1] = fy;
-                out3[3 * i + 2] = fz;
+                out3[3 * ic] = fx;
+                out3[3 * ic + 1] = fy;
+                out3[3 * ic + 2] = fz;
             }
             if (!(isfinite(fx) && isfinite(fy) && isfinite(fz))) set_flag(meta, SCHNET_FLAG_NONFINITE);
         }
@@ -68,7 +72,7 @@ cudaError_t launch_forces(schnet_ctx* c, float* d_forces)
     Workspace& w = c->ws;
     int blocks = (c->N + 7) / 8;   // 8 warps per block, one row per warp
     if (blocks > c->nsm * 16) blocks = c->nsm * 16;
-    k_forces<<<blocks, 256, 0, c->s>>>(c->N, w.row_ptr, w.col, w.rev, w.s_edge, w.pos4, c->box, c->cfg.cutoff,
+    k_forces<<<blocks, 256, 0, c->s>>>(c->N, w.row_ptr, w.col, w.rev, w.s_edge, w.pos4, w.perm, c->box, c->cfg.cutoff,
                                        c->cap, w.meta, w.frc4, d_forces);
     c->launches += 1;
     return cudaGetLastError();
@@ -105,14 +109,18 @@ __device__ __forceinline__ float3 normals3(unsigned long long seed, unsigned lon
     return make_float3((float)(r0 * c1), (float)(r0 * s1), (float)(r1 * c3));
 }
 
-// B (half kick with the current forces), A, O, A.
-__global__ void k_baoa(int n, float* __restrict__ pos, float* __restrict__ vel, const float* __restrict__ mass,
-                       const float4* __restrict__ frc4, float4* __restrict__ pos4, const float4* __restrict__ ref4,
-                       float dt, float c1, float kT_acc, int langevin, unsigned long long seed,
-                       const float* __restrict__ noise, int check_skin, float half_skin2, DevMeta* meta)
+// B (half kick with the current forces), A, O, A.  One thread per slot k: the
+// atom's caller index i addresses the caller's arrays and the noise counter,
+// k the slot-order positions of the force evaluation and the skin reference.
+__global__ void k_baoa(int n, const int32_t* __restrict__ perm, float* __restrict__ pos, float* __restrict__ vel,
+                       const float* __restrict__ mass, const float4* __restrict__ frc4, float4* __restrict__ pos4,
+                       const float4* __restrict__ ref4, float dt, float c1, float kT_acc, int langevin,
+                       unsigned long long seed, const float* __restrict__ noise, int check_skin, float half_skin2,
+                       DevMeta* meta)
 {
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n) return;
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= n) return;
+    const int i = perm[k];
     const float inv_m = 1.0f / mass[i];
     const float4 F = frc4[i];
     const float hk = 0.5f * dt * ACC * inv_m;
@@ -140,10 +148,10 @@ __global__ void k_baoa(int n, float* __restrict__ pos, float* __restrict__ vel, 
         vel[3 * i + d] = v[d];
         pos[3 * i + d] = r[d];
     }
-    pos4[i] = make_float4(r[0], r[1], r[2], 0.f);
+    pos4[k] = make_float4(r[0], r[1], r[2], 0.f);
     if (!(isfinite(r[0]) && isfinite(r[1]) && isfinite(r[2]))) set_flag(meta, SCHNET_FLAG_NONFINITE);
     if (check_skin) {
-        float4 q = ref4[i];
+        float4 q = ref4[k];
         float dx = r[0] - q.x, dy = r[1] - q.y, dz = r[2] - q.z;
         if (dx * dx + dy * dy + dz * dz > half_skin2) set_flag(meta, SCHNET_FLAG_SKIN);
     }
@@ -156,7 +164,7 @@ cudaError_t launch_baoa(schnet_ctx* c, float* d_pos, float* d_vel, const float* 
     double c1 = exp(-(double)gamma * 1e-3 * (double)dt);
     double kT_acc = KB * (double)temp * (double)ACC;
     float hs = 0.5f * c->cfg.skin;
-    k_baoa<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, d_pos, d_vel, d_mass, w.frc4, w.pos4, w.ref4, dt,
+    k_baoa<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, w.perm, d_pos, d_vel, d_mass, w.frc4, w.pos4, w.ref4, dt,
                                                   (float)c1, (float)kT_acc, gamma != 0.f ? 1 : 0, seed, d_noise,
                                                   check_skin ? 1 : 0, hs * hs, w.meta);
     c->launches += 1;

@@ -40,8 +40,9 @@ struct Workspace {
     float *bo1, *bo2;             // [L][FP]
     float *c1, *R2;               // [HP]
     float *c2;                    // [1]
-    // atoms
-    int32_t* atom_rep;            // [N]
+    // atoms (pos4, ref4 and every activation below in slot order; frc4 in caller order)
+    int32_t* atom_rep;            // [N]   replica of an atom (the same in both orders)
+    int32_t* perm;                // [N]   caller index of the atom in each slot
     float4 *pos4, *ref4, *frc4;   // [N]
     // neighbour list
     int32_t *row_ptr, *rowcnt;    // [N+1]
@@ -51,7 +52,8 @@ struct Workspace {
     int32_t* ccount;              // [ncta]
     int32_t* part;                // [ncta+1]
     // cell list
-    int32_t *cell_of, *cell_atoms;       // [N]
+    int32_t *cell_of, *cell_atoms;       // [N]  caller order
+    int32_t* cell_slot;                  // [N]  cell of each slot
     int32_t *cell_cnt, *cell_start, *cell_fill;  // [ncell+1]
     int32_t* rep_off;             // [R+1] replica offsets
     int4* rgrid_dims;             // [R]   (gx, gy, gz, first cell)
@@ -126,7 +128,10 @@ namespace schnet {
 
 // launchers (each enqueues on ctx->s and counts its kernels in ctx->launches)
 cudaError_t launch_pack_positions(schnet_ctx* c, const float* d_pos);
-cudaError_t launch_build_neighbors(schnet_ctx* c);
+cudaError_t launch_build_neighbors(schnet_ctx* c, const float* d_pos);
+cudaError_t launch_caller_order_list(schnet_ctx* c, const int32_t** row_ptr, const int32_t** col,
+                                     const int32_t** rev);
+cudaError_t launch_scatter_atoms(schnet_ctx* c, const float* v, float* out);
 cudaError_t launch_energy_forces(schnet_ctx* c, const int32_t* d_types, double* d_energy, float* d_forces);
 cudaError_t launch_baoa(schnet_ctx* c, float* d_pos, float* d_vel, const float* d_mass, float dt, float gamma,
                         float temp, unsigned long long seed, const float* d_noise, bool check_skin);

@@ -128,28 +128,39 @@ static cudaError_t scan_exclusive(schnet_ctx* c, const int32_t* in, int n, int32
 
 // ---------------------------------------------------------------------------
 // positions
+//
+// Between two builds every per-atom array of the energy / force path is held in
+// "slot" order: atoms sorted by cell (cells grouped by replica, raster order
+// inside a replica, ascending atom index inside a cell).  Atoms that are close
+// in space are then close in memory, so the per-edge gathers of neighbour
+// features hit cache lines and L2 sets that the neighbouring rows have just
+// used.  perm[k] is the caller's index of the atom in slot k.  Positions,
+// velocities, masses, forces and per-replica results stay in the caller's order.
 // ---------------------------------------------------------------------------
-__global__ void k_pack_positions(int n, const float* __restrict__ pos, float4* __restrict__ pos4,
-                                 const float4* __restrict__ ref4, int check_skin, float half_skin2,
-                                 DevMeta* meta)
+__global__ void k_pack_positions(int n, const float* __restrict__ pos, const int32_t* __restrict__ perm,
+                                 float4* __restrict__ pos4, const float4* __restrict__ ref4, int check_skin,
+                                 float half_skin2, DevMeta* meta)
 {
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n) return;
+    int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= n) return;
+    const int i = perm ? perm[k] : k;
     float x = pos[3 * i], y = pos[3 * i + 1], z = pos[3 * i + 2];
-    pos4[i] = make_float4(x, y, z, 0.0f);
+    pos4[k] = make_float4(x, y, z, 0.0f);
     if (!(isfinite(x) && isfinite(y) && isfinite(z))) set_flag(meta, SCHNET_FLAG_NONFINITE);
     if (check_skin) {
-        float4 r = ref4[i];
+        float4 r = ref4[k];
         float dx = x - r.x, dy = y - r.y, dz = z - r.z;
         if (dx * dx + dy * dy + dz * dz > half_skin2) set_flag(meta, SCHNET_FLAG_SKIN);
     }
 }
 
+// caller positions -> slot order, with the skin check against the last build
 cudaError_t launch_pack_positions(schnet_ctx* c, const float* d_pos)
 {
+    if (!c->have_list) return cudaErrorInvalidValue;
     float hs = 0.5f * c->cfg.skin;
-    k_pack_positions<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, d_pos, c->ws.pos4, c->ws.ref4,
-                                                            c->have_list ? 1 : 0, hs * hs, c->ws.meta);
+    k_pack_positions<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, d_pos, c->ws.perm, c->ws.pos4, c->ws.ref4, 1,
+                                                            hs * hs, c->ws.meta);
     c->launches += 1;
     return cudaGetLastError();
 }
@@ -259,6 +270,38 @@ __global__ void k_cell_fill(int n, const int32_t* __restrict__ cell_of, const in
     cell_atoms[cell_start[cell] + slot] = i;
 }
 
+// One warp per cell: the cell's atoms in ascending caller index (the fill above
+// places them in arrival order), so the slot order is a function of the
+// positions alone.
+__global__ void k_cell_order(int ncell, const int32_t* __restrict__ cell_start,
+                             const int32_t* __restrict__ cell_atoms, int32_t* __restrict__ perm)
+{
+    int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int lane = threadIdx.x & 31;
+    int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int cell = warp; cell < ncell; cell += nwarps) {
+        int a = cell_start[cell], b = cell_start[cell + 1];
+        for (int k = a + lane; k < b; k += 32) {
+            int v = cell_atoms[k];
+            int rank = 0;
+            for (int t = a; t < b; ++t) rank += cell_atoms[t] < v;
+            perm[a + rank] = v;
+        }
+    }
+}
+
+// slot-order positions and cells from the caller-order ones
+__global__ void k_gather_slots(int n, const int32_t* __restrict__ perm, const float4* __restrict__ posc4,
+                               const int32_t* __restrict__ cell_of, float4* __restrict__ pos4,
+                               int32_t* __restrict__ cell_slot)
+{
+    int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= n) return;
+    const int i = perm[k];
+    pos4[k] = posc4[i];
+    cell_slot[k] = cell_of[i];
+}
+
 // float64 pair test, each operation rounded separately (no contraction)
 __device__ __forceinline__ bool pair_in_list(float4 pi, float4 pj, double rl2, const Box& box)
 {
@@ -277,6 +320,8 @@ __device__ __forceinline__ bool pair_in_list(float4 pi, float4 pj, double rl2, c
 }
 
 // Visit every candidate j (cells around atom i's cell) passing the list test.
+// With cell_atoms == nullptr the atoms are already in cell order: the
+// candidates of a cell are the index range cell_start[cell] .. cell_start[cell+1].
 template <class Fn>
 __device__ __forceinline__ void for_each_neighbor(int i, const float4* __restrict__ pos4,
                                                   const int32_t* __restrict__ atom_rep,
@@ -313,7 +358,7 @@ __device__ __forceinline__ void for_each_neighbor(int i, const float4* __restric
                 int cell = g.w + x + g.x * (y + g.y * z);
                 int a = cell_start[cell], b = cell_start[cell + 1];
                 for (int k = a; k < b; ++k) {
-                    int j = cell_atoms[k];
+                    int j = cell_atoms ? cell_atoms[k] : k;
                     if (j == i) continue;
                     if (pair_in_list(pi, pos4[j], rl2, box)) fn(j);
                 }
@@ -424,7 +469,9 @@ __global__ void k_check_capacity(long long cap, DevMeta* meta)
     if (meta->n_edges > cap) set_flag(meta, SCHNET_FLAG_CAPACITY);
 }
 
-cudaError_t launch_build_neighbors(schnet_ctx* c)
+// Build from the caller-order positions d_pos: cell grid and cell sort in the
+// caller's order, then the slot permutation, then the list itself in slot order.
+cudaError_t launch_build_neighbors(schnet_ctx* c, const float* d_pos)
 {
     Workspace& w = c->ws;
     const int N = c->N, R = c->R;
@@ -435,30 +482,100 @@ cudaError_t launch_build_neighbors(schnet_ctx* c)
     gp.gmax = GMAX_NONPERIODIC;
     gp.cells_per_rep = c->ncell / R;
     cudaError_t err;
+    const int nb = (N + 255) / 256;
+    float4* posc4 = w.ref4;   // caller-order positions; replaced by the slot-order reference at the end
 
-    k_replica_grid<<<R, 256, 0, c->s>>>(R, w.rep_off, w.pos4, gp, c->box, w.rgrid_dims, w.rgrid_org, w.rgrid_inv);
+    k_pack_positions<<<nb, 256, 0, c->s>>>(N, d_pos, nullptr, posc4, nullptr, 0, 0.f, w.meta);
+    k_replica_grid<<<R, 256, 0, c->s>>>(R, w.rep_off, posc4, gp, c->box, w.rgrid_dims, w.rgrid_org, w.rgrid_inv);
     cudaMemsetAsync(w.cell_cnt, 0, sizeof(int32_t) * (c->ncell + 1), c->s);
     cudaMemsetAsync(w.cell_fill, 0, sizeof(int32_t) * (c->ncell + 1), c->s);
-    int nb = (N + 255) / 256;
-    k_cell_assign<<<nb, 256, 0, c->s>>>(N, w.pos4, w.atom_rep, w.rgrid_dims, w.rgrid_org, w.rgrid_inv,
+    k_cell_assign<<<nb, 256, 0, c->s>>>(N, posc4, w.atom_rep, w.rgrid_dims, w.rgrid_org, w.rgrid_inv,
                                         gp.periodic, w.cell_of, w.cell_cnt);
-    c->launches += 2;
+    c->launches += 3;
     if ((err = scan_exclusive(c, w.cell_cnt, c->ncell, w.cell_start, nullptr)) != cudaSuccess) return err;
     k_cell_fill<<<nb, 256, 0, c->s>>>(N, w.cell_of, w.cell_start, w.cell_fill, w.cell_atoms);
+    k_cell_order<<<c->nsm * 8, 256, 0, c->s>>>(c->ncell, w.cell_start, w.cell_atoms, w.perm);
+    k_gather_slots<<<nb, 256, 0, c->s>>>(N, w.perm, posc4, w.cell_of, w.pos4, w.cell_slot);
+    // slot space from here on: a replica's slots are its caller index range, so atom_rep serves both
     const int nb128 = (N + 127) / 128;
-    k_count<<<nb128, 128, 0, c->s>>>(N, w.pos4, w.atom_rep, w.cell_of, w.rgrid_dims, w.cell_start, w.cell_atoms,
-                                  c->rl2, c->box, w.rowcnt);
-    c->launches += 2;
+    k_count<<<nb128, 128, 0, c->s>>>(N, w.pos4, w.atom_rep, w.cell_slot, w.rgrid_dims, w.cell_start, nullptr,
+                                     c->rl2, c->box, w.rowcnt);
+    c->launches += 4;
     if ((err = scan_exclusive(c, w.rowcnt, N, w.row_ptr, &w.meta->n_edges)) != cudaSuccess) return err;
     k_check_capacity<<<1, 1, 0, c->s>>>(c->cap, w.meta);
-    k_fill<<<nb128, 128, 0, c->s>>>(N, w.pos4, w.atom_rep, w.cell_of, w.rgrid_dims, w.cell_start, w.cell_atoms,
-                                 c->rl2, c->box, w.row_ptr, c->cap, w.meta, w.coltmp, w.erow);
+    k_fill<<<nb128, 128, 0, c->s>>>(N, w.pos4, w.atom_rep, w.cell_slot, w.rgrid_dims, w.cell_start, nullptr,
+                                    c->rl2, c->box, w.row_ptr, c->cap, w.meta, w.coltmp, w.erow);
     int nsort = c->nsm * 8;
     k_sort_rows<<<nsort, 256, 0, c->s>>>(N, w.row_ptr, w.coltmp, c->cap, w.meta, w.col);
     k_rev<<<c->nsm * 8, 256, 0, c->s>>>(w.row_ptr, w.col, w.erow, c->cap, w.meta, w.rev);
     k_partition<<<(c->ncta + 1 + 127) / 128, 128, 0, c->s>>>(N, c->ncta, w.row_ptr, c->cap, w.meta, w.part);
     cudaMemcpyAsync(w.ref4, w.pos4, sizeof(float4) * N, cudaMemcpyDeviceToDevice, c->s);
     c->launches += 5;
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// the list and per-atom values in the caller's atom order (inspection taps)
+// ---------------------------------------------------------------------------
+__global__ void k_caller_rowlen(int n, const int32_t* __restrict__ perm, const int32_t* __restrict__ row_ptr,
+                                int32_t* __restrict__ cnt)
+{
+    int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= n) return;
+    cnt[perm[k]] = row_ptr[k + 1] - row_ptr[k];
+}
+
+// one warp per slot row: its columns, as caller indices, at the caller row's place
+__global__ void k_caller_cols(int n, const int32_t* __restrict__ perm, const int32_t* __restrict__ row_ptr,
+                              const int32_t* __restrict__ col, const int32_t* __restrict__ row_ptr_c, long long cap,
+                              const DevMeta* meta, int32_t* __restrict__ col_c)
+{
+    if (meta->n_edges > cap) return;
+    int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int lane = threadIdx.x & 31;
+    int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int k = warp; k < n; k += nwarps) {
+        const int a = row_ptr[k], b = row_ptr[k + 1], base = row_ptr_c[perm[k]];
+        for (int e = a + lane; e < b; e += 32) col_c[base + (e - a)] = perm[col[e]];
+    }
+}
+
+__global__ void k_scatter_atoms(int n, const int32_t* __restrict__ perm, const float* __restrict__ v,
+                                float* __restrict__ out)
+{
+    int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k < n) out[perm[k]] = v[k];
+}
+
+__global__ void k_rev_rows(int n, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
+                           long long cap, const DevMeta* meta, int32_t* __restrict__ rev);
+
+// Caller-order CSR of the current list in (row_ptr, col, rev) = (rowcnt, ccol,
+// cidx): scratch that only a build (rowcnt, coltmp) or the start of the next
+// energy evaluation (ccol, cidx) rewrites.
+cudaError_t launch_caller_order_list(schnet_ctx* c, const int32_t** row_ptr, const int32_t** col,
+                                     const int32_t** rev)
+{
+    Workspace& w = c->ws;
+    const int N = c->N;
+    cudaError_t err;
+    k_caller_rowlen<<<(N + 255) / 256, 256, 0, c->s>>>(N, w.perm, w.row_ptr, w.rowcnt);
+    c->launches += 1;
+    if ((err = scan_exclusive(c, w.rowcnt, N, w.rowcnt, nullptr)) != cudaSuccess) return err;   // in place
+    k_caller_cols<<<c->nsm * 8, 256, 0, c->s>>>(N, w.perm, w.row_ptr, w.col, w.rowcnt, c->cap, w.meta, w.coltmp);
+    k_sort_rows<<<c->nsm * 8, 256, 0, c->s>>>(N, w.rowcnt, w.coltmp, c->cap, w.meta, w.ccol);
+    k_rev_rows<<<c->nsm * 8, 256, 0, c->s>>>(N, w.rowcnt, w.ccol, c->cap, w.meta, w.cidx);
+    c->launches += 3;
+    *row_ptr = w.rowcnt;
+    *col = w.ccol;
+    *rev = w.cidx;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_atoms(schnet_ctx* c, const float* v, float* out)
+{
+    k_scatter_atoms<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, c->ws.perm, v, out);
+    c->launches += 1;
     return cudaGetLastError();
 }
 
@@ -634,7 +751,7 @@ extern "C" schnet_status schnet_build_neighbors_noalloc(const float* d_pos, int3
     if (cudaMemsetAsync(meta, 0, sizeof(DevMeta), s) != cudaSuccess) return SCHNET_ERR_CUDA;
     if (cudaMemsetAsync(ccnt, 0, sizeof(int32_t) * (ncell + 1), s) != cudaSuccess) return SCHNET_ERR_CUDA;
     if (cudaMemsetAsync(cfill, 0, sizeof(int32_t) * (ncell + 1), s) != cudaSuccess) return SCHNET_ERR_CUDA;
-    k_pack_positions<<<nb, 256, 0, s>>>(N, d_pos, pos4, nullptr, 0, 0.f, meta);
+    k_pack_positions<<<nb, 256, 0, s>>>(N, d_pos, nullptr, pos4, nullptr, 0, 0.f, meta);
     k_atom_replica<<<nb, 256, 0, s>>>(N, R, d_replica_offsets, arep);
     k_replica_grid<<<R, 256, 0, s>>>(R, d_replica_offsets, pos4, gp, bx, dims, org, inv);
     k_cell_assign<<<nb, 256, 0, s>>>(N, pos4, arep, dims, org, inv, gp.periodic, cell_of, ccnt);

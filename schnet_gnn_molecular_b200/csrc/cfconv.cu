@@ -729,7 +729,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 // backward epilogue 1 for this warp's 32 edges: a = sp2(p), b = ssp'(x) dx/dd, with
 // p = x log2e = s1 log2e P + b1 log2e and dx/dd = s1 2ln2 P' (P' from the scaled
 // Gaussian-derivative rows).  ssp'(x) = 1 / (1 + e^-x) shares 2^-|p| with sp2.
-// a goes to B rows e, b to B rows TE + e of GEMM2's operand.
+// a goes to B rows e, b to B rows TE + e of GEMM2's operand.  Pairs of
+// elements share the packed fp32x2 FMA/FMUL/FADD instructions.
 template <int FMT, int NX, int TE>
 __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* act,
                                        int col0, int f)
@@ -741,14 +742,20 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
         tmem_ld16(tPd + hh * 16, rd);
         tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            const float p = fmaf(s1L, r[q], b1L);
-            const float t = ex2_mufu(-fabsf(p));
-            const float y = 1.0f + t;
-            const float inv = rcp_1to2(y);                    // y = 1 + 2^-|p| in [1, 2]
-            const float sg = p >= 0.0f ? inv : t * inv;       // logistic(x)
-            r[q] = fmaxf(p, 0.0f) + lg2_mufu(y);
-            rd[q] = sg * (s1d * rd[q]);
+        for (int q = 0; q < 16; q += 2) {
+            const float2 p = fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L));
+            const float2 t = make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y)));
+            const float2 y = add2(dup2(1.0f), t);
+            const float2 inv = rcp2_1to2(y);                  // y = 1 + 2^-|p| in [1, 2]
+            const float2 ti = mul2(t, inv);
+            const float2 sg = make_float2(p.x >= 0.0f ? inv.x : ti.x, p.y >= 0.0f ? inv.y : ti.y);   // logistic(x)
+            const float2 a = add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)),
+                                  make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
+            const float2 d = mul2(sg, mul2(dup2(s1d), make_float2(rd[q], rd[q + 1])));
+            r[q] = a.x;
+            r[q + 1] = a.y;
+            rd[q] = d.x;
+            rd[q + 1] = d.y;
         }
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
@@ -789,6 +796,9 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     float* pf_s = reinterpret_cast<float*>(act);    // after GEMM2: [chunk][feature] partials
     float* pl_s = pf_s + NCH * 128;
     float* ps_s = pl_s + NCH * 128;                 // [quadrant][edge] partial of s_e
+    // per-warp [32 edges][36] scratch of the s_e transpose (behind the partials, inside the
+    // group's GEMM2 operand buffer, which is free between GEMM2's completion and the next E1)
+    float* s_w = reinterpret_cast<float*>(act + 4096) + (warp & 7) * (32 * 36);
     const int col0 = ch * 32;
     // accumulator columns: [P | P'] (64 each), then [Q | Q'] over them
     const uint32_t dacc = tmem + g * TM_ACC;
@@ -940,21 +950,24 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                             rd[q] = tval;
                         }
                     }
-                    // transpose-reduce the 16 per-edge values over the warp's 32 features:
-                    // afterwards lanes 2k and 2k+1 hold the sum for edge k of this half
+                    // stage this half's 16 per-edge values as S[edge][feature lane] (row stride 36:
+                    // the stores and the 16-byte row reads below are free of bank conflicts)
 #pragma unroll
-                    for (int sh = 16; sh >= 2; sh >>= 1) {
-                        const bool upper = (lane & sh) != 0;
-#pragma unroll
-                        for (int k = 0; k < sh / 2; ++k) {
-                            float send = upper ? rd[k] : rd[k + sh / 2];
-                            float keep = upper ? rd[k + sh / 2] : rd[k];
-                            rd[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
-                        }
-                    }
-                    rd[0] += __shfl_xor_sync(0xffffffffu, rd[0], 1);
-                    if ((lane & 1) == 0) ps_s[qd * TE + eb + hh * 16 + (lane >> 1)] = rd[0];
+                    for (int q = 0; q < 16; ++q) s_w[(hh * 16 + q) * 36 + lane] = rd[q];
                 }
+                // lane k sums edge k of the warp's chunk over the warp's 32 features (the same
+                // pairwise tree as a butterfly over the lanes)
+                __syncwarp();
+                {
+                    float v[32];
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 x = *reinterpret_cast<const float4*>(s_w + lane * 36 + c4 * 4);
+                        v[4 * c4] = x.x; v[4 * c4 + 1] = x.y; v[4 * c4 + 2] = x.z; v[4 * c4 + 3] = x.w;
+                    }
+                    ps_s[qd * TE + eb + lane] = tree_sum<32>(v);
+                }
+                __syncwarp();
                 if (kind == 1) {
                     pf = sf;
                 } else if (kind == 2) {

@@ -98,6 +98,16 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
+// rcp_1to2 of two values (the same seed and Newton steps, paired)
+__device__ __forceinline__ float2 rcp2_1to2(float2 y)
+{
+    float2 r = fma2(dup2(-0.47058823529411764f), y, dup2(1.4117647058823529f));
+    const float2 ny = make_float2(-y.x, -y.y);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) r = fma2(r, fma2(ny, r, dup2(1.0f)), r);
+    return r;
+}
+
 // sp2 of two values: max(p, 0) + log2(1 + 2^-|p|)
 __device__ __forceinline__ float2 sp2x2(float2 p)
 {

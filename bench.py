@@ -203,12 +203,14 @@ def _edge_stats(model, pos, w):
 
 def _traffic(kernel):
     """DRAM bytes per launch of `kernel` from the committed ncu capture, or None when
-    the kernel source has changed since that capture (hash recorded beside the figure)."""
+    the kernel sources have changed since that capture (hash recorded beside the figure)."""
     import hashlib
     try:
         d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-        src = open(os.path.join(ROOT, d["source"]), "rb").read()
-        if hashlib.sha256(src).hexdigest()[:16] != d["source_sha256_16"]:
+        h = hashlib.sha256()
+        for src in d["sources"]:
+            h.update(open(os.path.join(ROOT, src), "rb").read())
+        if h.hexdigest()[:16] != d["sources_sha256_16"]:
             return None
         return d.get(kernel)
     except Exception:

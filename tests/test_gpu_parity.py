@@ -135,13 +135,14 @@ def test_fp16_fast_mode():
     assert energy_rel(E, E32, eps32, ro) <= ENERGY_RTOL_16BIT
 
 
-def test_isolated_atoms_and_empty_rows():
-    # three replicas: a lone bead, two far-apart beads, and a short chain
-    w = workloads.TINY.with_(n_replicas=3, beads=1)
+@pytest.mark.parametrize("ro", [[0, 1, 3, 13], [0, 0, 1, 3, 13], [0, 1, 1, 3, 13, 13]],
+                         ids=["three", "empty_first", "empty_inner_and_last"])
+def test_isolated_atoms_and_empty_rows(ro):
+    # replicas: a lone bead, two far-apart beads, a short chain, and replicas without atoms
+    w = workloads.TINY.with_(n_replicas=len(ro) - 1, beads=1)
     rng = np.random.default_rng(5)
     chain = inputs.chain(10, rng)
     pos = np.concatenate([[[0.0, 0, 0]], [[0.0, 0, 0], [50.0, 0, 0]], chain]).astype(np.float32)
-    ro = [0, 1, 3, 13]
     types = inputs.bead_types(13, w.n_types, rng)
     weights = workloads.weights(workloads.TINY, bias_scale=0.3)
     model = api.SchNet(n_types=w.n_types, F=w.F, K=w.K, L=w.L, rbf_min=w.rbf_min, rbf_max=w.rbf_max,
@@ -150,6 +151,7 @@ def test_isolated_atoms_and_empty_rows():
     m = oracle_model(workloads.TINY, weights)
     Eo, eps_o, Fo = oracle.energy_forces(m, pos.astype(np.float64), types, ro)
     assert energy_rel(E, Eo, eps_o, ro) <= ENERGY_RTOL
+    assert np.all(E[np.diff(ro) == 0] == 0.0)
     assert np.all(F[:3] == 0.0)
     assert rel_frobenius(F, Fo) <= FORCE_RTOL
 

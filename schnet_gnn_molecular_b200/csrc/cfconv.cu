@@ -609,7 +609,8 @@ __device__ __forceinline__ void issue_gemm1(uint32_t tmem, uint32_t dacc, uint32
 // ---------------------------------------------------------------------------
 // Per group and tile t: [GEMM1(t) in flight] E1 -> issue GEMM2 -> stage R of
 // t+2 (into the group's own GEMM1 operand and second metadata buffer) and the
-// first gather under GEMM2 -> E2 -> issue GEMM1(t+2) -> merge under GEMM1(t+2).
+// first gather under GEMM2 -> E2 -> issue GEMM1(t+2) (by warp 4) -> merge under GEMM1(t+2)
+// (warps 0-3).
 template <int FMT, int NW, int NX>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {
@@ -709,7 +710,9 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         }
         tc_fence_before();
         group_sync(g);          // Q read out; partials and the next tile's Gaussians in place
-        if (next && mt == 0) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
+        // GEMM1(t+2) is issued by warp 4, which takes no part in the merge below (an issuing
+        // thread blocks while the tensor core's queue is full)
+        if (next && mt == 128) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
         if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
         group_sync(g);          // merge done with the partials before E1 of the next tile overwrites them
@@ -986,7 +989,9 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         }
         tc_fence_before();
         group_sync(g);          // Q, Q' read out; partials and the next tile's Gaussians in place
-        if (next && mt == 0) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
+        // GEMM1(t+2) is issued by warp 4, which takes no part in the merge below (an issuing
+        // thread blocks while the tensor core's queue is full)
+        if (next && mt == 128) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
         if (mt < ne) {
             const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];

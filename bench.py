@@ -298,16 +298,13 @@ def run_native(args):
                     "flop_per_launch": flops, "ms_per_launch": round(kms, 4),
                     "per_kernel_ms_per_step": {k: round(x[0] / n_rb, 4) for k, x in prof.items()},
                     "kernel_share": {k: round(x[0] / tot_ms, 4) for k, x in prof.items()}}
-        cfg = {"workload": w.name, "replicas": w.n_replicas, "beads_per_replica": w.beads, "atoms": w.n_atoms,
-               "F": w.F, "K": w.K, "L": w.L, "cutoff_A": w.cutoff, "skin_A": w.skin, "n_rebuild": n_rb,
-               "dt_fs": w.dt_fs, "integrator": "BAOAB" if w.gamma_per_ps > 0 else "velocity Verlet",
-               "weight_dtype": w.weight_dtype, "edges_listed": E_list, "edges_within_cutoff": E_cut,
+        cfg = dict(_workload_config(w, n_rb, ws))
+        cfg.update({"edges_listed": E_list, "edges_within_cutoff": E_cut,
                "edges_within_cutoff_at_start": edges_start[1],
                "edges_note": "no bonded terms: chains slowly expand, so the graph shrinks during the run; "
                              "edges_within_cutoff is counted after the timed steps",
                "l2": "no flush: state carried step to step; per-step working set "
-                     f"{(E_list * 20 + w.n_atoms * 128 * 4 * (2 * w.L + 4)) / 1e6:.0f} MB > 126 MB L2",
-               "parallelism": f"replicas x{ws} ranks (independent)"}
+                     f"{(E_list * 20 + w.n_atoms * 128 * 4 * (2 * w.L + 4)) / 1e6:.0f} MB > 126 MB L2"})
         out = {"metric": METRIC, "value": round(value, 1), "unit": "atom-steps/s", "n_gpus": ws, "steps": steps,
                "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 4), "higher_is_better": True,
                "scaling": "weak", "vs_baseline": None, "dtype": "f32",
@@ -405,6 +402,14 @@ def run_drift(args):
     print(json.dumps(out), flush=True)
 
 
+def _workload_config(w, n_rebuild, ranks):
+    """The static description of a workload, shared by both arms' `config`."""
+    return {"workload": w.name, "replicas": w.n_replicas, "beads_per_replica": w.beads, "atoms": w.n_atoms,
+            "F": w.F, "K": w.K, "L": w.L, "cutoff_A": w.cutoff, "skin_A": w.skin, "n_rebuild": n_rebuild,
+            "dt_fs": w.dt_fs, "integrator": "BAOAB" if w.gamma_per_ps > 0 else "velocity Verlet",
+            "weight_dtype": w.weight_dtype, "parallelism": f"replicas x{ranks} ranks (independent)"}
+
+
 def run_reference(args):
     """The float64 oracle as the reference arm (rank 0 only).  One step = one BAOAB
     step of a replica-shaped sample: a whole replica when the run fits the time
@@ -449,7 +454,8 @@ def run_reference(args):
     out = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "atom-steps/s", "n_gpus": ws,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": w.name, "sample": what},
+           "config": dict(_workload_config(w, w.n_rebuild, ws),
+                          sample=what),
            "cpu_baseline": {"value": round(value, 2), "unit": "atom-steps/s", "cores": cores, "kind": "oracle",
                             "sample": f"{args.steps} BAOAB steps of {what}"},
            "e2e": {"value": round(value, 2), "unit": "atom-steps/s", "h2d_bytes_per_step": 0,

@@ -226,6 +226,12 @@ SCHNET_API schnet_status schnet_get_neighbors(schnet_ctx *ctx, int32_t *h_row_pt
  * caller's atom order.  Errors: INVALID_ARG, STATE (no list), CUDA. */
 SCHNET_API schnet_status schnet_get_atom_energies(schnet_ctx *ctx, float *d_eps);
 
+/* Test tap: d_y[i] = 2^d_x[i] (device float32 arrays of n elements, d_x[i] <= 0;
+ * arguments below -30 are taken as -30) by the FMA-pipe exponential that part of
+ * the forward filter's softplus uses, enqueued on cuda_stream (a cudaStream_t,
+ * NULL = legacy default stream).  Errors: INVALID_ARG, CUDA. */
+SCHNET_API schnet_status schnet_test_exp2(const float *d_x, float *d_y, int64_t n, void *cuda_stream);
+
 /* Kernel classes reported by schnet_profile_steps. */
 enum {
     SCHNET_KERNEL_CFCONV_FWD = 0,  /* fused radial basis + filter MLP + message passing, forward */

@@ -560,7 +560,10 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
     tmem_ld_wait();
 #pragma unroll
     for (int q = 0; q < 32; q += 2) {
-        const float2 v = sp2x2(fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L)));
+        // one pair in four takes its exponentials on the FMA pipe: the MUFU, which the
+        // logarithms and the other exponentials keep busy, is this epilogue's bottleneck
+        const float2 pp = fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L));
+        const float2 v = ((q >> 1) & 3) == 3 ? sp2x2_fma(pp) : sp2x2(pp);
         r[q] = v.x;
         r[q + 1] = v.y;
     }
@@ -1170,3 +1173,26 @@ cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s)
 }
 
 }  // namespace schnet
+
+// ---------------------------------------------------------------------------
+// test tap: the FMA-pipe exponential on its own
+// ---------------------------------------------------------------------------
+namespace schnet {
+__global__ void k_test_exp2(const float* __restrict__ x, float* __restrict__ y, long long n)
+{
+    const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float2 v = ex2_fma2(make_float2(x[i], i + 1 < n ? x[i + 1] : 0.0f));
+    y[i] = v.x;
+    if (i + 1 < n) y[i + 1] = v.y;
+}
+}  // namespace schnet
+
+extern "C" schnet_status schnet_test_exp2(const float* d_x, float* d_y, int64_t n, void* cuda_stream)
+{
+    if (!d_x || !d_y || n < 0) return SCHNET_ERR_INVALID_ARG;
+    if (n == 0) return SCHNET_OK;
+    const long long pairs = (n + 1) / 2;
+    schnet::k_test_exp2<<<(unsigned)((pairs + 255) / 256), 256, 0, (cudaStream_t)cuda_stream>>>(d_x, d_y, n);
+    return cudaGetLastError() == cudaSuccess ? SCHNET_OK : SCHNET_ERR_CUDA;
+}

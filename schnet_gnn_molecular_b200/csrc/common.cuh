@@ -115,6 +115,37 @@ __device__ __forceinline__ float2 sp2x2(float2 p)
     return add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
 }
 
+// 2^x for two arguments x <= 0 on the FMA and integer pipes instead of the MUFU.
+// x is clamped at -30 (2^-30 is below half an ulp of 1, so 1 + 2^x rounds the same;
+// a NaN is clamped too: non-finite inputs are flagged where the positions enter).
+// Cody-Waite reduction x = n + f with n = round(x), found by adding and removing
+// 1.5 * 2^23, and f in [-1/2, 1/2]; 2^f by the degree-5 polynomial that
+// exp2_fit.py fits (reweighted least squares on Chebyshev nodes; relative error
+// <= 2.2e-7 in float32 Horner form); 2^n is added to the exponent field.
+__device__ __forceinline__ float2 ex2_fma2(float2 x)
+{
+    constexpr float RND = 12582912.0f;
+    x = make_float2(fmaxf(x.x, -30.0f), fmaxf(x.y, -30.0f));
+    const float2 y = add2(x, dup2(RND));
+    const float2 n = add2(y, dup2(-RND));
+    const float2 f = fma2(n, dup2(-1.0f), x);
+    float2 p = fma2(dup2(0.0013276470126584172f), f, dup2(0.009675540961325169f));
+    p = fma2(p, f, dup2(0.05550713092088699f));
+    p = fma2(p, f, dup2(0.24022120237350464f));
+    p = fma2(p, f, dup2(0.6931469440460205f));
+    p = fma2(p, f, dup2(1.0000001192092896f));
+    const int kx = (__float_as_int(y.x) - __float_as_int(RND)) << 23;
+    const int ky = (__float_as_int(y.y) - __float_as_int(RND)) << 23;
+    return make_float2(__int_as_float(__float_as_int(p.x) + kx), __int_as_float(__float_as_int(p.y) + ky));
+}
+
+// sp2x2 with its exponentials from ex2_fma2 (the logarithms stay on the MUFU)
+__device__ __forceinline__ float2 sp2x2_fma(float2 p)
+{
+    const float2 y = add2(dup2(1.0f), ex2_fma2(make_float2(-fabsf(p.x), -fabsf(p.y))));
+    return add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
+}
+
 // ssp(x) and ssp'(x) sharing one exponential
 __device__ __forceinline__ void ssp_and_grad(float x, float& s, float& g)
 {

@@ -292,6 +292,11 @@ def run_native(args):
         peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
         achieved = flops / (kms * 1e-3) / 1e12
         traffic = _traffic(dominant)
+        k_interval = max(1, int(round(launches / steps * n_rb)))
+        floor = {"ms_per_step": round(_launch_floor(dev, k_interval) / n_rb, 4),
+                 "kernels_per_step": round(launches / steps, 2),
+                 "how": f"one CUDA Graph of {k_interval} trivial kernels (one rebuild interval's count), "
+                        f"replayed; per step = replay time / {n_rb}"}
         roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 2),
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                     "peak_source": f"{src} dense bf16/fp16 sustained",
@@ -311,7 +316,8 @@ def run_native(args):
                "mma": "fp16 hi/lo split operands, fp32 accumulate (tcgen05 kind::f16)", "data": "synthetic",
                "ns_per_day_per_replica": round(ns_day_rep, 2),
                "ns_per_day_aggregate": round(ns_day_rep * w.n_replicas * ws, 1),
-               "config": cfg, "gpu_launches": int(launches), "clocks": clk, "roofline": roofline,
+               "config": cfg, "gpu_launches": int(launches), "launch_floor": floor, "clocks": clk,
+               "roofline": roofline,
                "memory": memory,
                "status": {"warmup": nat_status(flagged[0]), "timed": nat_status(flagged[1])}}
         if not args.no_e2e:
@@ -400,6 +406,33 @@ def run_drift(args):
                       "skin_A": w.skin, "read_every_steps": chunk}, "data": "synthetic"}
     model.close()
     print(json.dumps(out), flush=True)
+
+
+def _launch_floor(dev, kernels, reps=20):
+    """Device time of one CUDA Graph of `kernels` trivial one-element kernels (the
+    replay floor a graph of that many nodes cannot beat on this GPU), in ms."""
+    import torch
+    x = torch.zeros(1, device=dev)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        x.add_(1.0)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(kernels):
+            x.add_(1.0)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / reps
+    del g
+    return ms
 
 
 def _workload_config(w, n_rebuild, ranks):

@@ -232,6 +232,14 @@ SCHNET_API schnet_status schnet_get_atom_energies(schnet_ctx *ctx, float *d_eps)
  * NULL = legacy default stream).  Errors: INVALID_ARG, CUDA. */
 SCHNET_API schnet_status schnet_test_exp2(const float *d_x, float *d_y, int64_t n, void *cuda_stream);
 
+/* Test tap: the give-up path of the library's device-side waits, on its own.  One
+ * CTA holds tensor memory and waits on an mbarrier for at most max_polls polls;
+ * with complete = 0 nothing completes the barrier, so the wait gives up, raises
+ * SCHNET_FLAG_TIMEOUT in the context's status word, releases the tensor memory and
+ * returns (complete = 1: the barrier completes at once, no flag).  Read the flag
+ * with schnet_get_status; the context stays usable.  Errors: INVALID_ARG, CUDA. */
+SCHNET_API schnet_status schnet_test_timeout(schnet_ctx *ctx, uint32_t max_polls, int32_t complete);
+
 /* Kernel classes reported by schnet_profile_steps. */
 enum {
     SCHNET_KERNEL_CFCONV_FWD = 0,  /* fused radial basis + filter MLP + message passing, forward */

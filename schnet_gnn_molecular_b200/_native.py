@@ -20,7 +20,7 @@ WEIGHT_DTYPES = {"fp32": 0, "fp16": 1, "bf16": 2, "fp16fast": 3}
 EXPORTED = ["schnet_workspace_bytes", "schnet_create", "schnet_build_neighbors", "schnet_energy_forces",
             "schnet_step", "schnet_step_host", "schnet_get_status", "schnet_last_error", "schnet_destroy",
             "schnet_get_neighbors", "schnet_get_atom_energies", "schnet_kernel_launches", "schnet_profile_steps",
-            "schnet_build_neighbors_noalloc", "schnet_test_exp2"]
+            "schnet_build_neighbors_noalloc", "schnet_test_exp2", "schnet_test_timeout"]
 KERNEL_CLASSES = ["cfconv_fwd", "cfconv_bwd", "atomwise", "neighbors", "forces", "integrate", "reduce", "mask"]
 
 
@@ -74,6 +74,7 @@ def load() -> C.CDLL:
     L.schnet_get_neighbors.argtypes = [vp, vp, vp, vp, i64p, C.c_int64]
     L.schnet_get_atom_energies.argtypes = [vp, vp]
     L.schnet_test_exp2.argtypes = [vp, vp, C.c_int64, vp]
+    L.schnet_test_timeout.argtypes = [vp, C.c_uint32, C.c_int32]
     L.schnet_profile_steps.argtypes = [vp, vp, vp, vp, vp, C.c_int64, C.POINTER(StepParams), dp, i64p]
     L.schnet_build_neighbors_noalloc.argtypes = [vp, C.c_int32, C.c_int32, vp, C.c_float, C.c_float, C.c_int32,
                                                  C.POINTER(C.c_float), vp, vp, vp, C.c_int64, vp, vp]

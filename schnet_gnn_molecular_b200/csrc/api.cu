@@ -763,6 +763,15 @@ schnet_status schnet_profile_steps(schnet_ctx* c, float* d_pos, float* d_vel, co
     return status_from_flags(flags);
 }
 
+schnet_status schnet_test_timeout(schnet_ctx* c, uint32_t max_polls, int32_t complete)
+{
+    if (!c || max_polls < 1) return SCHNET_ERR_INVALID_ARG;
+    join_in(c);
+    CK(launch_test_timeout(c, max_polls, complete ? 1 : 0));
+    CK(join_out(c));
+    return SCHNET_OK;
+}
+
 int64_t schnet_kernel_launches(const schnet_ctx* c) { return c ? c->launches : 0; }
 
 }  // extern "C"

@@ -132,6 +132,7 @@ cudaError_t launch_build_neighbors(schnet_ctx* c, const float* d_pos);
 cudaError_t launch_caller_order_list(schnet_ctx* c, const int32_t** row_ptr, const int32_t** col,
                                      const int32_t** rev);
 cudaError_t launch_scatter_atoms(schnet_ctx* c, const float* v, float* out);
+cudaError_t launch_test_timeout(schnet_ctx* c, uint32_t max_polls, int complete);
 cudaError_t launch_energy_forces(schnet_ctx* c, const int32_t* d_types, double* d_energy, float* d_forces);
 cudaError_t launch_baoa(schnet_ctx* c, float* d_pos, float* d_vel, const float* d_mass, float dt, float gamma,
                         float temp, unsigned long long seed, const float* d_noise, bool check_skin);

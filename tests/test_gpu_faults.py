@@ -1,6 +1,7 @@
 """Failure detection without GPU faults: every fault is made on the host (bad
-input, undersized buffer, moved atom) and must come back as a status, with the
-context still usable afterwards."""
+input, undersized buffer, moved atom) or is a bounded device-side wait that
+nothing completes, and must come back as a status, with the context still
+usable afterwards."""
 import ctypes as C
 
 import numpy as np
@@ -77,6 +78,35 @@ def test_step_reports_flags_as_status():
     types[0] = -1
     _, _, st = m.step(p, v, _dev(types, torch.int32), _dev(workloads.masses(W)), 2, raise_on_flag=False)
     assert st == 6   # SCHNET_ERR_BADTYPE
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    lib = nat.load()
+    pos = workloads.positions(W)
+    types = workloads.types(W)
+    m = _model()
+    p, t = _dev(pos), _dev(types, torch.int32)
+    m.build_neighbors(p)
+    E0, F0 = m.energy_forces(p, t)
+    assert m.status() == 0
+    # a barrier that completes: the wait succeeds, no flag
+    assert lib.schnet_test_timeout(m.ctx, 1000, 1) == 0
+    assert m.status() == 0
+    # a barrier nothing completes: the wait gives up after its polls and raises TIMEOUT
+    assert lib.schnet_test_timeout(m.ctx, 1000, 0) == 0
+    assert m.status() == nat.FLAG_TIMEOUT
+    assert m.status() == 0                      # the read cleared it
+    # the context (and its tensor memory) is still usable: the same results again
+    E1, F1 = m.energy_forces(p, t)
+    torch.cuda.synchronize()
+    assert m.status() == 0
+    assert torch.equal(E0, E1) and torch.equal(F0, F1)
+    # a step reports a flag raised before it as its status
+    assert lib.schnet_test_timeout(m.ctx, 1000, 0) == 0
+    v = torch.zeros((W.n_atoms, 3), device="cuda")
+    _, _, st = m.step(p, v, t, _dev(workloads.masses(W)), 1, raise_on_flag=False)
+    assert st == 8   # SCHNET_ERR_TIMEOUT
+    assert lib.schnet_test_timeout(None, 1000, 0) == 1 and lib.schnet_test_timeout(m.ctx, 0, 0) == 1
 
 
 def test_argument_errors_and_state():

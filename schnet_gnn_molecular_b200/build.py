@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libschnet_b200.so")
-SOURCES = ["api.cu", "neighbors.cu", "cfconv.cu", "atomwise.cu", "integrate.cu"]
+SOURCES = ["api.cu", "neighbors.cu", "cfconv.cu", "atomwise.cu", "integrate.cu", "taps.cu"]
 HEADERS = ["common.cuh", "internal.h", os.path.join("..", "..", "include", "schnet.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

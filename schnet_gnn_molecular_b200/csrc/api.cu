@@ -512,7 +512,8 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
     SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd_top(c));
     for (int l = c->L - 1; l >= 0; --l) {
         SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_bwd(c, l, l < c->L - 1 ? 1 : 0));
-        SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd(c, l));
+        // interaction 0: dE/dx^0 is a gradient with respect to the embedding, not needed for forces
+        if (l > 0) SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd(c, l));
     }
     SCHNET_TIMED(SCHNET_KERNEL_FORCES, launch_forces(c, forces));
 #undef SCHNET_TIMED

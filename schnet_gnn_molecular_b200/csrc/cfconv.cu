@@ -524,13 +524,14 @@ __device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslo
     return tmem;
 }
 
-// Common epilogue: the carried row is complete; rows after it without edges are zero.
+// Common epilogue: the carried row is complete; rows after it without edges are zero
+// (nothing to write when the kernel produces no per-row output).
 __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r1, float* __restrict__ out, bool ok,
                                               uint64_t* bars, const uint32_t* phases, const uint32_t* pending,
-                                              uint32_t tmem)
+                                              uint32_t tmem, bool write_out = true)
 {
     const int warp = threadIdx.x >> 5;
-    if (ok) {
+    if (ok && write_out) {
         if (threadIdx.x < FP) {
             const int cur = cy->cur[(ntiles + 1) & 1];
             out[(size_t)cur * FP + threadIdx.x] = cy->acc[threadIdx.x];
@@ -772,7 +773,10 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
     }
 }
 
-template <int FMT, int NW, int NX>
+// DH = false: only the per-edge s_e (forces) -- no dE/dh_j segment sums, no u_j
+// gathers, no merge.  Used for the first interaction, whose dE/dh feeds only the
+// gradient with respect to the embedding, which forces do not need.
+template <int FMT, int NW, int NX, bool DH>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
     constexpr int TE = TE_B;
@@ -872,7 +876,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         }
         const int eb = col0;
         float uv[16], hv[16];
-        gather<16>(u_f, tm->col, eb, uv);
+        if (DH) gather<16>(u_f, tm->col, eb, uv);
         gather<16>(h_f, tm->col, eb, hv);
         if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2(t) done
         pending = 0;
@@ -894,7 +898,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     if (hh == 1) {
-                        gather<16>(u_f, tm->col, eb + 16, uv);
+                        if (DH) gather<16>(u_f, tm->col, eb + 16, uv);
                         gather<16>(h_f, tm->col, eb + 16, hv);
                     }
                     float r[16], rd[16];
@@ -913,7 +917,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                             for (int i = 0; i < 4; ++i) {
                                 const int q = gq + i;
                                 const float z = fmaf(s2L, r[q], b2s);
-                                sf = fmaf(fc[i] * z, uv[q], sf);
+                                if (DH) sf = fmaf(fc[i] * z, uv[q], sf);
                                 const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
                                 rd[q] = wd * (u_first * hv[q]);
                             }
@@ -928,10 +932,12 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                             for (int i = 0; i < 4; ++i) {
                                 const int q = gq + i;
                                 const float z = fmaf(s2L, r[q], b2s);
-                                const float dt = fc[i] * z * uv[q];
                                 const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
-                                sf += first ? dt : 0.f;
-                                sl += first ? 0.f : dt;
+                                if (DH) {
+                                    const float dt = fc[i] * z * uv[q];
+                                    sf += first ? dt : 0.f;
+                                    sl += first ? 0.f : dt;
+                                }
                                 const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
                                 rd[q] = wd * ((first ? u_first : u_last) * hv[q]);
                             }
@@ -944,13 +950,14 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                             if (e < ne) {
                                 const int row = __ldg(rows_g + e);
                                 if (row != c.lrow) {
-                                    seg_row(c, row, a.out, f);
+                                    if (DH) seg_row(c, row, a.out, f);
+                                    else c.lrow = row;
                                     u_row = __ldg(u_f + (size_t)row * FP);
                                 }
                                 const float fcq = fcp[q], dfcq = dfcp[q];
                                 const float z = fmaf(s2L, r[q], b2s);
                                 const float wd = fmaf(dfcq, z, fcq * (s2 * rd[q]));
-                                c.acc = fmaf(fcq * z, uv[q], c.acc);
+                                if (DH) c.acc = fmaf(fcq * z, uv[q], c.acc);
                                 tval = wd * (u_row * hv[q]);
                             }
                             rd[q] = tval;
@@ -974,7 +981,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                     ps_s[qd * TE + eb + lane] = tree_sum<32>(v);
                 }
                 __syncwarp();
-                if (kind == 1) {
+                if (!DH) {
+                } else if (kind == 1) {
                     pf = sf;
                 } else if (kind == 2) {
                     pf = sf;
@@ -987,8 +995,10 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                     pl = c.acc;
                 }
             }
-            pf_s[ch * 128 + f] = pf;
-            pl_s[ch * 128 + f] = pl;
+            if (DH) {
+                pf_s[ch * 128 + f] = pf;
+                pl_s[ch * 128 + f] = pl;
+            }
         }
         tc_fence_before();
         group_sync(g);          // Q, Q' read out; partials and the next tile's Gaussians in place
@@ -1000,7 +1010,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];
             a.s_edge[my_g] = a.accumulate_s ? my_so + sv : sv;
         }
-        if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
+        if (DH && !(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
         group_sync(g);          // merge and s_e done with the partials before E1 of the next tile overwrites them
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
@@ -1009,7 +1019,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         pend_s[g] = ok ? 0u : pending;
     }
     const bool all_ok = __syncthreads_or(!ok) == 0;
-    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem);
+    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, DH);
 }
 
 // ---------------------------------------------------------------------------
@@ -1122,7 +1132,10 @@ static cudaError_t set_attrs()
     cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_bytes<TE_F, false>());
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_bytes<TE_B, true>());
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_bytes<TE_B, true>());
 }
 
@@ -1154,20 +1167,29 @@ cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
     return cudaGetLastError();
 }
 
+template <bool DH>
+static void launch_bwd(schnet_ctx* c, const MPArgs& a)
+{
+    const size_t sm = smem_bytes<TE_B, true>();
+    if (c->n_xterms == 1)
+        k_cfconv_bwd<0, 1, 1, DH><<<c->ncta, NT, sm, c->s>>>(a);
+    else if (c->weight_fmt == 0 && c->n_wterms == 2)
+        k_cfconv_bwd<0, 2, 2, DH><<<c->ncta, NT, sm, c->s>>>(a);
+    else if (c->weight_fmt == 0)
+        k_cfconv_bwd<0, 1, 2, DH><<<c->ncta, NT, sm, c->s>>>(a);
+    else
+        k_cfconv_bwd<1, 1, 2, DH><<<c->ncta, NT, sm, c->s>>>(a);
+}
+
+// Interaction 0's dE/dh feeds only the gradient with respect to the embedding,
+// which forces do not need: its launch computes s_e alone.
 cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s)
 {
     MPArgs a = make_args(c, layer);
     a.out = c->ws.dh;
     a.accumulate_s = accumulate_s;
-    const size_t sm = smem_bytes<TE_B, true>();
-    if (c->n_xterms == 1)
-        k_cfconv_bwd<0, 1, 1><<<c->ncta, NT, sm, c->s>>>(a);
-    else if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_bwd<0, 2, 2><<<c->ncta, NT, sm, c->s>>>(a);
-    else if (c->weight_fmt == 0)
-        k_cfconv_bwd<0, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
-    else
-        k_cfconv_bwd<1, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
+    if (layer > 0) launch_bwd<true>(c, a);
+    else launch_bwd<false>(c, a);
     c->launches += 1;
     return cudaGetLastError();
 }

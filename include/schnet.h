@@ -160,7 +160,8 @@ SCHNET_API schnet_status schnet_build_neighbors(schnet_ctx *ctx, const float *d_
 
 /* Energy per replica and forces at d_pos using the current list.
  * d_types: device int32 [N]; d_energy: device float64 [R] (kcal/mol);
- * d_forces: device float32 [N][3] (kcal/mol/A), may be NULL for energy only.
+ * d_forces: device float32 [N][3] (kcal/mol/A), may be NULL for energy only (then no backward
+ * pass runs).
  * Sets SCHNET_FLAG_SKIN if an atom moved more than skin/2 since the build,
  * SCHNET_FLAG_BADTYPE for a type outside [0, T) (treated as type 0).
  * Errors: INVALID_ARG, STATE (no list built), CUDA. */

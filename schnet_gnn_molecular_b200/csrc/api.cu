@@ -404,7 +404,7 @@ cudaError_t enqueue_steps(schnet_ctx* c, int k, bool build_first, float* pos, fl
                                  p->d_noise, true)) != cudaSuccess)
                 return e;
         }
-        if ((e = launch_energy_forces(c, types, epot, nullptr)) != cudaSuccess) return e;
+        if ((e = launch_energy_forces(c, types, epot, nullptr, true)) != cudaSuccess) return e;
         {
             Timed t(c, SCHNET_KERNEL_INTEGRATE);
             if ((e = launch_b_kick(c, vel, mass, p->dt_fs, ekin)) != cudaSuccess) return e;
@@ -461,7 +461,7 @@ schnet_status step_impl(schnet_ctx* c, float* pos, float* vel, const int32_t* ty
         c->have_list = false;            // fresh start: the build below replaces the list
         CK(launch_build_neighbors(c, pos));
         c->have_list = true;
-        CK(launch_energy_forces(c, types, ep, nullptr));
+        CK(launch_energy_forces(c, types, ep, nullptr, true));
         c->since_build = p->n_rebuild;   // the first interval starts with a fresh build
     }
     if (c->since_build > p->n_rebuild) c->since_build = p->n_rebuild;
@@ -494,7 +494,9 @@ schnet_status step_impl(schnet_ctx* c, float* pos, float* vel, const int32_t* ty
 // ============================================================================
 // energy / forces orchestration
 // ============================================================================
-cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, double* energy, float* forces)
+// need_forces = false: energies only (no backward, internal forces left as they were)
+cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, double* energy, float* forces,
+                                         bool need_forces)
 {
     cudaError_t e;
 #define SCHNET_TIMED(kind, expr)                        \
@@ -509,6 +511,7 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
         SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_fwd(c, l));
     }
     SCHNET_TIMED(SCHNET_KERNEL_REDUCE, launch_replica_sum(c, c->ws.eps, energy ? energy : c->ws.epot));
+    if (!need_forces) return cudaSuccess;
     SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd_top(c));
     for (int l = c->L - 1; l >= 0; --l) {
         SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_bwd(c, l, l < c->L - 1 ? 1 : 0));
@@ -627,7 +630,7 @@ schnet_status schnet_energy_forces(schnet_ctx* c, const float* d_pos, const int3
     if (!c->have_list) return fail(c, SCHNET_ERR_STATE, "schnet_energy_forces: build the neighbour list first");
     join_in(c);
     CK(launch_pack_positions(c, d_pos));
-    CK(launch_energy_forces(c, d_types, d_energy, d_forces));
+    CK(launch_energy_forces(c, d_types, d_energy, d_forces, d_forces != nullptr));
     c->forces_valid = false;
     CK(join_out(c));
     return SCHNET_OK;

@@ -99,6 +99,20 @@ def test_energy_forces_periodic():
     assert rel_frobenius(F, Fo) <= FORCE_RTOL
 
 
+def test_energy_only_evaluation():
+    # d_forces = NULL runs no backward pass; the energies are those of the full evaluation
+    w = SMALL_PROTEIN
+    pos, types, weights, model = _setup(w, bias_scale=0.1)
+    p, t = _dev(pos, torch.float32), _dev(types, torch.int32)
+    model.build_neighbors(p)
+    E1, F1 = model.energy_forces(p, t)
+    E0, F0 = model.energy_forces(p, t, forces=False)
+    E2, F2 = model.energy_forces(p, t)
+    torch.cuda.synchronize()
+    assert F0 is None and model.status() == 0
+    assert torch.equal(E0, E1) and torch.equal(E2, E1) and torch.equal(F2, F1)
+
+
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 def test_sixteen_bit_filter_weights(dtype):
     w = SMALL_PROTEIN.with_(weight_dtype=dtype)

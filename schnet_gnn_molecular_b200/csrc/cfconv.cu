@@ -15,7 +15,9 @@
 //     accumulated in registers, no atomics, no edge tensor in HBM.
 // The backward kernel recomputes W and its distance derivative W' by forward-
 // mode tangents and produces dE/dh_j (segment sum over the symmetric list) and
-// the per-edge scalar s_e = sum_f W'_f u_i,f h_j,f (the edge's share of dE/dd).
+// the per-edge scalar s_e = sum_f W'_f u_i,f h_j,f (the edge's share of dE/dd);
+// for the first interaction, whose dE/dh only feeds the embedding's gradient,
+// it produces s_e alone.
 //
 // Tile orientation: the GEMMs are computed transposed, D[f][e] = W^T[f][k] B[e][k],
 // so TMEM lane = output feature and TMEM column = edge.  Each epilogue thread

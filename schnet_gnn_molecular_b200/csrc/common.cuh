@@ -50,7 +50,7 @@ __device__ __forceinline__ float sigmoidf(float x)
     return x >= 0.0f ? r : t * r;
 }
 
-// Single MUFU operations (PTX ex2.approx / lg2.approx / rcp.approx, denormals flushed).
+// Single MUFU operations (PTX ex2.approx / lg2.approx, denormals flushed).
 constexpr float LOG2EF = 1.44269504088896340736f;
 
 __device__ __forceinline__ float ex2_mufu(float x)
@@ -65,31 +65,6 @@ __device__ __forceinline__ float lg2_mufu(float x)
     asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-__device__ __forceinline__ float rcp_mufu(float x)
-{
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// Softplus in base 2: for p = x log2(e), sp2(p) = log2(1 + 2^p) = log2(1 + e^x),
-// so that ssp(x) = ln2 (sp2(p) - 1).  Written as max(p, 0) + log2(1 + 2^-|p|):
-// no overflow for any p, and 1 + 2^-|p| lies in [1, 2].
-__device__ __forceinline__ float sp2(float p)
-{
-    return fmaxf(p, 0.0f) + lg2_mufu(1.0f + ex2_mufu(-fabsf(p)));
-}
-
-// 1/y for y in [1, 2] on the FMA pipe (keeps the MUFU free): the linear seed
-// 24/17 - 8/17 y (relative error <= 1/17 on [1, 2]) refined by three Newton
-// steps r <- r + r (1 - y r), each squaring the relative error (1/17)^8 < 2e-10.
-__device__ __forceinline__ float rcp_1to2(float y)
-{
-    float r = fmaf(-0.47058823529411764f, y, 1.4117647058823529f);
-#pragma unroll
-    for (int i = 0; i < 3; ++i) r = fmaf(r, fmaf(-y, r, 1.0f), r);
-    return r;
-}
 
 // Two-wide fp32 arithmetic (sm_100 packed FFMA2 / FMUL2 / FADD2: two lanes of
 // ordinary round-to-nearest single precision per instruction).
@@ -98,7 +73,9 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-// rcp_1to2 of two values (the same seed and Newton steps, paired)
+// 1/y for two y in [1, 2] on the FMA pipe (keeps the MUFU free): the linear seed
+// 24/17 - 8/17 y (relative error <= 1/17 on [1, 2]) refined by three Newton
+// steps r <- r + r (1 - y r), each squaring the relative error (1/17)^8 < 2e-10.
 __device__ __forceinline__ float2 rcp2_1to2(float2 y)
 {
     float2 r = fma2(dup2(-0.47058823529411764f), y, dup2(1.4117647058823529f));
@@ -108,7 +85,9 @@ __device__ __forceinline__ float2 rcp2_1to2(float2 y)
     return r;
 }
 
-// sp2 of two values: max(p, 0) + log2(1 + 2^-|p|)
+// Softplus in base 2 of two values: for p = x log2(e), sp2(p) = log2(1 + 2^p) =
+// log2(1 + e^x), so that ssp(x) = ln2 (sp2(p) - 1).  Written as
+// max(p, 0) + log2(1 + 2^-|p|): no overflow for any p, and 1 + 2^-|p| lies in [1, 2].
 __device__ __forceinline__ float2 sp2x2(float2 p)
 {
     const float2 y = add2(dup2(1.0f), make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y))));
@@ -146,14 +125,6 @@ __device__ __forceinline__ float2 sp2x2_fma(float2 p)
     return add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
 }
 
-// ssp(x) and ssp'(x) sharing one exponential
-__device__ __forceinline__ void ssp_and_grad(float x, float& s, float& g)
-{
-    float t = __expf(-fabsf(x));
-    float r = __fdividef(1.0f, 1.0f + t);
-    s = fmaxf(x, 0.0f) + __logf(1.0f + t) - LN2F;
-    g = x >= 0.0f ? r : t * r;
-}
 
 // ---------------------------------------------------------------------------
 // minimum image (single precision, used for distances in the filters)
@@ -249,17 +220,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (f16 or bf16 inputs, f32 accumulate)
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
 // Arrive on an mbarrier once all previously issued tcgen05 ops of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar)
@@ -325,29 +285,6 @@ __host__ __device__ constexpr uint32_t mnmajor_off(int mn, int k, int MN)
     return (uint32_t)((k >> 3) * (MN * 16) + (mn >> 3) * 128 + (k & 7) * 16 + (mn & 7) * 2);
 }
 
-// 16-bit hi/lo split of an fp32 value (hi = RN(x), lo = RN(x - hi)).
-template <int FMT>
-struct Split;
-template <>
-struct Split<0> {
-    __device__ __forceinline__ static void run(float x, uint16_t& hi, uint16_t& lo)
-    {
-        __half h = __float2half_rn(x);
-        __half l = __float2half_rn(x - __half2float(h));
-        hi = __half_as_ushort(h);
-        lo = __half_as_ushort(l);
-    }
-};
-template <>
-struct Split<1> {
-    __device__ __forceinline__ static void run(float x, uint16_t& hi, uint16_t& lo)
-    {
-        __nv_bfloat16 h = __float2bfloat16_rn(x);
-        __nv_bfloat16 l = __float2bfloat16_rn(x - __bfloat162float(h));
-        hi = __bfloat16_as_ushort(h);
-        lo = __bfloat16_as_ushort(l);
-    }
-};
 
 // ---------------------------------------------------------------------------
 // tcgen05 helpers shared by the tensor-core kernels

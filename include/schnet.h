@@ -190,7 +190,7 @@ typedef struct {
  * The list is rebuilt at the start of every interval of n_rebuild steps.
  * d_pos, d_vel: device float32 [N][3] updated in place (A, A/fs);
  * d_types int32 [N]; d_mass float32 [N] (amu); d_epot, d_ekin: device float64
- * [R] for the last step (may be NULL).  Blocks at the end to read the
+ * [R] for the last step (may be NULL; the sums are formed at the last step only).  Blocks at the end to read the
  * status word once: returns SKIN/CAPACITY/NONFINITE/BADTYPE/TIMEOUT if the
  * corresponding flag was raised during the call (flags then cleared).
  * Errors: INVALID_ARG, CUDA, or a flag status as above. */

@@ -388,7 +388,10 @@ cudaError_t read_and_clear_flags(schnet_ctx* c, unsigned int* flags)
     return e;
 }
 
-// k MD steps, optionally preceded by a neighbour build at the current positions
+// k MD steps, optionally preceded by a neighbour build at the current positions.
+// The per-replica potential and kinetic energies are summed at the last of the k
+// steps only: they are returned for the last step of a call, and a call's steps
+// end at the end of an enqueued block.
 cudaError_t enqueue_steps(schnet_ctx* c, int k, bool build_first, float* pos, float* vel, const int32_t* types,
                           const float* mass, const schnet_step_params* p, double* epot, double* ekin)
 {
@@ -404,10 +407,11 @@ cudaError_t enqueue_steps(schnet_ctx* c, int k, bool build_first, float* pos, fl
                                  p->d_noise, true)) != cudaSuccess)
                 return e;
         }
-        if ((e = launch_energy_forces(c, types, epot, nullptr, true)) != cudaSuccess) return e;
+        const bool last = s == k - 1;
+        if ((e = launch_energy_forces(c, types, epot, nullptr, true, last)) != cudaSuccess) return e;
         {
             Timed t(c, SCHNET_KERNEL_INTEGRATE);
-            if ((e = launch_b_kick(c, vel, mass, p->dt_fs, ekin)) != cudaSuccess) return e;
+            if ((e = launch_b_kick(c, vel, mass, p->dt_fs, ekin, last)) != cudaSuccess) return e;
         }
     }
     return cudaSuccess;
@@ -494,9 +498,10 @@ schnet_status step_impl(schnet_ctx* c, float* pos, float* vel, const int32_t* ty
 // ============================================================================
 // energy / forces orchestration
 // ============================================================================
-// need_forces = false: energies only (no backward, internal forces left as they were)
+// need_forces = false: energies only (no backward, internal forces left as they were);
+// sum_energy = false: per-atom energies only, no per-replica sums
 cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, double* energy, float* forces,
-                                         bool need_forces)
+                                         bool need_forces, bool sum_energy)
 {
     cudaError_t e;
 #define SCHNET_TIMED(kind, expr)                        \
@@ -510,7 +515,8 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
         SCHNET_TIMED(SCHNET_KERNEL_CFCONV_FWD, launch_cfconv_fwd(c, l));
         SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_fwd(c, l));
     }
-    SCHNET_TIMED(SCHNET_KERNEL_REDUCE, launch_replica_sum(c, c->ws.eps, energy ? energy : c->ws.epot));
+    if (sum_energy)
+        SCHNET_TIMED(SCHNET_KERNEL_REDUCE, launch_replica_sum(c, c->ws.eps, energy ? energy : c->ws.epot));
     if (!need_forces) return cudaSuccess;
     SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd_top(c));
     for (int l = c->L - 1; l >= 0; --l) {

@@ -192,13 +192,13 @@ __global__ void k_b_kick(int n, float* __restrict__ vel, const float* __restrict
 
 cudaError_t launch_replica_sum(schnet_ctx* c, const float* v, double* out);
 
-cudaError_t launch_b_kick(schnet_ctx* c, float* d_vel, const float* d_mass, float dt, double* d_ekin)
+cudaError_t launch_b_kick(schnet_ctx* c, float* d_vel, const float* d_mass, float dt, double* d_ekin, bool sum_ke)
 {
     Workspace& w = c->ws;
     k_b_kick<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, d_vel, d_mass, w.frc4, dt, w.ke, w.meta);
     c->launches += 1;
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || !sum_ke) return e;
     return launch_replica_sum(c, w.ke, d_ekin ? d_ekin : w.ekin);
 }
 

@@ -134,10 +134,11 @@ cudaError_t launch_caller_order_list(schnet_ctx* c, const int32_t** row_ptr, con
 cudaError_t launch_scatter_atoms(schnet_ctx* c, const float* v, float* out);
 cudaError_t launch_test_timeout(schnet_ctx* c, uint32_t max_polls, int complete);
 cudaError_t launch_energy_forces(schnet_ctx* c, const int32_t* d_types, double* d_energy, float* d_forces,
-                                 bool need_forces);
+                                 bool need_forces, bool sum_energy = true);
 cudaError_t launch_baoa(schnet_ctx* c, float* d_pos, float* d_vel, const float* d_mass, float dt, float gamma,
                         float temp, unsigned long long seed, const float* d_noise, bool check_skin);
-cudaError_t launch_b_kick(schnet_ctx* c, float* d_vel, const float* d_mass, float dt, double* d_ekin);
+cudaError_t launch_b_kick(schnet_ctx* c, float* d_vel, const float* d_mass, float dt, double* d_ekin,
+                          bool sum_ke = true);
 cudaError_t launch_set_step(schnet_ctx* c, unsigned long long step);
 cudaError_t launch_forces(schnet_ctx* c, float* d_forces);
 cudaError_t launch_replica_sum(schnet_ctx* c, const float* v, double* out);

@@ -190,9 +190,10 @@ typedef struct {
  * The list is rebuilt at the start of every interval of n_rebuild steps.
  * d_pos, d_vel: device float32 [N][3] updated in place (A, A/fs);
  * d_types int32 [N]; d_mass float32 [N] (amu); d_epot, d_ekin: device float64
- * [R] for the last step (may be NULL; the sums are formed at the last step only).  Blocks at the end to read the
- * status word once: returns SKIN/CAPACITY/NONFINITE/BADTYPE/TIMEOUT if the
- * corresponding flag was raised during the call (flags then cleared).
+ * [R] for the last step (may be NULL; the sums are formed at the last step
+ * only).  Blocks at the end to read the status word once: returns
+ * SKIN/CAPACITY/NONFINITE/BADTYPE/TIMEOUT if the corresponding flag was raised
+ * during the call (flags then cleared).
  * Errors: INVALID_ARG, CUDA, or a flag status as above. */
 SCHNET_API schnet_status schnet_step(schnet_ctx *ctx, float *d_pos, float *d_vel, const int32_t *d_types,
                           const float *d_mass, int64_t n_steps, const schnet_step_params *p,

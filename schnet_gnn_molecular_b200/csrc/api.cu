@@ -135,6 +135,7 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.s1 = cv.take<float>(L * FP); w.s2 = cv.take<float>(L * FP);
     w.b1 = cv.take<float>(L * FP); w.b2s = cv.take<float>(L * FP);
     w.emb = cv.take<float>((size_t)d.T * FP);
+    w.emb_h0 = cv.take<float>((size_t)d.T * FP);
     w.aw_img = cv.take<uint8_t>((size_t)(6 * L + 2) * AW_IMG);
     w.aw_sc = cv.take<float>((size_t)(6 * L + 2) * FP);
     w.bo1 = cv.take<float>(L * FP); w.bo2 = cv.take<float>(L * FP);
@@ -296,6 +297,14 @@ void build_weight_blob(const schnet_ctx* c, const schnet_weights* wt, uint8_t* w
     pack_aw(wt->R1, F, Hh, true, H(w.aw_img) + (size_t)(6 * L) * AW_IMG, H(w.aw_sc) + (size_t)(6 * L) * FP);
     pack_aw(wt->R1, F, Hh, false, H(w.aw_img) + (size_t)(6 * L + 1) * AW_IMG, H(w.aw_sc) + (size_t)(6 * L + 1) * FP);
     pad_mat(wt->emb, c->T, F, H(w.emb), c->T, FP, false);
+    // x0 = emb[z] has one row per type, so h0 = x0 W_in of interaction 0 does too (float64 sums)
+    for (int t = 0; t < c->T; ++t)
+        for (int f = 0; f < FP; ++f) {
+            double acc = 0.0;
+            if (f < F)
+                for (int k = 0; k < F; ++k) acc += (double)wt->emb[(size_t)t * F + k] * (double)wt->W_in[(size_t)k * F + f];
+            H(w.emb_h0)[(size_t)t * FP + f] = (float)acc;
+        }
     for (int k = 0; k < HP; ++k) {
         H(w.c1)[k] = k < Hh ? wt->c1[k] : 0.f;
         H(w.R2)[k] = k < Hh ? wt->R2[k] : 0.f;
@@ -510,7 +519,7 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
         if ((e = (expr)) != cudaSuccess) return e;      \
     } while (0)
     SCHNET_TIMED(SCHNET_KERNEL_MASK, launch_compact(c));
-    SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_first(c, types));
+    SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_embed(c, types));
     for (int l = 0; l < c->L; ++l) {
         SCHNET_TIMED(SCHNET_KERNEL_CFCONV_FWD, launch_cfconv_fwd(c, l));
         SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_fwd(c, l));

@@ -1,6 +1,6 @@
-// Atom-wise parts of SchNet on the sm_100a tensor cores: embedding, the
-// interaction's in/out dense layers with the residual update, the per-atom
-// readout, their backward pass, and the per-replica sums.
+// Atom-wise parts of SchNet: the embedding (a per-type table gather), and on the
+// sm_100a tensor cores the interaction's in/out dense layers with the residual
+// update, the per-atom readout and their backward pass; the per-replica sums.
 //
 // Model reading (FlashSchNet paper-curation summary, How / Figure 2 caption:
 // positions and embeddings pass through interaction blocks; readout per atom
@@ -32,17 +32,15 @@ constexpr uint32_t AW_POLLS = 1u << 22;
 constexpr uint32_t AW_ACC = 0;                // TMEM columns 0..127: accumulator
 constexpr uint32_t AW_SLOT = 128;             // TMEM columns 128 + 128 s: weight slot s (hi 64, lo 64)
 
-enum { AW_FIRST = 0, AW_FWD = 1, AW_TOP = 2, AW_BWD = 3 };
+enum { AW_FWD = 1, AW_TOP = 2, AW_BWD = 3 };
 
 struct AWArgs {
-    int N, T, ntiles;
+    int N, ntiles;
     int ngemm;                    // dense layers chained in this launch (1..3)
     int last;                     // AW_FWD: readout instead of the next layer's h
-    const int32_t* types;         // caller order
-    const int32_t* perm;          // slot -> caller index
     const uint8_t* img[3];        // the layers' packed A images (hi term, then lo term)
     const float* sc[3];           // their per-row scales [FP]
-    const float *emb, *bo1, *bo2, *c1, *R2, *c2;
+    const float *bo1, *bo2, *c1, *R2, *c2;
     float *x, *h_out, *q, *m, *g, *dh, *pr, *eps;
     const float* q_in;            // backward: q of the layer whose u is formed
     DevMeta* meta;
@@ -160,22 +158,7 @@ __global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
         auto row_ok = [&](int q) { return i0 + q < a.N; };
         auto at = [&](int q, int w) { return (size_t)(i0 + q) * w + f; };
         // ---- input of the first layer
-        if (MODE == AW_FIRST) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                float xv = 0.f;
-                if (row_ok(q)) {
-                    int z = __ldg(a.types + __ldg(a.perm + i0 + q));
-                    if (z < 0 || z >= a.T) {
-                        if (f == 0) set_flag(a.meta, SCHNET_FLAG_BADTYPE);
-                        z = 0;
-                    }
-                    xv = __ldg(a.emb + (size_t)z * FP + f);
-                    a.x[at(q, FP)] = xv;
-                }
-                v[q] = xv;
-            }
-        } else if (MODE == AW_FWD) {
+        if (MODE == AW_FWD) {
 #pragma unroll
             for (int q = 0; q < 32; ++q) v[q] = row_ok(q) ? __ldg(a.m + at(q, FP)) : 0.f;
         } else if (MODE == AW_TOP) {
@@ -191,12 +174,6 @@ __global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
         stage_b(B, v, s, c, f);
         if (!(ok = aw_gemm(tmem, 0, sB, bar, phase, a.meta, tD, d))) break;
         const float k0 = sc[0] * inv;
-        if (MODE == AW_FIRST) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-                if (row_ok(q)) a.h_out[at(q, FP)] = d[q] * k0;
-            continue;
-        }
         if (MODE == AW_FWD) {
             // q = m Wo1 + bo1 ; a = ssp(q)
             const float b = __ldg(a.bo1 + f);
@@ -326,25 +303,19 @@ __global__ void k_replica_sums(int R, const int32_t* __restrict__ chunk_rep, int
 // images and scales of the atom-wise layers: per layer l, matrix id 6 l + j with
 // j = 0 Wo1^T, 1 Wo2^T, 2 W_in^T (forward), 3 W_in, 4 Wo2, 5 Wo1 (backward);
 // then 6 L = R1^T (readout), 6 L + 1 = R1 (readout backward)
-static AWArgs aw_args(schnet_ctx* c, const int32_t* types, int mode, int layer)
+static AWArgs aw_args(schnet_ctx* c, int mode, int layer)
 {
     Workspace& w = c->ws;
     const int L = c->L;
     AWArgs a{};
     a.N = c->N;
-    a.T = c->T;
     a.ntiles = (c->N + ATILE - 1) / ATILE;
-    a.types = types;
-    a.perm = w.perm;
-    a.emb = w.emb; a.bo1 = w.bo1 + layer * FP; a.bo2 = w.bo2 + layer * FP;
+    a.bo1 = w.bo1 + layer * FP; a.bo2 = w.bo2 + layer * FP;
     a.c1 = w.c1; a.R2 = w.R2; a.c2 = w.c2;
     a.x = w.x; a.q = w.q + (size_t)layer * c->N * FP; a.m = w.m; a.g = w.g; a.dh = w.dh; a.pr = w.pr;
     a.eps = w.eps; a.meta = w.meta;
     int ids[3] = {0, 0, 0};
-    if (mode == AW_FIRST) {
-        a.ngemm = 1; ids[0] = 2;
-        a.h_out = w.h;
-    } else if (mode == AW_FWD) {
+    if (mode == AW_FWD) {
         a.ngemm = 3; ids[0] = 6 * layer; ids[1] = 6 * layer + 1;
         a.last = layer + 1 == L;
         ids[2] = a.last ? 6 * L : 6 * (layer + 1) + 2;
@@ -370,8 +341,6 @@ static AWArgs aw_args(schnet_ctx* c, const int32_t* types, int mode, int layer)
 cudaError_t atomwise_init_attributes()
 {
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(k_atomwise<AW_FIRST>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM)))
-        return e;
     if ((e = cudaFuncSetAttribute(k_atomwise<AW_FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM)))
         return e;
     if ((e = cudaFuncSetAttribute(k_atomwise<AW_TOP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AW_SMEM)))
@@ -381,30 +350,54 @@ cudaError_t atomwise_init_attributes()
 
 static int aw_grid(schnet_ctx* c) { return std::min((c->N + ATILE - 1) / ATILE, c->nsm); }
 
-cudaError_t launch_aw_first(schnet_ctx* c, const int32_t* types)
+// Embedding and the first h: one warp per slot, four features per lane.  x0 = emb[z]
+// and h0 = (emb W_in)[z] are rows of per-type tables (the second formed on the host
+// in float64), so no GEMM is needed for interaction 0's input.
+__global__ void k_embed(int n, int T, const int32_t* __restrict__ types, const int32_t* __restrict__ perm,
+                        const float4* __restrict__ emb, const float4* __restrict__ emb_h0, float4* __restrict__ x,
+                        float4* __restrict__ h, DevMeta* meta)
 {
-    k_atomwise<AW_FIRST><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, types, AW_FIRST, 0));
+    const int k = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (k >= n) return;
+    int z = __ldg(types + __ldg(perm + k));
+    if (z < 0 || z >= T) {
+        if (lane == 0) set_flag(meta, SCHNET_FLAG_BADTYPE);
+        z = 0;
+    }
+    x[(size_t)k * (FP / 4) + lane] = __ldg(emb + (size_t)z * (FP / 4) + lane);
+    h[(size_t)k * (FP / 4) + lane] = __ldg(emb_h0 + (size_t)z * (FP / 4) + lane);
+}
+
+cudaError_t launch_embed(schnet_ctx* c, const int32_t* types)
+{
+    Workspace& w = c->ws;
+    static_assert(FP == 128, "one float4 per lane covers a padded feature row");
+    const long long threads = (long long)c->N * 32;
+    k_embed<<<(unsigned)((threads + 255) / 256), 256, 0, c->s>>>(
+        c->N, c->T, types, w.perm, reinterpret_cast<const float4*>(w.emb), reinterpret_cast<const float4*>(w.emb_h0),
+        reinterpret_cast<float4*>(w.x), reinterpret_cast<float4*>(w.h), w.meta);
     c->launches += 1;
     return cudaGetLastError();
 }
 
 cudaError_t launch_aw_fwd(schnet_ctx* c, int layer)
 {
-    k_atomwise<AW_FWD><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, nullptr, AW_FWD, layer));
+    k_atomwise<AW_FWD><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, AW_FWD, layer));
     c->launches += 1;
     return cudaGetLastError();
 }
 
 cudaError_t launch_aw_bwd_top(schnet_ctx* c)
 {
-    k_atomwise<AW_TOP><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, nullptr, AW_TOP, c->L - 1));
+    k_atomwise<AW_TOP><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, AW_TOP, c->L - 1));
     c->launches += 1;
     return cudaGetLastError();
 }
 
 cudaError_t launch_aw_bwd(schnet_ctx* c, int layer)
 {
-    k_atomwise<AW_BWD><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, nullptr, AW_BWD, layer));
+    k_atomwise<AW_BWD><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, AW_BWD, layer));
     c->launches += 1;
     return cudaGetLastError();
 }

@@ -35,6 +35,7 @@ struct Workspace {
     float *s1, *s2, *b1;          // [L][FP] filter channel scales, first-layer bias
     float* b2s;                   // [L][FP] second-layer bias minus ln2 s2 sum_k W2^[k][f] (base-2 softplus shift)
     float *emb;                   // [T][FP]
+    float *emb_h0;                // [T][FP] emb W_in of interaction 0 (the first h of every atom of a type)
     uint8_t* aw_img;              // [6 L + 2][AW_IMG] atom-wise layers as tensor-core A operands
     float* aw_sc;                 // [6 L + 2][FP] their per-row scales
     float *bo1, *bo2;             // [L][FP]
@@ -142,7 +143,7 @@ cudaError_t launch_b_kick(schnet_ctx* c, float* d_vel, const float* d_mass, floa
 cudaError_t launch_set_step(schnet_ctx* c, unsigned long long step);
 cudaError_t launch_forces(schnet_ctx* c, float* d_forces);
 cudaError_t launch_replica_sum(schnet_ctx* c, const float* v, double* out);
-cudaError_t launch_aw_first(schnet_ctx* c, const int32_t* types);
+cudaError_t launch_embed(schnet_ctx* c, const int32_t* types);
 cudaError_t launch_aw_fwd(schnet_ctx* c, int layer);
 cudaError_t launch_aw_bwd_top(schnet_ctx* c);
 cudaError_t launch_aw_bwd(schnet_ctx* c, int layer);

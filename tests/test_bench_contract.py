@@ -31,3 +31,22 @@ def test_reference_arm_json_line():
                         "d2h_bytes_per_step": 0}
     import bench
     assert d["metric"] == bench.METRIC
+
+
+def test_traffic_figure_is_keyed_to_the_kernel_sources(tmp_path, monkeypatch):
+    """The DRAM traffic in the roofline object is reported only while the kernel
+    sources hash to the value recorded beside the capture; an edit voids it."""
+    import shutil
+    import bench
+    d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    assert bench._traffic("cfconv_bwd") == d["cfconv_bwd"]
+    for src in d["sources"]:
+        os.makedirs(tmp_path / os.path.dirname(src), exist_ok=True)
+        shutil.copy(os.path.join(ROOT, src), tmp_path / src)
+    os.makedirs(tmp_path / "profiles")
+    shutil.copy(os.path.join(ROOT, "profiles", "traffic.json"), tmp_path / "profiles" / "traffic.json")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._traffic("cfconv_bwd") == d["cfconv_bwd"]
+    with open(tmp_path / d["sources"][0], "a") as f:
+        f.write("\n// edited\n")
+    assert bench._traffic("cfconv_bwd") is None

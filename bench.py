@@ -62,24 +62,32 @@ class ClockSampler:
         except Exception:
             self.p = None
 
-    def stop(self, t0=None, t1=None):
+    def stop(self):
+        """End sampling and keep the samples (summarise windows with ``window``)."""
+        self.rows = []
         if self.p is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return self
         self.p.terminate()
         self.p.wait(timeout=10)
         self.f.flush()
         self.f.seek(0)
-        rows = []
         for line in self.f.read().splitlines():
             t = [x.strip() for x in line.split(",")]
             if len(t) < 9:
                 continue
             try:
                 ts = datetime.datetime.strptime(t[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                rows.append((ts, float(t[1]), float(t[2]), t[5:9]))
+                self.rows.append((ts, float(t[1]), float(t[2]), t[5:9]))
             except ValueError:
                 continue
         os.unlink(self.f.name)
+        return self
+
+    def window(self, t0=None, t1=None):
+        """Median SM clock, max clock and active throttle reasons of the samples in [t0, t1]."""
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = self.rows
         inside = [r for r in rows if t0 is None or (t0 <= r[0] <= t1)]
         window = "timed region"
         if not inside:                       # region shorter than the sampling period
@@ -91,6 +99,41 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(r[2] for r in inside) if inside else None,
                 "reasons": sorted(reasons), "samples": len(inside), "window": window}
+
+
+def tensor_peak(peaks, clk):
+    """Dense fp16/bf16 tensor peak for kernels timed under the clocks `clk`: the burst
+    figure when the SM clock held its maximum with no power cap, else the sustained one."""
+    burst = peaks.get("bf16_tflops")
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    full = (clk and clk.get("sm_mhz") and clk.get("sm_max_mhz") and clk["sm_mhz"] >= 0.97 * clk["sm_max_mhz"]
+            and "sw_power_cap" not in clk.get("reasons", []))
+    return (burst, "burst") if full else (sustained, "sustained")
+
+
+# MUFU (special-function unit) operations per edge and interaction, counted from the kernel
+# source: forward -- one ex2 per evaluated Gaussian (K), and per feature one ex2 and one lg2
+# for the base-2 softplus, except that one feature pair in four takes its ex2 on the FMA pipe;
+# backward -- K Gaussian ex2, per feature ex2 + lg2 (the logistic's reciprocal runs on the FMA
+# pipe).  148 SMs x 16 MUFU results per clock.
+def mufu_per_edge(K, F):
+    return {"fwd": K + 2 * F - F // 4, "bwd": K + 2 * F}
+
+
+def hbm_kernel_bytes(w, E_list, E_cut):
+    """Algorithmic HBM bytes of the memory-bound kernels (per launch; the neighbour build per
+    build).  forces: per listed edge col, rev and s_e (4 B each), per atom the position (16 B),
+    row pointer and slot map (8 B) and the force (16 B).  integrate: per atom and step, B-A-O-A
+    reads slot map, mass, force, velocity, position, build reference (4+4+16+12+12+16 B) and
+    writes velocity, position, slot-order position (12+12+16 B); the closing B reads mass, force,
+    velocity (4+16+12 B) and writes velocity and kinetic energy (12+4 B).  mask: per listed edge
+    its row and column (8 B), per edge inside the cutoff row, column, index (12 B).  neighbours:
+    positions in (12 B per atom), col and rev out (8 B per listed edge), row pointers (4 B per atom)."""
+    N = w.n_atoms
+    return {"forces": 12 * E_list + 40 * N,
+            "integrate": (104 + 48) * N,
+            "mask": 8 * E_list + 12 * E_cut,
+            "neighbors": 12 * N + 8 * E_list + 4 * N}
 
 
 def _dist():
@@ -271,7 +314,6 @@ def run_native(args):
               "torch_peak_allocated_MB": round(torch.cuda.max_memory_allocated(dev) / 1e6, 1),
               "device_used_MB": round((total_b - free_b) / 1e6, 1),
               "note": "device_used includes the CUDA context, the library image and the captured graphs"}
-    clk = clocks.stop(wall0, wall1) if clocks else None
     t_max, atoms_total, value = aggregate_ranks(ms, w.n_atoms, steps, dist, dev)
     step_s = t_max * 1e-3 / steps
     ns_day_rep = (1.0 / step_s) * w.dt_fs * 86400 * 1e-6
@@ -279,19 +321,48 @@ def run_native(args):
     out = None
     if rank == 0:
         # per-kernel device times on the library stream (eager profiling pass, same trajectory)
+        prof_t0 = time.time()
         prof = model.profile_steps(p, v, t, m, n_rb, step0=args.warmup + steps, **kw)
+        prof_t1 = time.time()
+        clocks.stop()
+        clk = clocks.window(wall0, wall1)
+        clk_prof = clocks.window(prof_t0, prof_t1)
         E_list, E_cut = _edge_stats(model, p.cpu().numpy(), w)
         peaks, src = _peaks()
         flop_fwd = 2.0 * (w.K * w.F + w.F * w.F) * E_cut
         flop_bwd = 2.0 * flop_fwd
-        fwd_ms = prof["cfconv_fwd"][0] / max(prof["cfconv_fwd"][1], 1)
-        bwd_ms = prof["cfconv_bwd"][0] / max(prof["cfconv_bwd"][1], 1)
+        per_launch = {k: x[0] / max(x[1], 1) for k, x in prof.items()}
+        per_step = {k: x[0] / n_rb for k, x in prof.items()}
         tot_ms = sum(x[0] for x in prof.values())
         dominant = "cfconv_bwd" if prof["cfconv_bwd"][0] >= prof["cfconv_fwd"][0] else "cfconv_fwd"
-        flops, kms = (flop_bwd, bwd_ms) if dominant == "cfconv_bwd" else (flop_fwd, fwd_ms)
-        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        flops, kms = (flop_bwd, per_launch["cfconv_bwd"]) if dominant == "cfconv_bwd" else \
+            (flop_fwd, per_launch["cfconv_fwd"])
+        peak, peak_kind = tensor_peak(peaks, clk_prof)
         achieved = flops / (kms * 1e-3) / 1e12
         traffic = _traffic(dominant)
+        # end-to-end roofline: per kernel class the slowest of its tensor, MUFU and HBM bounds
+        hbm = peaks["hbm_gbs"] * 1e9
+        f_clk = (clk_prof.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)) * 1e6
+        mufu_peak = 148 * 16 * f_clk
+        mu = mufu_per_edge(w.K, w.F)
+        hb = hbm_kernel_bytes(w, E_list, E_cut)
+        n_aw = 6 * w.L                                    # atom-wise layer applications per step
+        bounds = {
+            "cfconv_fwd": max(w.L * flop_fwd / (peak * 1e12), w.L * mu["fwd"] * E_cut / mufu_peak),
+            "cfconv_bwd": max(w.L * flop_bwd / (peak * 1e12), w.L * mu["bwd"] * E_cut / mufu_peak),
+            "atomwise": max(n_aw * 2.0 * w.F * w.F * w.n_atoms / (peak * 1e12),
+                            n_aw * 2 * w.n_atoms * w.F * 4 / hbm),
+            "forces": hb["forces"] / hbm, "integrate": hb["integrate"] / hbm, "mask": hb["mask"] / hbm,
+            "neighbors": hb["neighbors"] / hbm / n_rb, "reduce": 8 * w.n_atoms / hbm}
+        bound_ms = {k: v * 1e3 for k, v in bounds.items()}
+        e2e_frac = sum(bound_ms.values()) / (step_s * 1e3)
+        hbm_kernels = {}
+        for k in ("forces", "integrate", "mask", "neighbors"):
+            ms_k = per_launch[k] if k == "neighbors" else per_step[k]
+            gbs = hb[k] / (ms_k * 1e-3) / 1e9 if ms_k > 0 else None
+            hbm_kernels[k] = {"bytes": int(hb[k]), "per": "build" if k == "neighbors" else "step",
+                              "ms": round(ms_k, 5), "achieved_GBs": round(gbs, 1) if gbs else None,
+                              "frac": round(gbs / peaks["hbm_gbs"], 4) if gbs else None}
         k_interval = max(1, int(round(launches / steps * n_rb)))
         floor = {"ms_per_step": round(_launch_floor(dev, k_interval) / n_rb, 4),
                  "kernels_per_step": round(launches / steps, 2),
@@ -299,10 +370,17 @@ def run_native(args):
                         f"replayed; per step = replay time / {n_rb}"}
         roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 2),
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                    "peak_source": f"{src} dense bf16/fp16 sustained",
+                    "peak_source": f"{src} dense bf16/fp16 {peak_kind} (per-kernel times taken at "
+                                   f"{clk_prof.get('sm_mhz')} MHz, reasons {clk_prof.get('reasons')})",
                     "flop_per_launch": flops, "ms_per_launch": round(kms, 4),
-                    "per_kernel_ms_per_step": {k: round(x[0] / n_rb, 4) for k, x in prof.items()},
-                    "kernel_share": {k: round(x[0] / tot_ms, 4) for k, x in prof.items()}}
+                    "per_kernel_ms_per_step": {k: round(x, 4) for k, x in per_step.items()},
+                    "kernel_share": {k: round(x[0] / tot_ms, 4) for k, x in prof.items()},
+                    "e2e_frac": round(e2e_frac, 4),
+                    "e2e_bound_ms_per_step": {k: round(x, 4) for k, x in bound_ms.items()},
+                    "e2e_how": "sum over kernel classes of max(tensor FLOP / tensor peak, MUFU ops / MUFU peak, "
+                               "algorithmic HBM bytes / HBM peak), divided by the measured ms_per_step",
+                    "mufu_per_edge_interaction": mu, "mufu_peak_per_s": mufu_peak,
+                    "hbm_peak_GBs": peaks["hbm_gbs"], "hbm_kernels": hbm_kernels}
         cfg = dict(_workload_config(w, n_rb, ws))
         cfg.update({"edges_listed": E_list, "edges_within_cutoff": E_cut,
                "edges_within_cutoff_at_start": edges_start[1],
@@ -317,6 +395,7 @@ def run_native(args):
                "ns_per_day_per_replica": round(ns_day_rep, 2),
                "ns_per_day_aggregate": round(ns_day_rep * w.n_replicas * ws, 1),
                "config": cfg, "gpu_launches": int(launches), "launch_floor": floor, "clocks": clk,
+               "clocks_profile_pass": clk_prof,
                "roofline": roofline,
                "memory": memory,
                "status": {"warmup": nat_status(flagged[0]), "timed": nat_status(flagged[1])}}
@@ -369,7 +448,11 @@ def e2e(model, w, pos, vel, types, mass, kw, args):
 def run_drift(args):
     """NVE drift: velocity Verlet (gamma = 0) on the workload for --drift-steps steps;
     total energy (potential + kinetic, summed over replicas) read after every rebuild
-    interval; reported as the least-squares slope per atom."""
+    interval; reported as the least-squares slope per atom, over the whole run and per
+    window of --drift-window steps, with the within-cutoff edge count at every window
+    boundary (the chains have no bonded terms and slowly fly apart, so the graph
+    shrinks; the slope over the leading windows whose graph keeps >= 90 % of its
+    starting edges is the one measured on an intact graph)."""
     import torch
     from schnet_gnn_molecular_b200 import api
     w = _workload(args.workload).with_(gamma_per_ps=0.0)
@@ -381,38 +464,61 @@ def run_drift(args):
     kw = dict(dt=w.dt_fs, gamma=0.0, temperature=w.temperature, n_rebuild=w.n_rebuild, seed=1234)
     chunk = w.n_rebuild
     n_chunks = max(1, args.drift_steps // chunk)
+    win_chunks = max(1, args.drift_window // chunk)
     ep, _, st = model.step(p, v, t, m, 0, step0=0, raise_on_flag=False, **kw)   # initial forces
-    edges0 = _edge_stats(model, pos, w)[1]
+    edges = [(0, _edge_stats(model, pos, w)[1])]
     ek0 = 0.5 * float((mass.astype(np.float64)[:, None] * vel.astype(np.float64) ** 2).sum()) / ACC
     times, etot, flags = [0.0], [float(ep.sum()) + ek0], int(st)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record()
+    ms = 0.0
     for c in range(n_chunks):
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
         ep, ek, st = model.step(p, v, t, m, chunk, step0=c * chunk, resume=c > 0, raise_on_flag=False, **kw)
+        ev1.record()
+        torch.cuda.synchronize()
+        ms += ev0.elapsed_time(ev1)
         flags |= int(st)
         times.append((c + 1) * chunk * w.dt_fs * 1e-6)          # ns
         etot.append(float((ep + ek).sum()))
-    ev1.record()
-    torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    model.build_neighbors(p)
-    edges1 = _edge_stats(model, p.cpu().numpy(), w)[1]
+        if (c + 1) % win_chunks == 0 or c == n_chunks - 1:
+            # the list of the last rebuild covers every pair within the cutoff at these positions
+            edges.append(((c + 1) * chunk, _edge_stats(model, p.cpu().numpy(), w)[1]))
     tt, ee = np.array(times), np.array(etot) / w.n_atoms
-    slope, icpt = np.polyfit(tt, ee, 1)
-    resid = ee - (slope * tt + icpt)
     kcal_to_uev = 4.3364e4                   # 1 kcal/mol = 43.364 meV
+
+    def fit(a, b):
+        sl, ic = np.polyfit(tt[a:b + 1], ee[a:b + 1], 1)
+        res = ee[a:b + 1] - (sl * tt[a:b + 1] + ic)
+        return float(sl), float(np.sqrt((res ** 2).mean()))
+
+    slope, rms = fit(0, len(tt) - 1)
+    windows, intact_end = [], 0
+    for (s0, e0), (s1, e1) in zip(edges[:-1], edges[1:]):
+        sl, _ = fit(s0 // chunk, s1 // chunk)
+        windows.append({"steps": [s0, s1], "slope_kcal_mol_atom_ns": sl, "slope_ueV_atom_ps": sl * kcal_to_uev / 1e3,
+                        "edges_within_cutoff": [e0, e1]})
+        if intact_end == s0 and min(e0, e1) >= 0.9 * edges[0][1]:
+            intact_end = s1
+    intact = None
+    if intact_end > 0:
+        sl, r = fit(0, intact_end // chunk)
+        intact = {"steps": [0, intact_end], "slope_kcal_mol_atom_ns": sl, "slope_ueV_atom_ps": sl * kcal_to_uev / 1e3,
+                  "rms_about_fit_kcal_mol_atom": r,
+                  "edges_within_cutoff_min": int(min(e for s_, e in edges if s_ <= intact_end))}
     ekin0 = float(ek.sum()) / w.n_atoms
-    out = {"metric": "NVE energy drift (velocity Verlet)", "value": float(slope), "unit": "kcal/mol/atom/ns",
-           "ueV_per_atom_per_ps": float(slope) * kcal_to_uev / 1e3, "steps": n_chunks * chunk,
+    out = {"metric": "NVE energy drift (velocity Verlet)", "value": slope, "unit": "kcal/mol/atom/ns",
+           "ueV_per_atom_per_ps": slope * kcal_to_uev / 1e3, "steps": n_chunks * chunk,
            "dt_fs": w.dt_fs, "simulated_ns": float(tt[-1]), "higher_is_better": False,
            "etot_per_atom_first_last": [float(ee[0]), float(ee[-1])],
-           "etot_per_atom_rms_about_fit": float(np.sqrt((resid ** 2).mean())),
-           "ekin_per_atom_last": ekin0, "status": nat_status(flags),
+           "etot_per_atom_rms_about_fit": rms, "ekin_per_atom_last": ekin0, "status": nat_status(flags),
            "ms_per_step": round(ms / (n_chunks * chunk), 4),
-           "edges_within_cutoff_first_last": [edges0, edges1],
-           "note": "no bonded terms: the chains expand during the run, so the graph shrinks",
+           "intact_graph": intact, "windows": windows,
+           "edges_within_cutoff_first_last": [edges[0][1], edges[-1][1]],
+           "note": "no bonded terms: the chains expand during the run, so the graph shrinks; 'intact_graph' is "
+                   "the fit over the leading windows that keep >= 90 % of the starting edges",
            "config": {"workload": w.name, "replicas": w.n_replicas, "atoms": w.n_atoms, "n_rebuild": w.n_rebuild,
-                      "skin_A": w.skin, "read_every_steps": chunk}, "data": "synthetic"}
+                      "skin_A": w.skin, "read_every_steps": chunk, "window_steps": win_chunks * chunk},
+           "data": "synthetic"}
     model.close()
     print(json.dumps(out), flush=True)
 
@@ -520,6 +626,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--nve-drift", action="store_true", help="measure NVE energy drift instead of throughput")
     ap.add_argument("--drift-steps", type=int, default=10000)
+    ap.add_argument("--drift-window", type=int, default=500)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -277,12 +277,19 @@ SCHNET_API schnet_status schnet_profile_steps(schnet_ctx *ctx, float *d_pos, flo
  *   [n_replicas+1] (0 .. n_atoms, non-decreasing); box: host float[3]
  *   (periodic only).  Outputs (caller-owned device buffers): d_row_ptr int32
  *   [n_atoms+1], d_col and d_rev int32 [edge_capacity], d_n_edges int64 [1]
- *   = edges found; if that exceeds edge_capacity, col and rev are left
- *   unspecified and the caller should retry with more room.
+ *   = edges found; if that exceeds edge_capacity, col and rev are not
+ *   written and the caller should retry with more room.  d_flags (device
+ *   uint32 [1], may be NULL) receives the SCHNET_FLAG_* bits of this call:
+ *   SCHNET_FLAG_NONFINITE when a position is NaN or infinite (the list is then
+ *   built with those atoms binned into an arbitrary cell, so it may miss
+ *   pairs and should not be used), SCHNET_FLAG_CAPACITY when the list did not
+ *   fit.  Both outputs are written on the stream; read them after it syncs.
  * Limits: n_atoms <= 65536, n_replicas <= 1024, cells <= 131072 (open
  * boundaries use 512 cells per replica, so n_replicas <= 256 there),
  * edge_capacity < 2^31; larger inputs return SCHNET_ERR_UNSUPPORTED, bad
  * pointers or sizes SCHNET_ERR_INVALID_ARG.  Asynchronous on cuda_stream.
+ * A CUDA error already pending on the calling thread when the call starts is
+ * left in place and reported as SCHNET_ERR_CUDA before anything is enqueued.
  * The first call on each device looks up the array's device address (with
  * that device current); make that first call before any stream capture.
  * Every call reuses the same array and zeroes what must start at zero, so
@@ -292,7 +299,7 @@ SCHNET_API schnet_status schnet_build_neighbors_noalloc(const float *d_pos, int3
                                                         const int32_t *d_replica_offsets, float cutoff, float skin,
                                                         int32_t periodic, const float *box, int32_t *d_row_ptr,
                                                         int32_t *d_col, int32_t *d_rev, int64_t edge_capacity,
-                                                        int64_t *d_n_edges, void *cuda_stream);
+                                                        int64_t *d_n_edges, uint32_t *d_flags, void *cuda_stream);
 
 /* Number of device kernels the library has launched on this context so far
  * (graph replays count each kernel node). */

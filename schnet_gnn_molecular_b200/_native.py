@@ -77,7 +77,7 @@ def load() -> C.CDLL:
     L.schnet_test_timeout.argtypes = [vp, C.c_uint32, C.c_int32]
     L.schnet_profile_steps.argtypes = [vp, vp, vp, vp, vp, C.c_int64, C.POINTER(StepParams), dp, i64p]
     L.schnet_build_neighbors_noalloc.argtypes = [vp, C.c_int32, C.c_int32, vp, C.c_float, C.c_float, C.c_int32,
-                                                 C.POINTER(C.c_float), vp, vp, vp, C.c_int64, vp, vp]
+                                                 C.POINTER(C.c_float), vp, vp, vp, C.c_int64, vp, vp, vp]
     L.schnet_kernel_launches.argtypes = [vp]
     L.schnet_kernel_launches.restype = C.c_int64
     for name in EXPORTED:

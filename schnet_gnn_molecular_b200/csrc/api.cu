@@ -95,8 +95,7 @@ Derived derive(const schnet_config* c)
     if (c->periodic) {
         long long cells = 1;
         for (int k = 0; k < 3; ++k) {
-            int g = (int)std::floor((double)c->box[k] / d.rl);
-            g = std::max(1, std::min(g, GMAX_PERIODIC));
+            const int g = cells_across((double)c->box[k], d.rl, GMAX_PERIODIC);
             d.gdim[k] = g;
             cells *= g;
         }
@@ -133,7 +132,7 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     if (wbegin) *wbegin = cv.off;
     w.img = cv.take<uint8_t>(L * LAYER_IMG);
     w.s1 = cv.take<float>(L * FP); w.s2 = cv.take<float>(L * FP);
-    w.b1 = cv.take<float>(L * FP); w.b2s = cv.take<float>(L * FP);
+    w.b1 = cv.take<float>(L * FP); w.b2 = cv.take<float>(L * FP);
     w.emb = cv.take<float>((size_t)d.T * FP);
     w.emb_h0 = cv.take<float>((size_t)d.T * FP);
     w.aw_img = cv.take<uint8_t>((size_t)(6 * L + 2) * AW_IMG);
@@ -158,7 +157,7 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.cell_of = cv.take<int32_t>(N); w.cell_atoms = cv.take<int32_t>(N);
     w.cell_cnt = cv.take<int32_t>((size_t)d.ncell + 1); w.cell_start = cv.take<int32_t>((size_t)d.ncell + 1);
     w.cell_fill = cv.take<int32_t>((size_t)d.ncell + 1);
-    w.rgrid_dims = cv.take<int4>(R); w.rgrid_org = cv.take<float4>(R); w.rgrid_inv = cv.take<float4>(R);
+    w.rgrid_dims = cv.take<int4>(R); w.rgrid_geom = cv.take<GridGeom>(R);
     w.scan_tmp = cv.take<long long>(SCAN_TILE);
     w.x = cv.take<float>(N * FP);
     w.h = cv.take<float>(L * N * FP);
@@ -271,21 +270,11 @@ void build_weight_blob(const schnet_ctx* c, const schnet_weights* wt, uint8_t* w
         uint16_t* w2lo = reinterpret_cast<uint16_t*>(img + 2 * W1_IMG + W2_IMG);
         pack_operand(W1, K, F, KP, s1, fmt, c->n_wterms, w1hi, w1lo);
         pack_operand(W2, F, F, FP, s2, fmt, c->n_wterms, w2hi, w2lo);
-        // The kernels feed the second layer a = log2(1 + e^x) instead of
-        // ssp(x) = ln2 (a - 1): ln2 goes into the scale, and the constant -ln2
-        // times the column sum of the stored weight terms into the bias.
-        std::vector<double> colsum(FP, 0.0);
-        for (int f = 0; f < FP; ++f)
-            for (int k = 0; k < FP; ++k) {
-                const size_t idx = kmajor_off(f, k, FP) / 2;
-                colsum[f] += from16(w2hi[idx], fmt) + (c->n_wterms == 2 ? from16(w2lo[idx], fmt) : 0.0);
-            }
         for (int f = 0; f < FP; ++f) {
             H(w.s1)[l * FP + f] = (float)s1[f];
             H(w.s2)[l * FP + f] = (float)s2[f];
             H(w.b1)[l * FP + f] = f < F ? wt->b1[l * F + f] : 0.f;
-            const double b2 = f < F ? (double)wt->b2[l * F + f] : 0.0;
-            H(w.b2s)[l * FP + f] = (float)(b2 - 0.69314718055994530942 * s2[f] * colsum[f]);
+            H(w.b2)[l * FP + f] = f < F ? wt->b2[l * F + f] : 0.f;
             H(w.bo1)[l * FP + f] = f < F ? wt->bo1[l * F + f] : 0.f;
             H(w.bo2)[l * FP + f] = f < F ? wt->bo2[l * F + f] : 0.f;
         }

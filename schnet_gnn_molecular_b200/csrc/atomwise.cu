@@ -92,12 +92,19 @@ __device__ __forceinline__ bool aw_gemm(uint32_t tmem, int slot, uint32_t sB, ui
         const uint32_t id = idesc_f16(128, ATILE, 0, 1);
         const uint32_t ahi = tmem + AW_SLOT + 128 * slot, alo = ahi + 64;
         const uint64_t bh0 = smem_desc(sB, ATILE * 16, 128), bl0 = smem_desc(sB + AW_BTERM, ATILE * 16, 128);
+        // the two small correction products first, the hi x hi product last: the tensor
+        // core's fp32 accumulation does not round to nearest, so every MMA added to an
+        // accumulator that already holds the large sum costs a little accuracy
 #pragma unroll
         for (int ks = 0; ks < FP / 16; ++ks) {
             const uint64_t step = (uint64_t)((ks * 2 * ATILE * 16) >> 4);   // start-address field only
-            mma_f16_ts(tmem + AW_ACC, ahi + ks * 8, bh0 + step, id, ks > 0 ? 1u : 0u);
-            mma_f16_ts(tmem + AW_ACC, alo + ks * 8, bh0 + step, id, 1u);
+            mma_f16_ts(tmem + AW_ACC, alo + ks * 8, bh0 + step, id, ks > 0 ? 1u : 0u);
             mma_f16_ts(tmem + AW_ACC, ahi + ks * 8, bl0 + step, id, 1u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < FP / 16; ++ks) {
+            const uint64_t step = (uint64_t)((ks * 2 * ATILE * 16) >> 4);
+            mma_f16_ts(tmem + AW_ACC, ahi + ks * 8, bh0 + step, id, 1u);
         }
         mma_commit(bar);
     }

@@ -23,10 +23,11 @@
 // so TMEM lane = output feature and TMEM column = edge.  Each epilogue thread
 // then owns one feature of every edge in the tile, the per-row reduction is a
 // running sum in one register, and the h_j gathers are 128-byte coalesced rows.
-// The weights (A) are re-read from shared memory by every MMA, so every MMA
-// has N = 128 to keep that re-read at half of the shared-memory bandwidth the
-// tensor core draws: the backward kernel stacks each edge's value and
-// derivative operands into one B tile instead of issuing two N = 64 GEMMs.
+// The weights (A) sit in tensor memory; only the edge operands (B) are read
+// from shared memory.  Every MMA has N = 128: a tcgen05 MMA of N = 64 costs
+// 70 % of the time of one of N = 128 for half the work, so the backward kernel
+// stacks each edge's value and derivative operands into one B tile instead of
+// issuing two N = 64 GEMMs.
 //
 // Ping-pong: the CTA's 16 warps form two math groups of 8 warps.  Group g takes
 // tiles g, g+2, g+4, ... of the CTA's edge run, each with its own TMEM columns,
@@ -58,7 +59,7 @@ struct MPArgs {
     int K;                // Gaussians (columns K .. KP-1 are padding)
     const uint8_t* img;   // this layer's packed W1^T / W2^T images
     const float *s1, *s2, *b1;  // this layer's channel scales and first-layer bias [FP]
-    const float* b2s;     // second-layer bias folded with the base-2 softplus shift [FP]
+    const float* b2;      // this layer's second-layer bias [FP]
     const float* h;       // [N][FP]
     const float* u;       // [N][FP]   (backward)
     float* out;           // m (forward) or dh (backward)   [N][FP]
@@ -275,23 +276,33 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMet
     }
 }
 
-// Issue D (+)= W^T * B over KSTEPS K-steps of 16 with the hi/lo split
-// (A: the weight term in TMEM, 8 columns per K-step; B: MN = 128 rows in
-// shared memory, no-swizzle core matrices).  The two B descriptors are built
-// once; a K-step advances only their 14-bit start-address field (operand
-// regions lie below 256 KB, so the field cannot carry into the strides).
+// Issue D = W^T * B over KSTEPS K-steps of 16 with the hi/lo split (A: the
+// weight term in TMEM, 8 columns per K-step; B: MN = 128 rows in shared
+// memory, no-swizzle core matrices).  The small correction products (lo
+// weight x hi operand, hi weight x lo operand) are issued first and the
+// hi x hi products last: the tensor core's fp32 accumulation does not round
+// to nearest, so each MMA added to an accumulator that already holds the large
+// sum costs accuracy, and this order keeps those additions to one per K-step.
+// The two B descriptors are built once; a K-step advances only their 14-bit
+// start-address field (operand regions lie below 256 KB, so the field cannot
+// carry into the strides).
 template <int NW, int NX, int KSTEPS>
 __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_hi_t, uint32_t a_lo_t, uint32_t b_base,
                                            uint32_t b_term, uint32_t idesc)
 {
     const uint64_t bh0 = smem_desc(b_base, MN * 16, 128);
     const uint64_t bl0 = smem_desc(b_base + b_term, MN * 16, 128);
+    constexpr bool corr = NW == 2 || NX == 2;
 #pragma unroll
     for (int ks = 0; ks < KSTEPS; ++ks) {
         const uint64_t step = (uint64_t)((ks * 2 * MN * 16) >> 4);   // 2 core matrices of 8 along K
-        mma_f16_ts(d_tmem, a_hi_t + ks * 8, bh0 + step, idesc, ks > 0 ? 1u : 0u);
-        if (NW == 2) mma_f16_ts(d_tmem, a_lo_t + ks * 8, bh0 + step, idesc, 1u);
-        if (NX == 2) mma_f16_ts(d_tmem, a_hi_t + ks * 8, bl0 + step, idesc, 1u);
+        if (NW == 2) mma_f16_ts(d_tmem, a_lo_t + ks * 8, bh0 + step, idesc, ks > 0 ? 1u : 0u);
+        if (NX == 2) mma_f16_ts(d_tmem, a_hi_t + ks * 8, bl0 + step, idesc, (NW == 2 || ks > 0) ? 1u : 0u);
+    }
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+        const uint64_t step = (uint64_t)((ks * 2 * MN * 16) >> 4);
+        mma_f16_ts(d_tmem, a_hi_t + ks * 8, bh0 + step, idesc, (corr || ks > 0) ? 1u : 0u);
     }
 }
 
@@ -552,9 +563,9 @@ __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r
     }
 }
 
-// forward epilogue 1 for 32 edges: a = sp2(s1 log2e P + b1 log2e) -> MN-major B
-// operand (the base-2 softplus; ssp = ln2 (a - 1), with ln2 and the shift folded
-// into the second layer's scale and bias)
+// forward epilogue 1 for 32 edges: a = ssp2(s1 log2e P + b1 log2e) -> MN-major B
+// operand (the base-2 shifted softplus: ssp = ln2 a, with ln2 folded into the
+// second layer's scale)
 template <int FMT, int NX>
 __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_t* act, int e0, int f)
 {
@@ -566,7 +577,7 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
         // one pair in four takes its exponentials on the FMA pipe: the MUFU, which the
         // logarithms and the other exponentials keep busy, is this epilogue's bottleneck
         const float2 pp = fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L));
-        const float2 v = ((q >> 1) & 3) == 3 ? sp2x2_fma(pp) : sp2x2(pp);
+        const float2 v = ((q >> 1) & 3) == 3 ? ssp2x2_fma(pp) : ssp2x2(pp);
         r[q] = v.x;
         r[q + 1] = v.y;
     }
@@ -577,10 +588,10 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
     }
 }
 
-// forward epilogue 2 for chunk cc: W = f_c (s2 ln2 Q + b2s), terms h_j W, chunk partials
+// forward epilogue 2 for chunk cc: W = f_c (s2 ln2 Q + b2), terms h_j W, chunk partials
 template <int TE>
 __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* tm, const int32_t* rows_g, int cc,
-                                       int ne, float s2L, float b2s, const float (&hv)[32], float* __restrict__ out,
+                                       int ne, float s2L, float b2, const float (&hv)[32], float* __restrict__ out,
                                        int f, float& pf, float& pl)
 {
     float r[32];
@@ -593,7 +604,7 @@ __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* t
     load_edges<32>(tm->fc, eb, fc);
 #pragma unroll
     for (int q = 0; q < 32; q += 2) {
-        const float2 z = fma2(dup2(s2L), make_float2(r[q], r[q + 1]), dup2(b2s));
+        const float2 z = fma2(dup2(s2L), make_float2(r[q], r[q + 1]), dup2(b2));
         const float2 v = mul2(mul2(make_float2(fc[q], fc[q + 1]), z), make_float2(hv[q], hv[q + 1]));
         r[q] = v.x;
         r[q + 1] = v.y;
@@ -652,7 +663,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     const uint32_t id = idesc_f16(128, MN, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, MN, FMT, 1);
     const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF;
-    const float s2L = a.s2[f] * LN2F, b2s = a.b2s[f];
+    const float s2L = a.s2[f] * LN2F, b2 = a.b2[f];
     const float* h_f = a.h + f;
 
     uint32_t phase = 0, pending = 0;   // pending: a commit of this group not yet waited for
@@ -710,7 +721,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
             const int cc = ch * 2 + c2;
             if (c2 == 1) gather<32>(h_f, tm->col, cc * 32, hv);
             float pf, pl;
-            fwd_e2<TE>(tA + c2 * 32, tm, rows_g, cc, ne, s2L, b2s, hv, a.out, f, pf, pl);
+            fwd_e2<TE>(tA + c2 * 32, tm, rows_g, cc, ne, s2L, b2, hv, a.out, f, pf, pl);
             pf_s[cc * 128 + f] = pf;
             pl_s[cc * 128 + f] = pl;
         }
@@ -735,13 +746,16 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 // ---------------------------------------------------------------------------
 // backward: dh_i = sum_j u_j (.) W_ij ;  s_e = sum_f W'_e,f u_i,f h_j,f
 // ---------------------------------------------------------------------------
-// backward epilogue 1 for this warp's 32 edges: a = sp2(p), b = ssp'(x) dx/dd, with
+// backward epilogue 1 for this warp's 32 edges: a = ssp2(p), b = ssp'(x) dx/dd, with
 // p = x log2e = s1 log2e P + b1 log2e and dx/dd = s1 2ln2 P' (P' from the scaled
-// Gaussian-derivative rows).  ssp'(x) = 1 / (1 + e^-x) shares 2^-|p| with sp2.
+// Gaussian-derivative rows).  With t = 2^-|p| and l = log2((1 + t) / 2) (the
+// logarithm ssp2 takes anyway), the logistic ssp'(x) = 1 / (1 + e^-x) is
+// 2^-l / 2 for p >= 0 and t 2^-l / 2 for p < 0: one more exponential, no
+// division and no cancellation; the factor 1/2 is folded into s1d_half.
 // a goes to B rows e, b to B rows TE + e of GEMM2's operand.  Pairs of
 // elements share the packed fp32x2 FMA/FMUL/FADD instructions.
 template <int FMT, int NX, int TE>
-__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* act,
+__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d_half, uint8_t* act,
                                        int col0, int f)
 {
 #pragma unroll
@@ -754,13 +768,12 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
         for (int q = 0; q < 16; q += 2) {
             const float2 p = fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L));
             const float2 t = make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y)));
-            const float2 y = add2(dup2(1.0f), t);
-            const float2 inv = rcp2_1to2(y);                  // y = 1 + 2^-|p| in [1, 2]
-            const float2 ti = mul2(t, inv);
-            const float2 sg = make_float2(p.x >= 0.0f ? inv.x : ti.x, p.y >= 0.0f ? inv.y : ti.y);   // logistic(x)
-            const float2 a = add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)),
-                                  make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
-            const float2 d = mul2(sg, mul2(dup2(s1d), make_float2(rd[q], rd[q + 1])));
+            const float2 y = fma2(dup2(0.5f), t, dup2(0.5f));               // (1 + t) / 2 in [1/2, 1]
+            const float2 l = make_float2(lg2_mufu(y.x), lg2_mufu(y.y));
+            const float2 g = make_float2(ex2_mufu(-l.x), ex2_mufu(-l.y));   // 2 / (1 + t)
+            const float2 sg = mul2(make_float2(p.x >= 0.0f ? 1.0f : t.x, p.y >= 0.0f ? 1.0f : t.y), g);
+            const float2 a = add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), l);
+            const float2 d = mul2(sg, mul2(dup2(s1d_half), make_float2(rd[q], rd[q + 1])));
             r[q] = a.x;
             r[q + 1] = a.y;
             rd[q] = d.x;
@@ -818,8 +831,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     const uint32_t srbf = smem_u32(rbf), sact = smem_u32(act);
     const uint32_t id = idesc_f16(128, MN, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, MN, FMT, 1);
-    const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF, s1d = a.s1[f] * (2.0f * LN2F);
-    const float s2 = a.s2[f], s2L = a.s2[f] * LN2F, b2s = a.b2s[f];
+    const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF, s1d_half = a.s1[f] * LN2F;
+    const float s2 = a.s2[f], s2L = a.s2[f] * LN2F, b2 = a.b2[f];
     const float* h_f = a.h + f;
     const float* u_f = a.u + f;
 
@@ -858,7 +871,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             if (mt == 0) mbar_arrive(&bars[3]);
             go_sent = true;
         }
-        bwd_e1<FMT, NX, TE>(tP, tPd, s1L, b1L, s1d, act, col0, f);
+        bwd_e1<FMT, NX, TE>(tP, tPd, s1L, b1L, s1d_half, act, col0, f);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
@@ -882,7 +895,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         gather<16>(h_f, tm->col, eb, hv);
         if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2(t) done
         pending = 0;
-        // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 ln2 Q + b2s, z' = s2 Q')
+        // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 ln2 Q + b2, z' = s2 Q')
         {
             const bool active = eb < ne;
             const ChunkInfo ci = tm->c[ch];
@@ -918,7 +931,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 const int q = gq + i;
-                                const float z = fmaf(s2L, r[q], b2s);
+                                const float z = fmaf(s2L, r[q], b2);
                                 if (DH) sf = fmaf(fc[i] * z, uv[q], sf);
                                 const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
                                 rd[q] = wd * (u_first * hv[q]);
@@ -933,7 +946,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
                                 const int q = gq + i;
-                                const float z = fmaf(s2L, r[q], b2s);
+                                const float z = fmaf(s2L, r[q], b2);
                                 const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
                                 if (DH) {
                                     const float dt = fc[i] * z * uv[q];
@@ -957,7 +970,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                                     u_row = __ldg(u_f + (size_t)row * FP);
                                 }
                                 const float fcq = fcp[q], dfcq = dfcp[q];
-                                const float z = fmaf(s2L, r[q], b2s);
+                                const float z = fmaf(s2L, r[q], b2);
                                 const float wd = fmaf(dfcq, z, fcq * (s2 * rd[q]));
                                 if (DH) c.acc = fmaf(fcq * z, uv[q], c.acc);
                                 tval = wd * (u_row * hv[q]);
@@ -1119,7 +1132,7 @@ static MPArgs make_args(schnet_ctx* c, int layer)
     a.s1 = w.s1 + layer * FP;
     a.s2 = w.s2 + layer * FP;
     a.b1 = w.b1 + layer * FP;
-    a.b2s = w.b2s + layer * FP;
+    a.b2 = w.b2 + layer * FP;
     a.h = w.h + (size_t)layer * c->N * FP;
     a.u = w.m;
     a.out = nullptr;

@@ -73,24 +73,14 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-// 1/y for two y in [1, 2] on the FMA pipe (keeps the MUFU free): the linear seed
-// 24/17 - 8/17 y (relative error <= 1/17 on [1, 2]) refined by three Newton
-// steps r <- r + r (1 - y r), each squaring the relative error (1/17)^8 < 2e-10.
-__device__ __forceinline__ float2 rcp2_1to2(float2 y)
+// Shifted softplus in base 2 of two values: for p = x log2(e),
+// ssp2(p) = log2(1 + 2^p) - 1 = log2((1 + e^x) / 2) = ssp(x) / ln2.  Written as
+// max(p, 0) + log2(1/2 + 2^-|p| / 2): no overflow for any p, the logarithm's
+// argument lies in [1/2, 1], and the result has no constant offset (ssp2(0) = 0),
+// so the products that consume it accumulate no large common term.
+__device__ __forceinline__ float2 ssp2x2(float2 p)
 {
-    float2 r = fma2(dup2(-0.47058823529411764f), y, dup2(1.4117647058823529f));
-    const float2 ny = make_float2(-y.x, -y.y);
-#pragma unroll
-    for (int i = 0; i < 3; ++i) r = fma2(r, fma2(ny, r, dup2(1.0f)), r);
-    return r;
-}
-
-// Softplus in base 2 of two values: for p = x log2(e), sp2(p) = log2(1 + 2^p) =
-// log2(1 + e^x), so that ssp(x) = ln2 (sp2(p) - 1).  Written as
-// max(p, 0) + log2(1 + 2^-|p|): no overflow for any p, and 1 + 2^-|p| lies in [1, 2].
-__device__ __forceinline__ float2 sp2x2(float2 p)
-{
-    const float2 y = add2(dup2(1.0f), make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y))));
+    const float2 y = fma2(dup2(0.5f), make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y))), dup2(0.5f));
     return add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
 }
 
@@ -118,10 +108,10 @@ __device__ __forceinline__ float2 ex2_fma2(float2 x)
     return make_float2(__int_as_float(__float_as_int(p.x) + kx), __int_as_float(__float_as_int(p.y) + ky));
 }
 
-// sp2x2 with its exponentials from ex2_fma2 (the logarithms stay on the MUFU)
-__device__ __forceinline__ float2 sp2x2_fma(float2 p)
+// ssp2x2 with its exponentials from ex2_fma2 (the logarithms stay on the MUFU)
+__device__ __forceinline__ float2 ssp2x2_fma(float2 p)
 {
-    const float2 y = add2(dup2(1.0f), ex2_fma2(make_float2(-fabsf(p.x), -fabsf(p.y))));
+    const float2 y = fma2(dup2(0.5f), ex2_fma2(make_float2(-fabsf(p.x), -fabsf(p.y))), dup2(0.5f));
     return add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
 }
 

@@ -1,6 +1,7 @@
 // Host-side context and launcher declarations shared by the library's .cu files.
 #pragma once
 
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 #include <string>
@@ -21,6 +22,26 @@ constexpr int SCAN_ITEMS = 4;         // items per thread
 constexpr int SCAN_TILE = SCAN_BLOCK * SCAN_ITEMS;
 constexpr int REDUCE_CHUNK = 4096;    // atoms per partial sum of a per-replica reduction
 
+// Cells are at least (r_c + skin) (1 + 2^-20) wide and atoms are binned in
+// float64, so the binning's rounding (a few float64 ulps of the cell
+// coordinate) can never put two atoms closer than r_c + skin two cells apart:
+// the 27-cell stencil always sees every listed pair.
+constexpr double CELL_MARGIN = 1.0 + 1.0 / 1048576.0;
+
+// Cells of one grid dimension of length `ext` (host and device agree on it).
+__host__ __device__ inline int cells_across(double ext, double rl, int gmax)
+{
+    const double q = ext / (rl * CELL_MARGIN);
+    int g = q >= (double)gmax ? gmax : (int)floor(q);   // also catches +inf
+    return g < 1 ? 1 : g;                                // and NaN, 0
+}
+
+// Cell-grid placement of one replica: cell coordinate u = (x - org) * inv.
+struct GridGeom {
+    double org[3];
+    double inv[3];
+};
+
 // Per-layer packed tensor-core operand images (bytes) for the filter network.
 constexpr size_t W1_IMG = (size_t)FP * KP * 2;   // one 16-bit term of W1^T (M=128 x K=64)
 constexpr size_t W2_IMG = (size_t)FP * FP * 2;   // one 16-bit term of W2^T (M=128 x K=128)
@@ -33,7 +54,7 @@ struct Workspace {
     // packed weights
     uint8_t* img;                 // [L][LAYER_IMG]
     float *s1, *s2, *b1;          // [L][FP] filter channel scales, first-layer bias
-    float* b2s;                   // [L][FP] second-layer bias minus ln2 s2 sum_k W2^[k][f] (base-2 softplus shift)
+    float* b2;                    // [L][FP] second-layer bias
     float *emb;                   // [T][FP]
     float *emb_h0;                // [T][FP] emb W_in of interaction 0 (the first h of every atom of a type)
     uint8_t* aw_img;              // [6 L + 2][AW_IMG] atom-wise layers as tensor-core A operands
@@ -58,8 +79,7 @@ struct Workspace {
     int32_t *cell_cnt, *cell_start, *cell_fill;  // [ncell+1]
     int32_t* rep_off;             // [R+1] replica offsets
     int4* rgrid_dims;             // [R]   (gx, gy, gz, first cell)
-    float4* rgrid_org;            // [R]   grid origin
-    float4* rgrid_inv;            // [R]   inverse cell sizes
+    GridGeom* rgrid_geom;         // [R]   grid origin and inverse cell sizes (float64)
     long long* scan_tmp;          // [SCAN_TILE] tile sums
     // activations
     float *x, *h, *q, *m, *g, *dh, *pr, *eps, *ke;

@@ -171,15 +171,16 @@ cudaError_t launch_pack_positions(schnet_ctx* c, const float* d_pos)
 struct GridParams {
     int periodic;
     int gp[3];          // periodic grid dims
-    float rl;           // list radius
+    double rl;          // list radius r_c + skin
     int gmax;           // non-periodic max dims
     int cells_per_rep;  // stride between replicas' cell ranges
 };
 
-// one block per replica: bounding box (non-periodic) and grid dims
+// One block per replica: grid dims and placement.  Periodic: the box's grid.
+// Open boundaries: the replica's bounding box, split into cells_across() cells
+// per dimension (at least r_c + skin wide, at most gmax per dimension).
 __global__ void k_replica_grid(int R, const int32_t* __restrict__ rep_off, const float4* __restrict__ pos4,
-                               GridParams gp, const Box box, int4* __restrict__ dims, float4* __restrict__ org,
-                               float4* __restrict__ inv)
+                               GridParams gp, const Box box, int4* __restrict__ dims, GridGeom* __restrict__ geom)
 {
     int r = blockIdx.x;
     if (r >= R) return;
@@ -187,8 +188,12 @@ __global__ void k_replica_grid(int R, const int32_t* __restrict__ rep_off, const
     if (gp.periodic) {
         if (threadIdx.x == 0) {
             dims[r] = make_int4(gp.gp[0], gp.gp[1], gp.gp[2], r * gp.cells_per_rep);
-            org[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-            inv[r] = make_float4(gp.gp[0] * box.invL[0], gp.gp[1] * box.invL[1], gp.gp[2] * box.invL[2], 0.f);
+            GridGeom gm;
+            for (int d = 0; d < 3; ++d) {
+                gm.org[d] = 0.0;
+                gm.inv[d] = (double)gp.gp[d] / (double)box.L[d];
+            }
+            geom[r] = gm;
         }
         return;
     }
@@ -213,48 +218,50 @@ __global__ void k_replica_grid(int R, const int32_t* __restrict__ rep_off, const
     if (threadIdx.x == 0) {
         int nw = blockDim.x >> 5;
         int g[3];
-        float o3[3], iv[3];
+        GridGeom gm;
         for (int d = 0; d < 3; ++d) {
             float l = 3.4e38f, h = -3.4e38f;
             for (int w = 0; w < nw; ++w) { l = fminf(l, slo[d][w]); h = fmaxf(h, shi[d][w]); }
             if (!(h >= l)) { l = 0.f; h = 0.f; }   // empty replica or non-finite
-            float ext = h - l;
-            int gd = (int)floorf(ext / gp.rl);
-            gd = gd < 1 ? 1 : (gd > gp.gmax ? gp.gmax : gd);
+            const double ext = (double)h - (double)l;   // exact for float inputs
+            const int gd = cells_across(ext, gp.rl, gp.gmax);
             g[d] = gd;
-            o3[d] = l;
-            iv[d] = ext > 0.f ? (float)gd / ext : 0.f;
+            gm.org[d] = (double)l;
+            gm.inv[d] = ext > 0.0 ? (double)gd / ext : 0.0;
         }
         dims[r] = make_int4(g[0], g[1], g[2], r * gp.cells_per_rep);
-        org[r] = make_float4(o3[0], o3[1], o3[2], 0.f);
-        inv[r] = make_float4(iv[0], iv[1], iv[2], 0.f);
+        geom[r] = gm;
     }
 }
 
-__device__ __forceinline__ int cell_coord(float x, float o, float iv, int g, int periodic)
+// Cell coordinate of x along one dimension: floor((x - o) inv) in float64
+// (periodic: wrapped into [0, g); open: clamped, only rounding can leave the range).
+__device__ __forceinline__ int cell_coord(float x, double o, double iv, int g, int periodic)
 {
-    int c = (int)floorf((x - o) * iv);
+    const double u = floor(((double)x - o) * iv);
     if (periodic) {
-        c %= g;
-        if (c < 0) c += g;
+        if (!(fabs(u) < 1.0e15)) return 0;   // non-finite or absurd positions (flagged elsewhere)
+        double w = u - (double)g * floor(u / (double)g);
+        int c = (int)w;
+        return c < 0 ? 0 : (c >= g ? g - 1 : c);
     }
-    return c < 0 ? 0 : (c >= g ? g - 1 : c);
+    if (!(u >= 0.0)) return 0;               // also NaN
+    return u >= (double)g ? g - 1 : (int)u;
 }
 
 __global__ void k_cell_assign(int n, const float4* __restrict__ pos4, const int32_t* __restrict__ atom_rep,
-                              const int4* __restrict__ dims, const float4* __restrict__ org,
-                              const float4* __restrict__ inv, int periodic, int32_t* __restrict__ cell_of,
-                              int32_t* __restrict__ cell_cnt)
+                              const int4* __restrict__ dims, const GridGeom* __restrict__ geom, int periodic,
+                              int32_t* __restrict__ cell_of, int32_t* __restrict__ cell_cnt)
 {
     int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
     int r = atom_rep[i];
     float4 p = pos4[i];
     int4 g = dims[r];
-    float4 o = org[r], v = inv[r];
-    int cx = cell_coord(p.x, o.x, v.x, g.x, periodic);
-    int cy = cell_coord(p.y, o.y, v.y, g.y, periodic);
-    int cz = cell_coord(p.z, o.z, v.z, g.z, periodic);
+    const GridGeom gm = geom[r];
+    int cx = cell_coord(p.x, gm.org[0], gm.inv[0], g.x, periodic);
+    int cy = cell_coord(p.y, gm.org[1], gm.inv[1], g.y, periodic);
+    int cz = cell_coord(p.z, gm.org[2], gm.inv[2], g.z, periodic);
     int cell = g.w + cx + g.x * (cy + g.y * cz);
     cell_of[i] = cell;
     atomicAdd(&cell_cnt[cell], 1);
@@ -336,24 +343,25 @@ __device__ __forceinline__ void for_each_neighbor(int i, const float4* __restric
     int local = cell_of[i] - g.w;
     int cx = local % g.x, cy = (local / g.x) % g.y, cz = local / (g.x * g.y);
     float4 pi = pos4[i];
-    // stencil offsets per dimension: periodic grids with < 3 cells visit each cell once
-    int lox = -1, hix = 1, loy = -1, hiy = 1, loz = -1, hiz = 1;
-    if (box.periodic) {
-        if (g.x < 3) { lox = 0; hix = g.x - 1; }
-        if (g.y < 3) { loy = 0; hiy = g.y - 1; }
-        if (g.z < 3) { loz = 0; hiz = g.z - 1; }
-    }
+    // Stencil per dimension: the cell and its two neighbours (wrapped when
+    // periodic, cut at the grid's edge when not).  A periodic dimension with
+    // fewer than 3 cells has every cell within reach: it visits each cell once
+    // by absolute index (wrapped offsets would visit one cell twice).
+    const bool allx = box.periodic && g.x < 3, ally = box.periodic && g.y < 3, allz = box.periodic && g.z < 3;
+    const int lox = allx ? 0 : -1, hix = allx ? g.x - 1 : 1;
+    const int loy = ally ? 0 : -1, hiy = ally ? g.y - 1 : 1;
+    const int loz = allz ? 0 : -1, hiz = allz ? g.z - 1 : 1;
     for (int oz = loz; oz <= hiz; ++oz) {
-        int z = cz + oz;
-        if (box.periodic) { if (g.z >= 3) z = (z + g.z) % g.z; }
+        int z = allz ? oz : cz + oz;
+        if (box.periodic) { if (!allz) z = (z + g.z) % g.z; }
         else if (z < 0 || z >= g.z) continue;
         for (int oy = loy; oy <= hiy; ++oy) {
-            int y = cy + oy;
-            if (box.periodic) { if (g.y >= 3) y = (y + g.y) % g.y; }
+            int y = ally ? oy : cy + oy;
+            if (box.periodic) { if (!ally) y = (y + g.y) % g.y; }
             else if (y < 0 || y >= g.y) continue;
             for (int ox = lox; ox <= hix; ++ox) {
-                int x = cx + ox;
-                if (box.periodic) { if (g.x >= 3) x = (x + g.x) % g.x; }
+                int x = allx ? ox : cx + ox;
+                if (box.periodic) { if (!allx) x = (x + g.x) % g.x; }
                 else if (x < 0 || x >= g.x) continue;
                 int cell = g.w + x + g.x * (y + g.y * z);
                 int a = cell_start[cell], b = cell_start[cell + 1];
@@ -478,7 +486,7 @@ cudaError_t launch_build_neighbors(schnet_ctx* c, const float* d_pos)
     GridParams gp;
     gp.periodic = c->cfg.periodic;
     gp.gp[0] = c->gdim[0]; gp.gp[1] = c->gdim[1]; gp.gp[2] = c->gdim[2];
-    gp.rl = c->cfg.cutoff + c->cfg.skin;
+    gp.rl = (double)c->cfg.cutoff + (double)c->cfg.skin;
     gp.gmax = GMAX_NONPERIODIC;
     gp.cells_per_rep = c->ncell / R;
     cudaError_t err;
@@ -486,11 +494,11 @@ cudaError_t launch_build_neighbors(schnet_ctx* c, const float* d_pos)
     float4* posc4 = w.ref4;   // caller-order positions; replaced by the slot-order reference at the end
 
     k_pack_positions<<<nb, 256, 0, c->s>>>(N, d_pos, nullptr, posc4, nullptr, 0, 0.f, w.meta);
-    k_replica_grid<<<R, 256, 0, c->s>>>(R, w.rep_off, posc4, gp, c->box, w.rgrid_dims, w.rgrid_org, w.rgrid_inv);
+    k_replica_grid<<<R, 256, 0, c->s>>>(R, w.rep_off, posc4, gp, c->box, w.rgrid_dims, w.rgrid_geom);
     cudaMemsetAsync(w.cell_cnt, 0, sizeof(int32_t) * (c->ncell + 1), c->s);
     cudaMemsetAsync(w.cell_fill, 0, sizeof(int32_t) * (c->ncell + 1), c->s);
-    k_cell_assign<<<nb, 256, 0, c->s>>>(N, posc4, w.atom_rep, w.rgrid_dims, w.rgrid_org, w.rgrid_inv,
-                                        gp.periodic, w.cell_of, w.cell_cnt);
+    k_cell_assign<<<nb, 256, 0, c->s>>>(N, posc4, w.atom_rep, w.rgrid_dims, w.rgrid_geom, gp.periodic,
+                                        w.cell_of, w.cell_cnt);
     c->launches += 3;
     if ((err = scan_exclusive(c, w.cell_cnt, c->ncell, w.cell_start, nullptr)) != cudaSuccess) return err;
     k_cell_fill<<<nb, 256, 0, c->s>>>(N, w.cell_of, w.cell_start, w.cell_fill, w.cell_atoms);
@@ -612,9 +620,8 @@ constexpr size_t NA_OFF_CCNT = na_align(NA_OFF_ROWCNT + sizeof(int32_t) * (NA_MA
 constexpr size_t NA_OFF_CSTART = na_align(NA_OFF_CCNT + sizeof(int32_t) * (NA_MAX_CELLS + 1));
 constexpr size_t NA_OFF_CFILL = na_align(NA_OFF_CSTART + sizeof(int32_t) * (NA_MAX_CELLS + 1));
 constexpr size_t NA_OFF_DIMS = na_align(NA_OFF_CFILL + sizeof(int32_t) * (NA_MAX_CELLS + 1));
-constexpr size_t NA_OFF_ORG = na_align(NA_OFF_DIMS + sizeof(int4) * NA_MAX_REPLICAS);
-constexpr size_t NA_OFF_INV = na_align(NA_OFF_ORG + sizeof(float4) * NA_MAX_REPLICAS);
-constexpr size_t NA_OFF_SCAN = na_align(NA_OFF_INV + sizeof(float4) * NA_MAX_REPLICAS);
+constexpr size_t NA_OFF_GEOM = na_align(NA_OFF_DIMS + sizeof(int4) * NA_MAX_REPLICAS);
+constexpr size_t NA_OFF_SCAN = na_align(NA_OFF_GEOM + sizeof(GridGeom) * NA_MAX_REPLICAS);
 constexpr size_t NA_BYTES = na_align(NA_OFF_SCAN + sizeof(long long) * SCAN_TILE);   // about 3.6 MB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NA_BYTES];
@@ -676,7 +683,13 @@ __global__ void k_rev_rows(int n, const int32_t* __restrict__ row_ptr, const int
     }
 }
 
-__global__ void k_copy_edge_count(const DevMeta* meta, int64_t* out) { *out = meta->n_edges; }
+// edge count and status bits (non-finite positions, list over capacity) out to the caller
+__global__ void k_copy_edge_count(DevMeta* meta, long long cap, int64_t* out, uint32_t* flags)
+{
+    if (meta->n_edges > cap) set_flag(meta, SCHNET_FLAG_CAPACITY);
+    *out = meta->n_edges;
+    if (flags) *flags = meta->status;
+}
 
 static cudaError_t scan_exclusive_raw(cudaStream_t s, const int32_t* in, int n, int32_t* out, long long* total64,
                                       long long* tmp)
@@ -696,12 +709,15 @@ extern "C" schnet_status schnet_build_neighbors_noalloc(const float* d_pos, int3
                                                         const int32_t* d_replica_offsets, float cutoff, float skin,
                                                         int32_t periodic, const float* box, int32_t* d_row_ptr,
                                                         int32_t* d_col, int32_t* d_rev, int64_t edge_capacity,
-                                                        int64_t* d_n_edges, void* cuda_stream)
+                                                        int64_t* d_n_edges, uint32_t* d_flags, void* cuda_stream)
 {
     using namespace schnet;
     if (!d_pos || !d_replica_offsets || !d_row_ptr || !d_col || !d_rev || !d_n_edges || n_atoms < 1 ||
         n_replicas < 1 || edge_capacity < 1 || !(cutoff > 0.f) || !(skin >= 0.f) || (periodic && !box))
         return SCHNET_ERR_INVALID_ARG;
+    // An error left pending by someone else's earlier launch is theirs to read: report it
+    // without clearing it, so that the launch-error check at the end sees only this call's.
+    if (cudaPeekAtLastError() != cudaSuccess) return SCHNET_ERR_CUDA;
     const double rl = (double)cutoff + (double)skin;
     int gdim[3] = {GMAX_NONPERIODIC, GMAX_NONPERIODIC, GMAX_NONPERIODIC};
     Box bx;
@@ -711,8 +727,7 @@ extern "C" schnet_status schnet_build_neighbors_noalloc(const float* d_pos, int3
         bx.invL[d] = periodic ? 1.0f / box[d] : 0.f;
         if (periodic) {
             if (!(box[d] >= 2.0f * (cutoff + skin))) return SCHNET_ERR_UNSUPPORTED;
-            int g = (int)std::floor((double)box[d] / rl);
-            gdim[d] = g < 1 ? 1 : (g > GMAX_PERIODIC ? GMAX_PERIODIC : g);
+            gdim[d] = cells_across((double)box[d], rl, GMAX_PERIODIC);
         }
     }
     const long long cells_per_rep = (long long)gdim[0] * gdim[1] * gdim[2];
@@ -733,8 +748,7 @@ extern "C" schnet_status schnet_build_neighbors_noalloc(const float* d_pos, int3
     int32_t* cstart = reinterpret_cast<int32_t*>(base + NA_OFF_CSTART);
     int32_t* cfill = reinterpret_cast<int32_t*>(base + NA_OFF_CFILL);
     int4* dims = reinterpret_cast<int4*>(base + NA_OFF_DIMS);
-    float4* org = reinterpret_cast<float4*>(base + NA_OFF_ORG);
-    float4* inv = reinterpret_cast<float4*>(base + NA_OFF_INV);
+    GridGeom* geom = reinterpret_cast<GridGeom*>(base + NA_OFF_GEOM);
     long long* scan_tmp = reinterpret_cast<long long*>(base + NA_OFF_SCAN);
 
     cudaStream_t s = (cudaStream_t)cuda_stream;
@@ -743,7 +757,7 @@ extern "C" schnet_status schnet_build_neighbors_noalloc(const float* d_pos, int3
     GridParams gp;
     gp.periodic = bx.periodic;
     gp.gp[0] = gdim[0]; gp.gp[1] = gdim[1]; gp.gp[2] = gdim[2];
-    gp.rl = cutoff + skin;
+    gp.rl = rl;
     gp.gmax = GMAX_NONPERIODIC;
     gp.cells_per_rep = (int)cells_per_rep;
     const double rl2 = rl * rl;
@@ -753,8 +767,8 @@ extern "C" schnet_status schnet_build_neighbors_noalloc(const float* d_pos, int3
     if (cudaMemsetAsync(cfill, 0, sizeof(int32_t) * (ncell + 1), s) != cudaSuccess) return SCHNET_ERR_CUDA;
     k_pack_positions<<<nb, 256, 0, s>>>(N, d_pos, nullptr, pos4, nullptr, 0, 0.f, meta);
     k_atom_replica<<<nb, 256, 0, s>>>(N, R, d_replica_offsets, arep);
-    k_replica_grid<<<R, 256, 0, s>>>(R, d_replica_offsets, pos4, gp, bx, dims, org, inv);
-    k_cell_assign<<<nb, 256, 0, s>>>(N, pos4, arep, dims, org, inv, gp.periodic, cell_of, ccnt);
+    k_replica_grid<<<R, 256, 0, s>>>(R, d_replica_offsets, pos4, gp, bx, dims, geom);
+    k_cell_assign<<<nb, 256, 0, s>>>(N, pos4, arep, dims, geom, gp.periodic, cell_of, ccnt);
     if (scan_exclusive_raw(s, ccnt, (int)ncell, cstart, nullptr, scan_tmp) != cudaSuccess) return SCHNET_ERR_CUDA;
     k_cell_fill<<<nb, 256, 0, s>>>(N, cell_of, cstart, cfill, catoms);
     k_count<<<nb128, 128, 0, s>>>(N, pos4, arep, cell_of, dims, cstart, catoms, rl2, bx, rowcnt);
@@ -765,6 +779,6 @@ extern "C" schnet_status schnet_build_neighbors_noalloc(const float* d_pos, int3
                                  meta, d_rev, d_col);
     k_sort_rows<<<256, 256, 0, s>>>(N, d_row_ptr, d_rev, edge_capacity, meta, d_col);
     k_rev_rows<<<256, 256, 0, s>>>(N, d_row_ptr, d_col, edge_capacity, meta, d_rev);
-    k_copy_edge_count<<<1, 1, 0, s>>>(meta, d_n_edges);
+    k_copy_edge_count<<<1, 1, 0, s>>>(meta, edge_capacity, d_n_edges, d_flags);
     return cudaGetLastError() == cudaSuccess ? SCHNET_OK : SCHNET_ERR_CUDA;
 }

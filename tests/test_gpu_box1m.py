@@ -30,8 +30,9 @@ def box_run():
     eps = model.atom_energies()
     torch.cuda.synchronize()
     assert model.status() == 0
+    rp, col, _ = model.neighbors()
     out = dict(pos=pos, types=types, weights=weights, E=E.cpu().numpy(), F=F.cpu().numpy(),
-               eps=eps.cpu().numpy(), E_list=len(model.neighbors()[1]))
+               eps=eps.cpu().numpy(), E_list=len(col), row_ptr=rp, col=col)
     model.close()
     return out
 
@@ -42,6 +43,36 @@ def _cluster(pos, c, radius):
     sel = np.flatnonzero((d * d).sum(1) < radius * radius)
     local = np.concatenate([[c], sel[sel != c]])
     return local, pos[c].astype(np.float64) + d[local]
+
+
+def test_sampled_rows_bit_exact(box_run):
+    # 1,000 seeded atoms: each one's row of the full 10^6-bead list against the brute-force
+    # definition on the atoms of its (r_c + skin + 1 A) ball, kept in their original (unwrapped)
+    # coordinates so the oracle's periodic pair test is the very one the full list uses.  The
+    # balls go to the oracle as separate replicas of one call (edges never cross replicas).
+    from scipy.spatial import cKDTree
+    pos = box_run["pos"]
+    rl = W.cutoff + W.skin
+    rng = np.random.default_rng(99)
+    centres = rng.choice(W.n_atoms, size=1000, replace=False)
+    wrapped = np.mod(pos.astype(np.float64), W.box)
+    wrapped[wrapped >= W.box] = 0.0
+    tree = cKDTree(wrapped, boxsize=W.box)
+    balls = [np.asarray(sorted(tree.query_ball_point(wrapped[c], rl + 1.0)), dtype=np.int64) for c in centres]
+    balls = [np.concatenate([[c], b[b != c]]) for c, b in zip(centres, balls)]
+    ro = np.concatenate([[0], np.cumsum([len(b) for b in balls])]).astype(np.int32)
+    sub = pos[np.concatenate(balls)]
+    rp_o, col_o = oracle.neighbors(sub, W.cutoff, W.skin, ro, True, (W.box,) * 3)
+    rp, col = box_run["row_ptr"], box_run["col"]
+    n_checked = 0
+    for k, (c, b) in enumerate(zip(centres, balls)):
+        first = ro[k]                      # atom c is its ball's first atom
+        local = col_o[rp_o[first]:rp_o[first + 1]] - first
+        expect = np.sort(b[local])
+        got = col[rp[c]:rp[c + 1]]
+        assert np.array_equal(got, expect), f"row {c}"
+        n_checked += len(got)
+    assert n_checked > 1000 * 100
 
 
 def test_edge_count_matches_density(box_run):

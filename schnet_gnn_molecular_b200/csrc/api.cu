@@ -154,6 +154,8 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.crow = cv.take<int32_t>(d.cap); w.ccol = cv.take<int32_t>(d.cap); w.cidx = cv.take<int32_t>(d.cap);
     w.ccount = cv.take<int32_t>(MAX_CTA);
     w.part = cv.take<int32_t>(MAX_CTA + 1);
+    w.ccount_h = cv.take<int32_t>(MAX_CTA);
+    w.part_h = cv.take<int32_t>(MAX_CTA + 1);
     w.cell_of = cv.take<int32_t>(N); w.cell_atoms = cv.take<int32_t>(N);
     w.cell_cnt = cv.take<int32_t>((size_t)d.ncell + 1); w.cell_start = cv.take<int32_t>((size_t)d.ncell + 1);
     w.cell_fill = cv.take<int32_t>((size_t)d.ncell + 1);
@@ -270,11 +272,22 @@ void build_weight_blob(const schnet_ctx* c, const schnet_weights* wt, uint8_t* w
         uint16_t* w2lo = reinterpret_cast<uint16_t*>(img + 2 * W1_IMG + W2_IMG);
         pack_operand(W1, K, F, KP, s1, fmt, c->n_wterms, w1hi, w1lo);
         pack_operand(W2, F, F, FP, s2, fmt, c->n_wterms, w2hi, w2lo);
+        // With one 16-bit activation term the kernels feed the second layer
+        // a = log2(1 + e^x) = ssp(x) / ln2 + 1 (see the forward epilogue): the -1 goes
+        // into the bias as -ln2 s2 times the column sum of the stored weight terms.
+        std::vector<double> colsum(FP, 0.0);
+        if (c->n_xterms == 1)
+            for (int f = 0; f < FP; ++f)
+                for (int k = 0; k < FP; ++k) {
+                    const size_t idx = kmajor_off(f, k, FP) / 2;
+                    colsum[f] += from16(w2hi[idx], fmt) + (c->n_wterms == 2 ? from16(w2lo[idx], fmt) : 0.0);
+                }
         for (int f = 0; f < FP; ++f) {
             H(w.s1)[l * FP + f] = (float)s1[f];
             H(w.s2)[l * FP + f] = (float)s2[f];
             H(w.b1)[l * FP + f] = f < F ? wt->b1[l * F + f] : 0.f;
-            H(w.b2)[l * FP + f] = f < F ? wt->b2[l * F + f] : 0.f;
+            const double b2 = f < F ? (double)wt->b2[l * F + f] : 0.0;
+            H(w.b2)[l * FP + f] = (float)(b2 - 0.69314718055994530942 * s2[f] * colsum[f]);
             H(w.bo1)[l * FP + f] = f < F ? wt->bo1[l * F + f] : 0.f;
             H(w.bo2)[l * FP + f] = f < F ? wt->bo2[l * F + f] : 0.f;
         }
@@ -518,6 +531,9 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
     if (!need_forces) return cudaSuccess;
     SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd_top(c));
     for (int l = c->L - 1; l >= 0; --l) {
+        // interaction 0 runs over the half list (one edge per unordered pair), which
+        // replaces the compacted runs of the later interactions' launches
+        if (l == 0) SCHNET_TIMED(SCHNET_KERNEL_MASK, launch_compact_half(c));
         SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_bwd(c, l, l < c->L - 1 ? 1 : 0));
         // interaction 0: dE/dx^0 is a gradient with respect to the embedding, not needed for forces
         if (l > 0) SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd(c, l));

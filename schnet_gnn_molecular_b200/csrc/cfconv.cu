@@ -17,7 +17,8 @@
 // mode tangents and produces dE/dh_j (segment sum over the symmetric list) and
 // the per-edge scalar s_e = sum_f W'_f u_i,f h_j,f (the edge's share of dE/dd);
 // for the first interaction, whose dE/dh only feeds the embedding's gradient,
-// it produces s_e alone.
+// it visits each unordered pair once (the half list, exploiting W_ij = W_ji)
+// and produces the pair's whole derivative sum_f W'_f (u_i h_j + u_j h_i).
 //
 // Tile orientation: the GEMMs are computed transposed, D[f][e] = W^T[f][k] B[e][k],
 // so TMEM lane = output feature and TMEM column = edge.  Each epilogue thread
@@ -565,7 +566,8 @@ __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r
 
 // forward epilogue 1 for 32 edges: a = ssp2(s1 log2e P + b1 log2e) -> MN-major B
 // operand (the base-2 shifted softplus: ssp = ln2 a, with ln2 folded into the
-// second layer's scale)
+// second layer's scale).  With one 16-bit activation term (NX = 1) the operand is
+// sp2 = ssp2 + 1 instead, and the -1 is folded into the second layer's bias.
 template <int FMT, int NX>
 __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_t* act, int e0, int f)
 {
@@ -577,7 +579,7 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
         // one pair in four takes its exponentials on the FMA pipe: the MUFU, which the
         // logarithms and the other exponentials keep busy, is this epilogue's bottleneck
         const float2 pp = fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L));
-        const float2 v = ((q >> 1) & 3) == 3 ? ssp2x2_fma(pp) : ssp2x2(pp);
+        const float2 v = ((q >> 1) & 3) == 3 ? sp2x2_fma<NX == 2>(pp) : sp2x2<NX == 2>(pp);
         r[q] = v.x;
         r[q + 1] = v.y;
     }
@@ -751,11 +753,13 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 // Gaussian-derivative rows).  With t = 2^-|p| and l = log2((1 + t) / 2) (the
 // logarithm ssp2 takes anyway), the logistic ssp'(x) = 1 / (1 + e^-x) is
 // 2^-l / 2 for p >= 0 and t 2^-l / 2 for p < 0: one more exponential, no
-// division and no cancellation; the factor 1/2 is folded into s1d_half.
+// division and no cancellation; the factor 1/2 is folded into s1d.  With one
+// 16-bit activation term (NX = 1) a is sp2 = ssp2 + 1 and l = log2(1 + t) (see
+// the forward epilogue), and s1d has no factor 1/2.
 // a goes to B rows e, b to B rows TE + e of GEMM2's operand.  Pairs of
 // elements share the packed fp32x2 FMA/FMUL/FADD instructions.
 template <int FMT, int NX, int TE>
-__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d_half, uint8_t* act,
+__device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, float b1L, float s1d, uint8_t* act,
                                        int col0, int f)
 {
 #pragma unroll
@@ -768,12 +772,13 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
         for (int q = 0; q < 16; q += 2) {
             const float2 p = fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L));
             const float2 t = make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y)));
-            const float2 y = fma2(dup2(0.5f), t, dup2(0.5f));               // (1 + t) / 2 in [1/2, 1]
+            constexpr float c = NX == 2 ? 0.5f : 1.0f;
+            const float2 y = fma2(dup2(c), t, dup2(c));                     // c (1 + t)
             const float2 l = make_float2(lg2_mufu(y.x), lg2_mufu(y.y));
-            const float2 g = make_float2(ex2_mufu(-l.x), ex2_mufu(-l.y));   // 2 / (1 + t)
+            const float2 g = make_float2(ex2_mufu(-l.x), ex2_mufu(-l.y));   // 1 / (c (1 + t))
             const float2 sg = mul2(make_float2(p.x >= 0.0f ? 1.0f : t.x, p.y >= 0.0f ? 1.0f : t.y), g);
             const float2 a = add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), l);
-            const float2 d = mul2(sg, mul2(dup2(s1d_half), make_float2(rd[q], rd[q + 1])));
+            const float2 d = mul2(sg, mul2(dup2(s1d), make_float2(rd[q], rd[q + 1])));
             r[q] = a.x;
             r[q + 1] = a.y;
             rd[q] = d.x;
@@ -788,9 +793,14 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
     }
 }
 
-// DH = false: only the per-edge s_e (forces) -- no dE/dh_j segment sums, no u_j
-// gathers, no merge.  Used for the first interaction, whose dE/dh feeds only the
-// gradient with respect to the embedding, which forces do not need.
+// DH = false: the pair derivative over the half list -- no dE/dh_j segment sums,
+// no merge.  Used for the first interaction, whose dE/dh feeds only the gradient
+// with respect to the embedding, which forces do not need; its forces need only
+// dE/dd_ij = D_ij = sum_f W'_f(d_ij) (u_i,f h_j,f + u_j,f h_i,f), the same for
+// (i, j) and (j, i) because W_ij = W_ji.  So the launch runs over one edge per
+// unordered pair (the edges (i, j) with j > i, in rows balanced by their own
+// partition) and adds D_ij to s_e of that edge alone; the force assembly sums
+// s_e + s_rev(e), so both atoms of the pair receive it.
 template <int FMT, int NW, int NX, bool DH>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
@@ -831,7 +841,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     const uint32_t srbf = smem_u32(rbf), sact = smem_u32(act);
     const uint32_t id = idesc_f16(128, MN, FMT, 0);
     const uint32_t id_mn = idesc_f16(128, MN, FMT, 1);
-    const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF, s1d_half = a.s1[f] * LN2F;
+    const float s1L = a.s1[f] * LOG2EF, b1L = a.b1[f] * LOG2EF, s1d = a.s1[f] * (NX == 2 ? LN2F : 2.0f * LN2F);
     const float s2 = a.s2[f], s2L = a.s2[f] * LN2F, b2 = a.b2[f];
     const float* h_f = a.h + f;
     const float* u_f = a.u + f;
@@ -871,7 +881,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             if (mt == 0) mbar_arrive(&bars[3]);
             go_sent = true;
         }
-        bwd_e1<FMT, NX, TE>(tP, tPd, s1L, b1L, s1d_half, act, col0, f);
+        bwd_e1<FMT, NX, TE>(tP, tPd, s1L, b1L, s1d, act, col0, f);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
@@ -891,7 +901,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         }
         const int eb = col0;
         float uv[16], hv[16];
-        if (DH) gather<16>(u_f, tm->col, eb, uv);
+        gather<16>(u_f, tm->col, eb, uv);
         gather<16>(h_f, tm->col, eb, hv);
         if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2(t) done
         pending = 0;
@@ -906,6 +916,10 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             if (kind != 0) {
                 const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
                 const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
+                // half list: the row atom's own h_i for the reverse direction's term u_j h_i
+                const float h_first = DH ? 0.f : __ldg(h_f + (size_t)ci.rfirst * FP);
+                const float h_last = DH ? 0.f : __ldg(h_f + (size_t)ci.rlast * FP);
+                float h_row = h_first;
                 float sf = 0.f, sl = 0.f;
                 ChunkSeg c;
                 seg_begin(c, ci.rfirst);
@@ -913,7 +927,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     if (hh == 1) {
-                        if (DH) gather<16>(u_f, tm->col, eb + 16, uv);
+                        gather<16>(u_f, tm->col, eb + 16, uv);
                         gather<16>(h_f, tm->col, eb + 16, hv);
                     }
                     float r[16], rd[16];
@@ -934,7 +948,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                                 const float z = fmaf(s2L, r[q], b2);
                                 if (DH) sf = fmaf(fc[i] * z, uv[q], sf);
                                 const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
-                                rd[q] = wd * (u_first * hv[q]);
+                                rd[q] = DH ? wd * (u_first * hv[q]) : wd * fmaf(uv[q], h_first, u_first * hv[q]);
                             }
                         }
                     } else if (kind == 2) {
@@ -954,7 +968,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                                     sl += first ? 0.f : dt;
                                 }
                                 const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
-                                rd[q] = wd * ((first ? u_first : u_last) * hv[q]);
+                                const float ui = first ? u_first : u_last;
+                                rd[q] = DH ? wd * (ui * hv[q]) : wd * fmaf(uv[q], first ? h_first : h_last, ui * hv[q]);
                             }
                         }
                     } else {
@@ -968,12 +983,13 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                                     if (DH) seg_row(c, row, a.out, f);
                                     else c.lrow = row;
                                     u_row = __ldg(u_f + (size_t)row * FP);
+                                    if (!DH) h_row = __ldg(h_f + (size_t)row * FP);
                                 }
                                 const float fcq = fcp[q], dfcq = dfcp[q];
                                 const float z = fmaf(s2L, r[q], b2);
                                 const float wd = fmaf(dfcq, z, fcq * (s2 * rd[q]));
                                 if (DH) c.acc = fmaf(fcq * z, uv[q], c.acc);
-                                tval = wd * (u_row * hv[q]);
+                                tval = DH ? wd * (u_row * hv[q]) : wd * fmaf(uv[q], h_row, u_row * hv[q]);
                             }
                             rd[q] = tval;
                         }
@@ -1040,6 +1056,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 // ---------------------------------------------------------------------------
 // cutoff masking: per CTA row range, the listed edges with d < r_c, in order
 // ---------------------------------------------------------------------------
+template <bool HALF>
 __global__ void __launch_bounds__(1024) k_compact(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ part,
                                                   const int32_t* __restrict__ erow, const int32_t* __restrict__ col,
                                                   const float4* __restrict__ pos4, Box box, float rc, long long cap,
@@ -1047,6 +1064,7 @@ __global__ void __launch_bounds__(1024) k_compact(const int32_t* __restrict__ ro
                                                   int32_t* __restrict__ ccol, int32_t* __restrict__ cidx,
                                                   int32_t* __restrict__ ccount)
 {
+    constexpr int CI = 4;             // consecutive edges per thread and pass
     __shared__ int wcount[32];
     __shared__ int total_s;
     const int c = blockIdx.x;
@@ -1058,37 +1076,59 @@ __global__ void __launch_bounds__(1024) k_compact(const int32_t* __restrict__ ro
     const long long e0 = row_ptr[r0], e1 = row_ptr[r1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     long long base = e0;
-    for (long long eb = e0; eb < e1; eb += blockDim.x) {
-        const long long e = eb + threadIdx.x;
-        bool valid = false;
-        int i = 0, j = 0;
-        if (e < e1) {
-            i = erow[e];
-            j = col[e];
-            float3 v;
-            const float d = edge_distance(pos4[i], pos4[j], box, v);
-            valid = d < rc && d > 0.f;
+    for (long long eb = e0; eb < e1; eb += (long long)CI * blockDim.x) {
+        const long long ef = eb + (long long)CI * threadIdx.x;
+        int ii[CI], jj[CI];
+        unsigned vmask = 0;
+#pragma unroll
+        for (int q = 0; q < CI; ++q) {
+            ii[q] = 0;
+            jj[q] = 0;
+            if (ef + q < e1) {
+                ii[q] = erow[ef + q];
+                jj[q] = col[ef + q];
+            }
         }
-        const unsigned mask = __ballot_sync(0xffffffffu, valid);
-        if (lane == 0) wcount[warp] = __popc(mask);
+#pragma unroll
+        for (int q = 0; q < CI; ++q) {
+            if (ef + q < e1) {
+                float3 v;
+                const float d = edge_distance(pos4[ii[q]], pos4[jj[q]], box, v);
+                if (d < rc && d > 0.f && (!HALF || jj[q] > ii[q])) vmask |= 1u << q;
+            }
+        }
+        // block-wide exclusive scan of the per-thread counts, edge order kept
+        const int cnt = __popc(vmask);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        if (lane == 31) wcount[warp] = incl;
         __syncthreads();
         if (warp == 0) {
-            int v = wcount[lane];
-            int incl = v;
+            const int nw = blockDim.x >> 5;
+            const int v = lane < nw ? wcount[lane] : 0;
+            int wi = v;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                int t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += t;
+                const int t = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += t;
             }
-            wcount[lane] = incl - v;
-            if (lane == 31) total_s = incl;
+            if (lane < nw) wcount[lane] = wi - v;
+            if (lane == 31) total_s = wi;
         }
         __syncthreads();
-        if (valid) {
-            const long long k = base + wcount[warp] + __popc(mask & ((1u << lane) - 1u));
-            crow[k] = i;
-            ccol[k] = j;
-            cidx[k] = (int32_t)e;
+        long long k = base + wcount[warp] + (incl - cnt);
+#pragma unroll
+        for (int q = 0; q < CI; ++q) {
+            if ((vmask >> q) & 1u) {
+                crow[k] = ii[q];
+                ccol[k] = jj[q];
+                cidx[k] = (int32_t)(ef + q);
+                ++k;
+            }
         }
         base += total_s;
         __syncthreads();
@@ -1099,8 +1139,20 @@ __global__ void __launch_bounds__(1024) k_compact(const int32_t* __restrict__ ro
 cudaError_t launch_compact(schnet_ctx* c)
 {
     Workspace& w = c->ws;
-    k_compact<<<c->ncta, 1024, 0, c->s>>>(w.row_ptr, w.part, w.erow, w.col, w.pos4, c->box, c->cfg.cutoff, c->cap,
-                                          w.meta, w.crow, w.ccol, w.cidx, w.ccount);
+    k_compact<false><<<c->ncta, 1024, 0, c->s>>>(w.row_ptr, w.part, w.erow, w.col, w.pos4, c->box, c->cfg.cutoff,
+                                                 c->cap, w.meta, w.crow, w.ccol, w.cidx, w.ccount);
+    c->launches += 1;
+    return cudaGetLastError();
+}
+
+// The half list (edges (i, j) with j > i and d < r_c) in the runs of its own row
+// partition, over the same arrays: it runs after the last launch that reads the
+// full compacted list of the step.
+cudaError_t launch_compact_half(schnet_ctx* c)
+{
+    Workspace& w = c->ws;
+    k_compact<true><<<c->ncta, 1024, 0, c->s>>>(w.row_ptr, w.part_h, w.erow, w.col, w.pos4, c->box, c->cfg.cutoff,
+                                                c->cap, w.meta, w.crow, w.ccol, w.cidx, w.ccount_h);
     c->launches += 1;
     return cudaGetLastError();
 }
@@ -1197,14 +1249,26 @@ static void launch_bwd(schnet_ctx* c, const MPArgs& a)
 }
 
 // Interaction 0's dE/dh feeds only the gradient with respect to the embedding,
-// which forces do not need: its launch computes s_e alone.
+// which forces do not need: its launch computes the pair derivatives alone, over
+// the half list in its own row partition.
 cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s)
 {
     MPArgs a = make_args(c, layer);
     a.out = c->ws.dh;
     a.accumulate_s = accumulate_s;
-    if (layer > 0) launch_bwd<true>(c, a);
-    else launch_bwd<false>(c, a);
+    if (layer > 0) {
+        launch_bwd<true>(c, a);
+    } else {
+        // the half list writes s_e of one edge per pair; with no later interaction to
+        // have set them, the other edges' s_e must read zero in the force assembly
+        if (!accumulate_s) {
+            cudaError_t e = cudaMemsetAsync(c->ws.s_edge, 0, sizeof(float) * (size_t)c->cap, c->s);
+            if (e != cudaSuccess) return e;
+        }
+        a.part = c->ws.part_h;
+        a.ccount = c->ws.ccount_h;
+        launch_bwd<false>(c, a);
+    }
     c->launches += 1;
     return cudaGetLastError();
 }

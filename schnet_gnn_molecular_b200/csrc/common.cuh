@@ -73,14 +73,19 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-// Shifted softplus in base 2 of two values: for p = x log2(e),
-// ssp2(p) = log2(1 + 2^p) - 1 = log2((1 + e^x) / 2) = ssp(x) / ln2.  Written as
-// max(p, 0) + log2(1/2 + 2^-|p| / 2): no overflow for any p, the logarithm's
-// argument lies in [1/2, 1], and the result has no constant offset (ssp2(0) = 0),
-// so the products that consume it accumulate no large common term.
-__device__ __forceinline__ float2 ssp2x2(float2 p)
+// Softplus in base 2 of two values, p = x log2(e).  SHIFT = true: the shifted
+// form ssp2(p) = log2(1 + 2^p) - 1 = log2((1 + e^x) / 2) = ssp(x) / ln2, written
+// max(p, 0) + log2(1/2 + 2^-|p| / 2); it has no constant offset (ssp2(0) = 0), so
+// the products that consume it accumulate no large common term.  SHIFT = false:
+// sp2(p) = log2(1 + 2^p) = max(p, 0) + log2(1 + 2^-|p|), which is near 0 rather
+// than near -1 for strongly negative x, the better choice for an operand rounded
+// once to 16 bits (the -1 then goes into the consumer's bias).  No overflow for
+// any p; the logarithm's argument lies in [1/2, 1] or [1, 2].
+template <bool SHIFT>
+__device__ __forceinline__ float2 sp2x2(float2 p)
 {
-    const float2 y = fma2(dup2(0.5f), make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y))), dup2(0.5f));
+    const float c = SHIFT ? 0.5f : 1.0f;
+    const float2 y = fma2(dup2(c), make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y))), dup2(c));
     return add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
 }
 
@@ -108,10 +113,12 @@ __device__ __forceinline__ float2 ex2_fma2(float2 x)
     return make_float2(__int_as_float(__float_as_int(p.x) + kx), __int_as_float(__float_as_int(p.y) + ky));
 }
 
-// ssp2x2 with its exponentials from ex2_fma2 (the logarithms stay on the MUFU)
-__device__ __forceinline__ float2 ssp2x2_fma(float2 p)
+// sp2x2 with its exponentials from ex2_fma2 (the logarithms stay on the MUFU)
+template <bool SHIFT>
+__device__ __forceinline__ float2 sp2x2_fma(float2 p)
 {
-    const float2 y = fma2(dup2(0.5f), ex2_fma2(make_float2(-fabsf(p.x), -fabsf(p.y))), dup2(0.5f));
+    const float c = SHIFT ? 0.5f : 1.0f;
+    const float2 y = fma2(dup2(c), ex2_fma2(make_float2(-fabsf(p.x), -fabsf(p.y))), dup2(c));
     return add2(make_float2(fmaxf(p.x, 0.0f), fmaxf(p.y, 0.0f)), make_float2(lg2_mufu(y.x), lg2_mufu(y.y)));
 }
 

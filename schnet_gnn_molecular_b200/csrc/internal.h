@@ -54,7 +54,7 @@ struct Workspace {
     // packed weights
     uint8_t* img;                 // [L][LAYER_IMG]
     float *s1, *s2, *b1;          // [L][FP] filter channel scales, first-layer bias
-    float* b2;                    // [L][FP] second-layer bias
+    float* b2;                    // [L][FP] second-layer bias (one 16-bit activation term: minus ln2 s2 sum_k W2^[k][f])
     float *emb;                   // [T][FP]
     float *emb_h0;                // [T][FP] emb W_in of interaction 0 (the first h of every atom of a type)
     uint8_t* aw_img;              // [6 L + 2][AW_IMG] atom-wise layers as tensor-core A operands
@@ -73,6 +73,8 @@ struct Workspace {
     int32_t *crow, *ccol, *cidx;  // [cap] edges with d < r_c, per CTA row range
     int32_t* ccount;              // [ncta]
     int32_t* part;                // [ncta+1]
+    int32_t* ccount_h;            // [ncta]    the half list (j > i): per-CTA edge counts
+    int32_t* part_h;              // [ncta+1]  and row partition (its runs reuse crow/ccol/cidx)
     // cell list
     int32_t *cell_of, *cell_atoms;       // [N]  caller order
     int32_t* cell_slot;                  // [N]  cell of each slot
@@ -168,6 +170,7 @@ cudaError_t launch_aw_fwd(schnet_ctx* c, int layer);
 cudaError_t launch_aw_bwd_top(schnet_ctx* c);
 cudaError_t launch_aw_bwd(schnet_ctx* c, int layer);
 cudaError_t launch_compact(schnet_ctx* c);
+cudaError_t launch_compact_half(schnet_ctx* c);
 cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer);
 cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s);
 cudaError_t cfconv_init_attributes();

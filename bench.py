@@ -330,10 +330,12 @@ def run_native(args):
         E_list, E_cut = _edge_stats(model, p.cpu().numpy(), w)
         peaks, src = _peaks()
         flop_fwd = 2.0 * (w.K * w.F + w.F * w.F) * E_cut
-        # backward: W and its derivative W' (twice the forward's contraction) per directed edge
-        # for interactions 1..L-1; per unordered pair (E_cut / 2, the half list) for interaction 0
-        bwd_edges = (w.L - 1 + 0.5) * E_cut
-        flop_bwd = 2.0 * 2.0 * (w.K * w.F + w.F * w.F) * bwd_edges / w.L     # per launch, averaged
+        # backward class, per step: for every interaction the pair derivatives, W and W' (twice
+        # the forward's contraction) per unordered pair (E_cut / 2, the half list); for
+        # interactions 1..L-1 dE/dh, the forward's contraction per directed edge.  L + (L - 1)
+        # launches, each one forward's worth on average.
+        n_bwd_launch = 2 * w.L - 1
+        flop_bwd = 2.0 * (w.K * w.F + w.F * w.F) * E_cut * (w.L + (w.L - 1)) / n_bwd_launch
         per_launch = {k: x[0] / max(x[1], 1) for k, x in prof.items()}
         per_step = {k: x[0] / n_rb for k, x in prof.items()}
         tot_ms = sum(x[0] for x in prof.values())
@@ -352,7 +354,8 @@ def run_native(args):
         n_aw = 6 * w.L                                    # atom-wise layer applications per step
         bounds = {
             "cfconv_fwd": max(w.L * flop_fwd / (peak * 1e12), w.L * mu["fwd"] * E_cut / mufu_peak),
-            "cfconv_bwd": max(w.L * flop_bwd / (peak * 1e12), mu["bwd"] * bwd_edges / mufu_peak),
+            "cfconv_bwd": max(n_bwd_launch * flop_bwd / (peak * 1e12),
+                              (w.L * mu["bwd"] * E_cut / 2 + (w.L - 1) * mu["fwd"] * E_cut) / mufu_peak),
             "atomwise": max(n_aw * 2.0 * w.F * w.F * w.n_atoms / (peak * 1e12),
                             n_aw * 2 * w.n_atoms * w.F * 4 / hbm),
             "forces": hb["forces"] / hbm, "integrate": hb["integrate"] / hbm, "mask": hb["mask"] / hbm,

@@ -154,6 +154,7 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.crow = cv.take<int32_t>(d.cap); w.ccol = cv.take<int32_t>(d.cap); w.cidx = cv.take<int32_t>(d.cap);
     w.ccount = cv.take<int32_t>(MAX_CTA);
     w.part = cv.take<int32_t>(MAX_CTA + 1);
+    w.crow_h = cv.take<int32_t>(d.cap); w.ccol_h = cv.take<int32_t>(d.cap); w.cidx_h = cv.take<int32_t>(d.cap);
     w.ccount_h = cv.take<int32_t>(MAX_CTA);
     w.part_h = cv.take<int32_t>(MAX_CTA + 1);
     w.cell_of = cv.take<int32_t>(N); w.cell_atoms = cv.take<int32_t>(N);
@@ -520,7 +521,7 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
         Timed t_(c, kind);                              \
         if ((e = (expr)) != cudaSuccess) return e;      \
     } while (0)
-    SCHNET_TIMED(SCHNET_KERNEL_MASK, launch_compact(c));
+    SCHNET_TIMED(SCHNET_KERNEL_MASK, launch_compact(c, need_forces));
     SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_embed(c, types));
     for (int l = 0; l < c->L; ++l) {
         SCHNET_TIMED(SCHNET_KERNEL_CFCONV_FWD, launch_cfconv_fwd(c, l));
@@ -531,12 +532,14 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
     if (!need_forces) return cudaSuccess;
     SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd_top(c));
     for (int l = c->L - 1; l >= 0; --l) {
-        // interaction 0 runs over the half list (one edge per unordered pair), which
-        // replaces the compacted runs of the later interactions' launches
-        if (l == 0) SCHNET_TIMED(SCHNET_KERNEL_MASK, launch_compact_half(c));
-        SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_bwd(c, l, l < c->L - 1 ? 1 : 0));
-        // interaction 0: dE/dx^0 is a gradient with respect to the embedding, not needed for forces
-        if (l > 0) SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd(c, l));
+        // pair derivatives over the half list (one edge per unordered pair)
+        SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_pair(c, l, l < c->L - 1 ? 1 : 0));
+        // dE/dh and the atom-wise backward carry the gradient to the earlier interactions;
+        // interaction 0's would only reach the embedding, which forces do not need
+        if (l > 0) {
+            SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_dh(c, l));
+            SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd(c, l));
+        }
     }
     SCHNET_TIMED(SCHNET_KERNEL_FORCES, launch_forces(c, forces));
 #undef SCHNET_TIMED

@@ -793,19 +793,18 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
     }
 }
 
-// DH = false: the pair derivative over the half list -- no dE/dh_j segment sums,
-// no merge.  Used for the first interaction, whose dE/dh feeds only the gradient
-// with respect to the embedding, which forces do not need; its forces need only
+// Backward of one interaction for the forces: the pair derivative
 // dE/dd_ij = D_ij = sum_f W'_f(d_ij) (u_i,f h_j,f + u_j,f h_i,f), the same for
-// (i, j) and (j, i) because W_ij = W_ji.  So the launch runs over one edge per
-// unordered pair (the edges (i, j) with j > i, in rows balanced by their own
-// partition) and adds D_ij to s_e of that edge alone; the force assembly sums
-// s_e + s_rev(e), so both atoms of the pair receive it.
-template <int FMT, int NW, int NX, bool DH>
+// (i, j) and (j, i) because W_ij = W_ji.  The launch runs over one edge per
+// unordered pair (the half list: edges (i, j) with j > i, in rows balanced by
+// their own partition) and writes (adds, for the later interactions' sums) D_ij
+// to s_e of that edge; the force assembly reads each pair's value from its
+// owning edge, so both atoms receive it.  dE/dh_j = sum_i u_i (.) W_ij is the
+// forward kernel's segment sum with u in place of h, launched separately.
+template <int FMT, int NW, int NX>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
     constexpr int TE = TE_B;
-    constexpr int NCH = TE / 32;
     using Meta = TileMeta<TE, true>;
     extern __shared__ __align__(1024) uint8_t smem[];
     Carry* cy = reinterpret_cast<Carry*>(smem + sm_carry<TE, true>());
@@ -828,10 +827,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     uint8_t* rbf = smem + SM_RBF + g * 2 * RBF_TERM;
     uint8_t* act = smem + SM_ACT + g * 2 * ACT_TERM;
     Meta* tmb = reinterpret_cast<Meta*>(smem + sm_meta<TE, true>() + g * 2 * sizeof(Meta));
-    float* pf_s = reinterpret_cast<float*>(act);    // after GEMM2: [chunk][feature] partials
-    float* pl_s = pf_s + NCH * 128;
-    float* ps_s = pl_s + NCH * 128;                 // [quadrant][edge] partial of s_e
-    // per-warp [32 edges][36] scratch of the s_e transpose (behind the partials, inside the
+    float* ps_s = reinterpret_cast<float*>(act);    // after GEMM2: [quadrant][edge] partial of D
+    // per-warp [32 edges][36] scratch of the D transpose (behind the partials, inside the
     // group's GEMM2 operand buffer, which is free between GEMM2's completion and the next E1)
     float* s_w = reinterpret_cast<float*>(act + 4096) + (warp & 7) * (32 * 36);
     const int col0 = ch * 32;
@@ -905,144 +902,109 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         gather<16>(h_f, tm->col, eb, hv);
         if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2(t) done
         pending = 0;
-        // epilogue 2: W = f_c z, W' = f_c' z + f_c z'  (z = s2 ln2 Q + b2, z' = s2 Q')
-        {
-            const bool active = eb < ne;
+        // epilogue 2: W' = f_c' z + f_c z' (z = s2 ln2 Q + b2, z' = s2 Q'), and per edge the
+        // pair derivative D = sum_f W'_f (u_i,f h_j,f + u_j,f h_i,f)
+        if (eb < ne) {
             const ChunkInfo ci = tm->c[ch];
-            // 1: one row in the chunk; 2: two rows (the first a prefix); 3: the general
-            // serial segmented sum with a row change test per edge
-            const int kind = !active ? 0 : ci.other ? 3 : (ci.rfirst == ci.rlast ? 1 : 2);
-            float pf = 0.f, pl = 0.f;
-            if (kind != 0) {
-                const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
-                const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
-                // half list: the row atom's own h_i for the reverse direction's term u_j h_i
-                const float h_first = DH ? 0.f : __ldg(h_f + (size_t)ci.rfirst * FP);
-                const float h_last = DH ? 0.f : __ldg(h_f + (size_t)ci.rlast * FP);
-                float h_row = h_first;
-                float sf = 0.f, sl = 0.f;
-                ChunkSeg c;
-                seg_begin(c, ci.rfirst);
-                float u_row = u_first;
+            // 1: one row in the chunk; 2: two rows (the first a prefix); 3: a third row occurs,
+            // rows read per edge
+            const int kind = ci.other ? 3 : (ci.rfirst == ci.rlast ? 1 : 2);
+            const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
+            const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
+            const float h_first = __ldg(h_f + (size_t)ci.rfirst * FP);
+            const float h_last = __ldg(h_f + (size_t)ci.rlast * FP);
+            int lrow = ci.rfirst;
+            float u_row = u_first, h_row = h_first;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    if (hh == 1) {
-                        gather<16>(u_f, tm->col, eb + 16, uv);
-                        gather<16>(h_f, tm->col, eb + 16, hv);
-                    }
-                    float r[16], rd[16];
-                    tmem_ld16(tP + hh * 16, r);          // Q
-                    tmem_ld16(tPd + hh * 16, rd);        // Q'
-                    tmem_ld_wait();
-                    const float* fcp = tm->fc + eb + hh * 16;
-                    const float* dfcp = tm->dfc + eb + hh * 16;
-                    if (kind == 1) {
-#pragma unroll
-                        for (int gq = 0; gq < 16; gq += 4) {
-                            float fc[4], dfc[4];
-                            load_edges<4>(fcp, gq, fc);
-                            load_edges<4>(dfcp, gq, dfc);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int q = gq + i;
-                                const float z = fmaf(s2L, r[q], b2);
-                                if (DH) sf = fmaf(fc[i] * z, uv[q], sf);
-                                const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
-                                rd[q] = DH ? wd * (u_first * hv[q]) : wd * fmaf(uv[q], h_first, u_first * hv[q]);
-                            }
-                        }
-                    } else if (kind == 2) {
-#pragma unroll
-                        for (int gq = 0; gq < 16; gq += 4) {
-                            float fc[4], dfc[4];
-                            load_edges<4>(fcp, gq, fc);
-                            load_edges<4>(dfcp, gq, dfc);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int q = gq + i;
-                                const float z = fmaf(s2L, r[q], b2);
-                                const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
-                                if (DH) {
-                                    const float dt = fc[i] * z * uv[q];
-                                    sf += first ? dt : 0.f;
-                                    sl += first ? 0.f : dt;
-                                }
-                                const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
-                                const float ui = first ? u_first : u_last;
-                                rd[q] = DH ? wd * (ui * hv[q]) : wd * fmaf(uv[q], first ? h_first : h_last, ui * hv[q]);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const int e = eb + hh * 16 + q;
-                            float tval = 0.f;
-                            if (e < ne) {
-                                const int row = __ldg(rows_g + e);
-                                if (row != c.lrow) {
-                                    if (DH) seg_row(c, row, a.out, f);
-                                    else c.lrow = row;
-                                    u_row = __ldg(u_f + (size_t)row * FP);
-                                    if (!DH) h_row = __ldg(h_f + (size_t)row * FP);
-                                }
-                                const float fcq = fcp[q], dfcq = dfcp[q];
-                                const float z = fmaf(s2L, r[q], b2);
-                                const float wd = fmaf(dfcq, z, fcq * (s2 * rd[q]));
-                                if (DH) c.acc = fmaf(fcq * z, uv[q], c.acc);
-                                tval = DH ? wd * (u_row * hv[q]) : wd * fmaf(uv[q], h_row, u_row * hv[q]);
-                            }
-                            rd[q] = tval;
-                        }
-                    }
-                    // stage this half's 16 per-edge values as S[edge][feature lane] (row stride 36:
-                    // the stores and the 16-byte row reads below are free of bank conflicts)
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) s_w[(hh * 16 + q) * 36 + lane] = rd[q];
+            for (int hh = 0; hh < 2; ++hh) {
+                if (hh == 1) {
+                    gather<16>(u_f, tm->col, eb + 16, uv);
+                    gather<16>(h_f, tm->col, eb + 16, hv);
                 }
-                // lane k sums edge k of the warp's chunk over the warp's 32 features (the same
-                // pairwise tree as a butterfly over the lanes)
-                __syncwarp();
-                {
-                    float v[32];
+                float r[16], rd[16];
+                tmem_ld16(tP + hh * 16, r);          // Q
+                tmem_ld16(tPd + hh * 16, rd);        // Q'
+                tmem_ld_wait();
+                const float* fcp = tm->fc + eb + hh * 16;
+                const float* dfcp = tm->dfc + eb + hh * 16;
+                if (kind == 1) {
 #pragma unroll
-                    for (int c4 = 0; c4 < 8; ++c4) {
-                        const float4 x = *reinterpret_cast<const float4*>(s_w + lane * 36 + c4 * 4);
-                        v[4 * c4] = x.x; v[4 * c4 + 1] = x.y; v[4 * c4 + 2] = x.z; v[4 * c4 + 3] = x.w;
+                    for (int gq = 0; gq < 16; gq += 4) {
+                        float fc[4], dfc[4];
+                        load_edges<4>(fcp, gq, fc);
+                        load_edges<4>(dfcp, gq, dfc);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int q = gq + i;
+                            const float z = fmaf(s2L, r[q], b2);
+                            const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
+                            rd[q] = wd * fmaf(uv[q], h_first, u_first * hv[q]);
+                        }
                     }
-                    ps_s[qd * TE + eb + lane] = tree_sum<32>(v);
-                }
-                __syncwarp();
-                if (!DH) {
-                } else if (kind == 1) {
-                    pf = sf;
                 } else if (kind == 2) {
-                    pf = sf;
-                    pl = sl;
-                    for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
-                } else if (c.lrow == c.rfirst) {
-                    pf = c.acc;
+#pragma unroll
+                    for (int gq = 0; gq < 16; gq += 4) {
+                        float fc[4], dfc[4];
+                        load_edges<4>(fcp, gq, fc);
+                        load_edges<4>(dfcp, gq, dfc);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int q = gq + i;
+                            const float z = fmaf(s2L, r[q], b2);
+                            const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
+                            const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
+                            rd[q] = wd * fmaf(uv[q], first ? h_first : h_last, (first ? u_first : u_last) * hv[q]);
+                        }
+                    }
                 } else {
-                    pf = c.pf;
-                    pl = c.acc;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        const int e = eb + hh * 16 + q;
+                        float tval = 0.f;
+                        if (e < ne) {
+                            const int row = __ldg(rows_g + e);
+                            if (row != lrow) {
+                                lrow = row;
+                                u_row = __ldg(u_f + (size_t)row * FP);
+                                h_row = __ldg(h_f + (size_t)row * FP);
+                            }
+                            const float z = fmaf(s2L, r[q], b2);
+                            const float wd = fmaf(dfcp[q], z, fcp[q] * (s2 * rd[q]));
+                            tval = wd * fmaf(uv[q], h_row, u_row * hv[q]);
+                        }
+                        rd[q] = tval;
+                    }
                 }
+                // stage this half's 16 per-edge values as S[edge][feature lane] (row stride 36:
+                // the stores and the 16-byte row reads below are free of bank conflicts)
+#pragma unroll
+                for (int q = 0; q < 16; ++q) s_w[(hh * 16 + q) * 36 + lane] = rd[q];
             }
-            if (DH) {
-                pf_s[ch * 128 + f] = pf;
-                pl_s[ch * 128 + f] = pl;
+            // lane k sums edge k of the warp's chunk over the warp's 32 features (the same
+            // pairwise tree as a butterfly over the lanes)
+            __syncwarp();
+            {
+                float v[32];
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4) {
+                    const float4 x = *reinterpret_cast<const float4*>(s_w + lane * 36 + c4 * 4);
+                    v[4 * c4] = x.x; v[4 * c4 + 1] = x.y; v[4 * c4 + 2] = x.z; v[4 * c4 + 3] = x.w;
+                }
+                ps_s[qd * TE + eb + lane] = tree_sum<32>(v);
             }
+            __syncwarp();
         }
         tc_fence_before();
-        group_sync(g);          // Q, Q' read out; partials and the next tile's Gaussians in place
-        // GEMM1(t+2) is issued by warp 4, which takes no part in the merge below (an issuing
-        // thread blocks while the tensor core's queue is full)
+        group_sync(g);          // Q, Q' read out; per-edge partials and the next tile's Gaussians in place
+        // GEMM1(t+2) is issued by warp 4, which does not write s_e below (an issuing thread
+        // blocks while the tensor core's queue is full)
         if (next && mt == 128) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
         if (mt < ne) {
             const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];
             a.s_edge[my_g] = a.accumulate_s ? my_so + sv : sv;
         }
-        if (DH && !(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
-        group_sync(g);          // merge and s_e done with the partials before E1 of the next tile overwrites them
+        group_sync(g);          // s_e done with the partials before E1 of the next tile overwrites them
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
     if (mt == 0) {
@@ -1050,24 +1012,36 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         pend_s[g] = ok ? 0u : pending;
     }
     const bool all_ok = __syncthreads_or(!ok) == 0;
-    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, DH);
+    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, false);
 }
 
 // ---------------------------------------------------------------------------
-// cutoff masking: per CTA row range, the listed edges with d < r_c, in order
+// cutoff masking: per CTA row range, the listed edges with d < r_c, in order;
+// list 1 (the half list) keeps only the edges (i, j) with j > i, in the row
+// ranges of its own partition.  One launch builds both lists (CTAs ncta ..
+// 2 ncta - 1 take the half list), so the two passes share the GPU.
 // ---------------------------------------------------------------------------
-template <bool HALF>
-__global__ void __launch_bounds__(1024) k_compact(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ part,
+struct CompactList {
+    const int32_t* part;
+    int32_t *crow, *ccol, *cidx, *ccount;
+};
+
+__global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__ row_ptr, int ncta,
                                                   const int32_t* __restrict__ erow, const int32_t* __restrict__ col,
                                                   const float4* __restrict__ pos4, Box box, float rc, long long cap,
-                                                  const DevMeta* meta, int32_t* __restrict__ crow,
-                                                  int32_t* __restrict__ ccol, int32_t* __restrict__ cidx,
-                                                  int32_t* __restrict__ ccount)
+                                                  const DevMeta* meta, CompactList full, CompactList half)
 {
+    const bool is_half = (int)blockIdx.x >= ncta;
+    const CompactList L = is_half ? half : full;
+    int32_t* __restrict__ crow = L.crow;
+    int32_t* __restrict__ ccol = L.ccol;
+    int32_t* __restrict__ cidx = L.cidx;
+    int32_t* __restrict__ ccount = L.ccount;
+    const int32_t* __restrict__ part = L.part;
     constexpr int CI = 4;             // consecutive edges per thread and pass
     __shared__ int wcount[32];
     __shared__ int total_s;
-    const int c = blockIdx.x;
+    const int c = is_half ? (int)blockIdx.x - ncta : (int)blockIdx.x;
     const int r0 = part[c], r1 = part[c + 1];
     if (meta->n_edges > cap || r0 >= r1) {
         if (threadIdx.x == 0) ccount[c] = 0;
@@ -1094,7 +1068,7 @@ __global__ void __launch_bounds__(1024) k_compact(const int32_t* __restrict__ ro
             if (ef + q < e1) {
                 float3 v;
                 const float d = edge_distance(pos4[ii[q]], pos4[jj[q]], box, v);
-                if (d < rc && d > 0.f && (!HALF || jj[q] > ii[q])) vmask |= 1u << q;
+                if (d < rc && d > 0.f && (!is_half || jj[q] > ii[q])) vmask |= 1u << q;
             }
         }
         // block-wide exclusive scan of the per-thread counts, edge order kept
@@ -1136,23 +1110,15 @@ __global__ void __launch_bounds__(1024) k_compact(const int32_t* __restrict__ ro
     if (threadIdx.x == 0) ccount[c] = (int32_t)(base - e0);
 }
 
-cudaError_t launch_compact(schnet_ctx* c)
+// The full list of the step's edges inside the cutoff and, when forces follow, the
+// half list of the pair-derivative launches
+cudaError_t launch_compact(schnet_ctx* c, bool with_half)
 {
     Workspace& w = c->ws;
-    k_compact<false><<<c->ncta, 1024, 0, c->s>>>(w.row_ptr, w.part, w.erow, w.col, w.pos4, c->box, c->cfg.cutoff,
-                                                 c->cap, w.meta, w.crow, w.ccol, w.cidx, w.ccount);
-    c->launches += 1;
-    return cudaGetLastError();
-}
-
-// The half list (edges (i, j) with j > i and d < r_c) in the runs of its own row
-// partition, over the same arrays: it runs after the last launch that reads the
-// full compacted list of the step.
-cudaError_t launch_compact_half(schnet_ctx* c)
-{
-    Workspace& w = c->ws;
-    k_compact<true><<<c->ncta, 1024, 0, c->s>>>(w.row_ptr, w.part_h, w.erow, w.col, w.pos4, c->box, c->cfg.cutoff,
-                                                c->cap, w.meta, w.crow, w.ccol, w.cidx, w.ccount_h);
+    const CompactList full{w.part, w.crow, w.ccol, w.cidx, w.ccount};
+    const CompactList half{w.part_h, w.crow_h, w.ccol_h, w.cidx_h, w.ccount_h};
+    k_compact<<<c->ncta * (with_half ? 2 : 1), 1024, 0, c->s>>>(w.row_ptr, c->ncta, w.erow, w.col, w.pos4, c->box,
+                                                                c->cfg.cutoff, c->cap, w.meta, full, half);
     c->launches += 1;
     return cudaGetLastError();
 }
@@ -1199,10 +1165,7 @@ static cudaError_t set_attrs()
     cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_bytes<TE_F, false>());
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_bytes<TE_B, true>());
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_bytes<TE_B, true>());
 }
 
@@ -1217,10 +1180,8 @@ cudaError_t cfconv_init_attributes()
 
 // operand formats: fp32 weights (fp16 hi+lo weights and activations), fp16 or bf16
 // weights (one weight term, hi+lo activations), fp16 weights with fp16 activations
-cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
+static void launch_fwd(schnet_ctx* c, const MPArgs& a)
 {
-    MPArgs a = make_args(c, layer);
-    a.out = c->ws.m;
     const size_t sm = smem_bytes<TE_F, false>();
     if (c->n_xterms == 1)
         k_cfconv_fwd<0, 1, 1><<<c->ncta, NT, sm, c->s>>>(a);
@@ -1230,45 +1191,50 @@ cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
         k_cfconv_fwd<0, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
     else
         k_cfconv_fwd<1, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
+}
+
+// m = sum_j h_j (.) W_ij of interaction `layer`
+cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
+{
+    MPArgs a = make_args(c, layer);
+    a.out = c->ws.m;
+    launch_fwd(c, a);
     c->launches += 1;
     return cudaGetLastError();
 }
 
-template <bool DH>
-static void launch_bwd(schnet_ctx* c, const MPArgs& a)
-{
-    const size_t sm = smem_bytes<TE_B, true>();
-    if (c->n_xterms == 1)
-        k_cfconv_bwd<0, 1, 1, DH><<<c->ncta, NT, sm, c->s>>>(a);
-    else if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_bwd<0, 2, 2, DH><<<c->ncta, NT, sm, c->s>>>(a);
-    else if (c->weight_fmt == 0)
-        k_cfconv_bwd<0, 1, 2, DH><<<c->ncta, NT, sm, c->s>>>(a);
-    else
-        k_cfconv_bwd<1, 1, 2, DH><<<c->ncta, NT, sm, c->s>>>(a);
-}
-
-// Interaction 0's dE/dh feeds only the gradient with respect to the embedding,
-// which forces do not need: its launch computes the pair derivatives alone, over
-// the half list in its own row partition.
-cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s)
+// dE/dh_j = sum_i u_i (.) W_ij with u = dE/dm of interaction `layer`: the same
+// segment sum over the symmetric list, with u gathered in place of h
+cudaError_t launch_cfconv_dh(schnet_ctx* c, int layer)
 {
     MPArgs a = make_args(c, layer);
+    a.h = c->ws.m;
     a.out = c->ws.dh;
+    launch_fwd(c, a);
+    c->launches += 1;
+    return cudaGetLastError();
+}
+
+// Pair derivatives of interaction `layer` over the half list, written to s_e of
+// each pair's owning edge (added to the later interactions' when accumulate_s)
+cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s)
+{
+    MPArgs a = make_args(c, layer);
+    a.crow = c->ws.crow_h;
+    a.ccol = c->ws.ccol_h;
+    a.cidx = c->ws.cidx_h;
+    a.ccount = c->ws.ccount_h;
+    a.part = c->ws.part_h;
     a.accumulate_s = accumulate_s;
-    if (layer > 0) {
-        launch_bwd<true>(c, a);
-    } else {
-        // the half list writes s_e of one edge per pair; with no later interaction to
-        // have set them, the other edges' s_e must read zero in the force assembly
-        if (!accumulate_s) {
-            cudaError_t e = cudaMemsetAsync(c->ws.s_edge, 0, sizeof(float) * (size_t)c->cap, c->s);
-            if (e != cudaSuccess) return e;
-        }
-        a.part = c->ws.part_h;
-        a.ccount = c->ws.ccount_h;
-        launch_bwd<false>(c, a);
-    }
+    const size_t sm = smem_bytes<TE_B, true>();
+    if (c->n_xterms == 1)
+        k_cfconv_bwd<0, 1, 1><<<c->ncta, NT, sm, c->s>>>(a);
+    else if (c->weight_fmt == 0 && c->n_wterms == 2)
+        k_cfconv_bwd<0, 2, 2><<<c->ncta, NT, sm, c->s>>>(a);
+    else if (c->weight_fmt == 0)
+        k_cfconv_bwd<0, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
+    else
+        k_cfconv_bwd<1, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
     c->launches += 1;
     return cudaGetLastError();
 }

@@ -1,13 +1,13 @@
 // Forces from the per-edge scalars of the backward pass, and the Langevin /
 // velocity-Verlet update of many replicas at once.
 //
-// Forces: the backward kernels leave s_e = sum_f W'_e,f u_i,f h_j,f for every
-// directed edge e = (i, j) of every interaction (summed over interactions);
-// the pair derivative dE/dd_ij is s_e + s_rev(e), and
-// F_i = sum_{e in row i} (s_e + s_rev(e)) (r_j - r_i) / d_ij  -- a per-row
-// segment sum over the CSR and its transpose map, no atomics (FlashSchNet
-// paper-curation summary, How: contention-free accumulation forward and
-// backward).
+// Forces: the backward kernels leave, on the owning edge e = (i, j), j > i, of
+// every pair within the cutoff, its derivative dE/dd_ij summed over the
+// interactions (the half list visits each pair once); and
+// F_i = sum_{e in row i} dE/dd_ij (r_j - r_i) / d_ij, with the value read from
+// e or from its transpose rev(e) -- a per-row segment sum over the CSR, no
+// atomics (FlashSchNet paper-curation summary, How: contention-free
+// accumulation forward and backward).
 // Rows are slots (atoms in cell order); perm maps a slot to the caller's
 // index, under which forces are stored for the integrator and the caller.
 // Integrator (the pages name Langevin / velocity-Verlet dynamics but give no
@@ -40,8 +40,9 @@ __global__ void k_forces(int n, const int32_t* __restrict__ row_ptr, const int32
             float3 v;
             const float d = edge_distance(pi, pos4[j], box, v);
             if (d < rc && d > 0.f) {
+                // the pair's derivative sits on its owning edge (i, j) with j > i
                 const int re = rev[e];
-                float D = s_edge[e] + (re >= 0 ? s_edge[re] : 0.f);
+                const float D = j > i ? s_edge[e] : (re >= 0 ? s_edge[re] : 0.f);
                 float k = D / d;
                 fx = fmaf(k, v.x, fx);
                 fy = fmaf(k, v.y, fy);

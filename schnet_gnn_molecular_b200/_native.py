@@ -21,7 +21,8 @@ EXPORTED = ["schnet_workspace_bytes", "schnet_create", "schnet_build_neighbors",
             "schnet_step", "schnet_step_host", "schnet_get_status", "schnet_last_error", "schnet_destroy",
             "schnet_get_neighbors", "schnet_get_atom_energies", "schnet_kernel_launches", "schnet_profile_steps",
             "schnet_build_neighbors_noalloc", "schnet_test_exp2", "schnet_test_timeout"]
-KERNEL_CLASSES = ["cfconv_fwd", "cfconv_bwd", "atomwise", "neighbors", "forces", "integrate", "reduce", "mask"]
+KERNEL_CLASSES = ["cfconv_fwd", "cfconv_bwd", "atomwise", "neighbors", "forces", "integrate", "reduce", "mask",
+                  "cfconv_dh"]
 
 
 class Config(C.Structure):

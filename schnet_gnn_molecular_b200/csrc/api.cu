@@ -537,7 +537,7 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
         // dE/dh and the atom-wise backward carry the gradient to the earlier interactions;
         // interaction 0's would only reach the embedding, which forces do not need
         if (l > 0) {
-            SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_dh(c, l));
+            SCHNET_TIMED(SCHNET_KERNEL_CFCONV_DH, launch_cfconv_dh(c, l));
             SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd(c, l));
         }
     }

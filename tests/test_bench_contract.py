@@ -51,14 +51,14 @@ def test_traffic_figure_is_keyed_to_the_kernel_sources(tmp_path, monkeypatch):
     os.makedirs(tmp_path / "profiles")
     json.dump(rec, open(tmp_path / "profiles" / "traffic.json", "w"))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    assert bench._traffic("cfconv_bwd") == d["cfconv_bwd"]
+    assert bench._traffic("k_cfconv_bwd") == d["k_cfconv_bwd"]
     with open(tmp_path / d["sources"][0], "a") as f:
         f.write("\n// edited\n")
-    assert bench._traffic("cfconv_bwd") is None
+    assert bench._traffic("k_cfconv_bwd") is None
     # and the committed record is honoured only if it matches the committed sources
     monkeypatch.setattr(bench, "ROOT", ROOT)
     h = hashlib.sha256()
     for src in d["sources"]:
         h.update(open(os.path.join(ROOT, src), "rb").read())
     current = h.hexdigest()[:16] == d["sources_sha256_16"]
-    assert (bench._traffic("cfconv_bwd") is not None) == current
+    assert (bench._traffic("k_cfconv_bwd") is not None) == current

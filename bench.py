@@ -165,6 +165,10 @@ def _workload(name):
         return workloads.sweep(int(name[len("cg_protein_"):-len("x269")]))
     if name.startswith("cg_globule_"):
         return workloads.globule(int(name[len("cg_globule_"):]))
+    if name.startswith("periodic_box_") and name[len("periodic_box_"):].isdigit():
+        # the 10^6-bead box's model and density, n beads
+        n = int(name[len("periodic_box_"):])
+        return workloads.BOX1M.with_(name=name, beads=n, box=(n / workloads.BOX1M.density) ** (1.0 / 3.0))
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -644,7 +648,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--nve-drift", action="store_true", help="measure NVE energy drift instead of throughput")
     ap.add_argument("--drift-steps", type=int, default=10000)
-    ap.add_argument("--drift-window", type=int, default=500)
+    ap.add_argument("--drift-window", type=int, default=100)
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
     const int qd = warp & 3, c = warp >> 2;
     const int f = qd * 32 + lane;                    // this thread's feature (output row / next K index)
 
+    pdl_trigger();
     if (warp == 0) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
@@ -155,6 +156,7 @@ __global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
     float sc[3];
 #pragma unroll
     for (int s = 0; s < 3; ++s) sc[s] = s < a.ngemm ? a.sc[s][f] : 0.f;
+    pdl_wait();                                      // the previous kernel's results from here on
     uint32_t phase = 0;
     bool ok = true;
 
@@ -280,6 +282,8 @@ __global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
 __global__ void k_chunk_sums(const float* __restrict__ v, const int32_t* __restrict__ lo,
                              const int32_t* __restrict__ hi, double* __restrict__ partial)
 {
+    pdl_trigger();
+    pdl_wait();
     int c = blockIdx.x;
     double s = 0.0;
     for (int i = lo[c] + threadIdx.x; i < hi[c]; i += blockDim.x) s += (double)v[i];
@@ -297,6 +301,8 @@ __global__ void k_chunk_sums(const float* __restrict__ v, const int32_t* __restr
 __global__ void k_replica_sums(int R, const int32_t* __restrict__ chunk_rep, int nchunk,
                                const double* __restrict__ partial, double* __restrict__ out, DevMeta* meta)
 {
+    pdl_trigger();
+    pdl_wait();
     int r = blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= R) return;
     // chunks of replica r are contiguous; find them by scanning the (small) table
@@ -364,6 +370,8 @@ __global__ void k_embed(int n, int T, const int32_t* __restrict__ types, const i
                         const float4* __restrict__ emb, const float4* __restrict__ emb_h0, float4* __restrict__ x,
                         float4* __restrict__ h, DevMeta* meta)
 {
+    pdl_trigger();
+    pdl_wait();
     const int k = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (k >= n) return;
@@ -381,41 +389,40 @@ cudaError_t launch_embed(schnet_ctx* c, const int32_t* types)
     Workspace& w = c->ws;
     static_assert(FP == 128, "one float4 per lane covers a padded feature row");
     const long long threads = (long long)c->N * 32;
-    k_embed<<<(unsigned)((threads + 255) / 256), 256, 0, c->s>>>(
-        c->N, c->T, types, w.perm, reinterpret_cast<const float4*>(w.emb), reinterpret_cast<const float4*>(w.emb_h0),
-        reinterpret_cast<float4*>(w.x), reinterpret_cast<float4*>(w.h), w.meta);
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_pdl(k_embed, (unsigned)((threads + 255) / 256), 256, 0, c->s, c->N, c->T, types,
+                      (const int32_t*)w.perm, reinterpret_cast<const float4*>(w.emb),
+                      reinterpret_cast<const float4*>(w.emb_h0), reinterpret_cast<float4*>(w.x),
+                      reinterpret_cast<float4*>(w.h), w.meta);
 }
 
 cudaError_t launch_aw_fwd(schnet_ctx* c, int layer)
 {
-    k_atomwise<AW_FWD><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, AW_FWD, layer));
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_pdl(k_atomwise<AW_FWD>, aw_grid(c), AWT, AW_SMEM, c->s, aw_args(c, AW_FWD, layer));
 }
 
 cudaError_t launch_aw_bwd_top(schnet_ctx* c)
 {
-    k_atomwise<AW_TOP><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, AW_TOP, c->L - 1));
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_pdl(k_atomwise<AW_TOP>, aw_grid(c), AWT, AW_SMEM, c->s, aw_args(c, AW_TOP, c->L - 1));
 }
 
 cudaError_t launch_aw_bwd(schnet_ctx* c, int layer)
 {
-    k_atomwise<AW_BWD><<<aw_grid(c), AWT, AW_SMEM, c->s>>>(aw_args(c, AW_BWD, layer));
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_pdl(k_atomwise<AW_BWD>, aw_grid(c), AWT, AW_SMEM, c->s, aw_args(c, AW_BWD, layer));
 }
 
 cudaError_t launch_replica_sum(schnet_ctx* c, const float* v, double* out)
 {
     Workspace& w = c->ws;
-    k_chunk_sums<<<c->nchunk, 256, 0, c->s>>>(v, w.chunk_lo, w.chunk_hi, w.partial);
-    k_replica_sums<<<(c->R + 127) / 128, 128, 0, c->s>>>(c->R, w.chunk_rep, c->nchunk, w.partial, out, w.meta);
     c->launches += 2;
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(k_chunk_sums, c->nchunk, 256, 0, c->s, v, (const int32_t*)w.chunk_lo,
+                               (const int32_t*)w.chunk_hi, w.partial);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(k_replica_sums, (c->R + 127) / 128, 128, 0, c->s, c->R, (const int32_t*)w.chunk_rep,
+                      c->nchunk, (const double*)w.partial, out, w.meta);
 }
 
 }  // namespace schnet

@@ -498,10 +498,11 @@ __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_
     if (c.lrow == c.rfirst) { pf = c.acc; pl = 0.f; } else { pf = c.pf; pl = c.acc; }
 }
 
-// Common prologue of both kernels: TMEM allocation, mbarriers, the filter
-// weights into TMEM (warps 0-3, one output channel per lane), the initial
-// carry.  Returns the TMEM base address.
-__device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslot, uint64_t* bars, Carry* cy, int r0)
+// Common prologue of both kernels, on constant data only (it runs before
+// pdl_wait): TMEM allocation, mbarriers, the filter weights into TMEM (warps
+// 0-3, one output channel per lane), the zero carry.  Returns the TMEM base
+// address.
+__device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslot, uint64_t* bars, Carry* cy)
 {
     const int warp = threadIdx.x >> 5;
     if (warp == 0) {
@@ -514,7 +515,6 @@ __device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslo
         mbar_init(&bars[2], 128);    // merge token: the 128 merging threads of a tile
         mbar_init(&bars[3], 1);      // group 1 start
         fence_mbar_init();
-        cy->cur[1] = r0;             // tile 0 reads the carry of "tile -1"
     }
     if (threadIdx.x < FP) cy->acc[threadIdx.x] = 0.f;
     tc_fence_before();
@@ -536,6 +536,29 @@ __device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslo
     __syncthreads();
     tc_fence_after();
     return tmem;
+}
+
+// After pdl_wait: this CTA's row range [r0, r1) (empty when the list overflowed
+// its capacity); a CTA without rows releases its tensor memory and returns false.
+__device__ __forceinline__ bool kernel_rows(const MPArgs& a, uint32_t tmem, Carry* cy, int& r0, int& r1)
+{
+    r0 = r1 = 0;
+    if (a.meta->n_edges <= a.cap) {
+        r0 = a.part[blockIdx.x];
+        r1 = a.part[blockIdx.x + 1];
+    }
+    if (r0 >= r1) {
+        tc_fence_before();
+        __syncthreads();
+        if ((threadIdx.x >> 5) == 0) {
+            tc_fence_after();
+            tmem_dealloc(tmem, 512);
+        }
+        return false;
+    }
+    if (threadIdx.x == 0) cy->cur[1] = r0;   // tile 0 reads the carry of "tile -1"
+    __syncthreads();
+    return true;
 }
 
 // Common epilogue: the carried row is complete; rows after it without edges are zero
@@ -643,17 +666,18 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     uint32_t* phases_s = tslot + 1;
     uint32_t* pend_s = tslot + 3;
 
-    if (a.meta->n_edges > a.cap) return;
-    const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
-    if (r0 >= r1) return;
-    const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = warp >> 3;                        // math group
     const int mt = threadIdx.x & (GT - 1);          // thread within the group
     const int qd = warp & 3, ch = (warp >> 2) & 1;  // TMEM lane quadrant, 64-edge half of the tile
     const int f = qd * 32 + lane;                   // this thread's output feature
 
-    const uint32_t tmem = kernel_setup(a, tslot, bars, cy, r0);
+    pdl_trigger();
+    const uint32_t tmem = kernel_setup(a, tslot, bars, cy);
+    pdl_wait();                                     // the previous kernel's results from here on
+    int r0, r1;
+    if (!kernel_rows(a, tmem, cy, r0, r1)) return;
+    const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     uint8_t* rbf = smem + SM_RBF + g * 2 * RBF_TERM;
     uint8_t* act = smem + SM_ACT + g * 2 * ACT_TERM;
     Meta* tmb = reinterpret_cast<Meta*>(smem + sm_meta<TE, false>() + g * 2 * sizeof(Meta));
@@ -813,17 +837,18 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     uint32_t* phases_s = tslot + 1;
     uint32_t* pend_s = tslot + 3;
 
-    if (a.meta->n_edges > a.cap) return;
-    const int r0 = a.part[blockIdx.x], r1 = a.part[blockIdx.x + 1];
-    if (r0 >= r1) return;
-    const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = warp >> 3;
     const int mt = threadIdx.x & (GT - 1);
     const int qd = warp & 3, ch = (warp >> 2) & 1;  // TMEM lane quadrant, 32-edge chunk of the tile
     const int f = qd * 32 + lane;
 
-    const uint32_t tmem = kernel_setup(a, tslot, bars, cy, r0);
+    pdl_trigger();
+    const uint32_t tmem = kernel_setup(a, tslot, bars, cy);
+    pdl_wait();                                     // the previous kernel's results from here on
+    int r0, r1;
+    if (!kernel_rows(a, tmem, cy, r0, r1)) return;
+    const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     uint8_t* rbf = smem + SM_RBF + g * 2 * RBF_TERM;
     uint8_t* act = smem + SM_ACT + g * 2 * ACT_TERM;
     Meta* tmb = reinterpret_cast<Meta*>(smem + sm_meta<TE, true>() + g * 2 * sizeof(Meta));
@@ -1031,6 +1056,8 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
                                                   const float4* __restrict__ pos4, Box box, float rc, long long cap,
                                                   const DevMeta* meta, CompactList full, CompactList half)
 {
+    pdl_trigger();
+    pdl_wait();
     const bool is_half = (int)blockIdx.x >= ncta;
     const CompactList L = is_half ? half : full;
     int32_t* __restrict__ crow = L.crow;
@@ -1117,10 +1144,10 @@ cudaError_t launch_compact(schnet_ctx* c, bool with_half)
     Workspace& w = c->ws;
     const CompactList full{w.part, w.crow, w.ccol, w.cidx, w.ccount};
     const CompactList half{w.part_h, w.crow_h, w.ccol_h, w.cidx_h, w.ccount_h};
-    k_compact<<<c->ncta * (with_half ? 2 : 1), 1024, 0, c->s>>>(w.row_ptr, c->ncta, w.erow, w.col, w.pos4, c->box,
-                                                                c->cfg.cutoff, c->cap, w.meta, full, half);
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_pdl(k_compact, c->ncta * (with_half ? 2 : 1), 1024, 0, c->s, (const int32_t*)w.row_ptr,
+                      (int)c->ncta, (const int32_t*)w.erow, (const int32_t*)w.col, (const float4*)w.pos4, c->box,
+                      c->cfg.cutoff, (long long)c->cap, (const DevMeta*)w.meta, full, half);
 }
 
 // ---------------------------------------------------------------------------
@@ -1180,17 +1207,17 @@ cudaError_t cfconv_init_attributes()
 
 // operand formats: fp32 weights (fp16 hi+lo weights and activations), fp16 or bf16
 // weights (one weight term, hi+lo activations), fp16 weights with fp16 activations
-static void launch_fwd(schnet_ctx* c, const MPArgs& a)
+static cudaError_t launch_fwd(schnet_ctx* c, const MPArgs& a)
 {
     const size_t sm = smem_bytes<TE_F, false>();
     if (c->n_xterms == 1)
-        k_cfconv_fwd<0, 1, 1><<<c->ncta, NT, sm, c->s>>>(a);
+        return launch_pdl(k_cfconv_fwd<0, 1, 1>, c->ncta, NT, sm, c->s, a);
     else if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_fwd<0, 2, 2><<<c->ncta, NT, sm, c->s>>>(a);
+        return launch_pdl(k_cfconv_fwd<0, 2, 2>, c->ncta, NT, sm, c->s, a);
     else if (c->weight_fmt == 0)
-        k_cfconv_fwd<0, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
+        return launch_pdl(k_cfconv_fwd<0, 1, 2>, c->ncta, NT, sm, c->s, a);
     else
-        k_cfconv_fwd<1, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
+        return launch_pdl(k_cfconv_fwd<1, 1, 2>, c->ncta, NT, sm, c->s, a);
 }
 
 // m = sum_j h_j (.) W_ij of interaction `layer`
@@ -1198,9 +1225,8 @@ cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
 {
     MPArgs a = make_args(c, layer);
     a.out = c->ws.m;
-    launch_fwd(c, a);
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_fwd(c, a);
 }
 
 // dE/dh_j = sum_i u_i (.) W_ij with u = dE/dm of interaction `layer`: the same
@@ -1210,9 +1236,8 @@ cudaError_t launch_cfconv_dh(schnet_ctx* c, int layer)
     MPArgs a = make_args(c, layer);
     a.h = c->ws.m;
     a.out = c->ws.dh;
-    launch_fwd(c, a);
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_fwd(c, a);
 }
 
 // Pair derivatives of interaction `layer` over the half list, written to s_e of
@@ -1227,16 +1252,17 @@ cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s)
     a.part = c->ws.part_h;
     a.accumulate_s = accumulate_s;
     const size_t sm = smem_bytes<TE_B, true>();
+    cudaError_t e;
     if (c->n_xterms == 1)
-        k_cfconv_bwd<0, 1, 1><<<c->ncta, NT, sm, c->s>>>(a);
+        e = launch_pdl(k_cfconv_bwd<0, 1, 1>, c->ncta, NT, sm, c->s, a);
     else if (c->weight_fmt == 0 && c->n_wterms == 2)
-        k_cfconv_bwd<0, 2, 2><<<c->ncta, NT, sm, c->s>>>(a);
+        e = launch_pdl(k_cfconv_bwd<0, 2, 2>, c->ncta, NT, sm, c->s, a);
     else if (c->weight_fmt == 0)
-        k_cfconv_bwd<0, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
+        e = launch_pdl(k_cfconv_bwd<0, 1, 2>, c->ncta, NT, sm, c->s, a);
     else
-        k_cfconv_bwd<1, 1, 2><<<c->ncta, NT, sm, c->s>>>(a);
+        e = launch_pdl(k_cfconv_bwd<1, 1, 2>, c->ncta, NT, sm, c->s, a);
     c->launches += 1;
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace schnet

@@ -27,6 +27,8 @@ __global__ void k_forces(int n, const int32_t* __restrict__ row_ptr, const int32
                          float rc, long long cap, DevMeta* meta, float4* __restrict__ frc4,
                          float* __restrict__ out3)
 {
+    pdl_trigger();
+    pdl_wait();
     if (meta->n_edges > cap) return;
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -73,10 +75,10 @@ cudaError_t launch_forces(schnet_ctx* c, float* d_forces)
     Workspace& w = c->ws;
     int blocks = (c->N + 7) / 8;   // 8 warps per block, one row per warp
     if (blocks > c->nsm * 16) blocks = c->nsm * 16;
-    k_forces<<<blocks, 256, 0, c->s>>>(c->N, w.row_ptr, w.col, w.rev, w.s_edge, w.pos4, w.perm, c->box, c->cfg.cutoff,
-                                       c->cap, w.meta, w.frc4, d_forces);
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_pdl(k_forces, blocks, 256, 0, c->s, c->N, (const int32_t*)w.row_ptr, (const int32_t*)w.col,
+                      (const int32_t*)w.rev, (const float*)w.s_edge, (const float4*)w.pos4, (const int32_t*)w.perm,
+                      c->box, c->cfg.cutoff, (long long)c->cap, w.meta, w.frc4, d_forces);
 }
 
 // --- Philox4x32-10 -----------------------------------------------------------
@@ -119,6 +121,8 @@ __global__ void k_baoa(int n, const int32_t* __restrict__ perm, float* __restric
                        unsigned long long seed, const float* __restrict__ noise, int check_skin, float half_skin2,
                        DevMeta* meta)
 {
+    pdl_trigger();
+    pdl_wait();
     const int k = blockIdx.x * blockDim.x + threadIdx.x;
     if (k >= n) return;
     const int i = perm[k];
@@ -165,17 +169,18 @@ cudaError_t launch_baoa(schnet_ctx* c, float* d_pos, float* d_vel, const float* 
     double c1 = exp(-(double)gamma * 1e-3 * (double)dt);
     double kT_acc = KB * (double)temp * (double)ACC;
     float hs = 0.5f * c->cfg.skin;
-    k_baoa<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, w.perm, d_pos, d_vel, d_mass, w.frc4, w.pos4, w.ref4, dt,
-                                                  (float)c1, (float)kT_acc, gamma != 0.f ? 1 : 0, seed, d_noise,
-                                                  check_skin ? 1 : 0, hs * hs, w.meta);
     c->launches += 1;
-    return cudaGetLastError();
+    return launch_pdl(k_baoa, (c->N + 255) / 256, 256, 0, c->s, c->N, (const int32_t*)w.perm, d_pos, d_vel, d_mass,
+                      (const float4*)w.frc4, w.pos4, (const float4*)w.ref4, dt, (float)c1, (float)kT_acc,
+                      gamma != 0.f ? 1 : 0, (unsigned long long)seed, d_noise, check_skin ? 1 : 0, hs * hs, w.meta);
 }
 
 // closing half kick; per-atom kinetic energy (kcal/mol) into tmp; step += 1
 __global__ void k_b_kick(int n, float* __restrict__ vel, const float* __restrict__ mass,
                          const float4* __restrict__ frc4, float dt, float* __restrict__ ke, DevMeta* meta)
 {
+    pdl_trigger();
+    pdl_wait();
     int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i == 0) meta->step += 1ull;
     if (i >= n) return;
@@ -196,9 +201,9 @@ cudaError_t launch_replica_sum(schnet_ctx* c, const float* v, double* out);
 cudaError_t launch_b_kick(schnet_ctx* c, float* d_vel, const float* d_mass, float dt, double* d_ekin, bool sum_ke)
 {
     Workspace& w = c->ws;
-    k_b_kick<<<(c->N + 255) / 256, 256, 0, c->s>>>(c->N, d_vel, d_mass, w.frc4, dt, w.ke, w.meta);
     c->launches += 1;
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(k_b_kick, (c->N + 255) / 256, 256, 0, c->s, c->N, d_vel, d_mass, (const float4*)w.frc4,
+                               dt, w.ke, w.meta);
     if (e != cudaSuccess || !sum_ke) return e;
     return launch_replica_sum(c, w.ke, d_ekin ? d_ekin : w.ekin);
 }

@@ -109,6 +109,28 @@ struct GraphKey {
     }
 };
 
+// Launch on `s` with programmatic stream serialization: the kernel's CTAs may be
+// scheduled while the previous kernel on the stream is still finishing, run
+// their prologue on constant data, and wait in pdl_wait for its results.  Every
+// kernel launched this way calls pdl_wait before reading anything an earlier
+// kernel wrote and before writing anything an earlier kernel reads.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                              Args... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace schnet
 
 struct schnet_ctx {

@@ -224,3 +224,32 @@ def test_protein64_sampled_replicas():
         print(f"[errors fp32 replica {r}] forces {rel_frobenius(F[sl], Fo):.3e}")
         check_energies(E[r:r + 1], Eo, eps_o, label=f"64 x 269 replica {r}")
         assert rel_frobenius(F[sl], Fo) <= FORCE_RTOL
+
+
+# ---------------------------------------------------------------------------
+# depth: one interaction (its single pair-derivative launch over the half list
+# starts the per-edge sums afresh) and four (three launches add to them)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("L", [1, 4])
+def test_energy_forces_other_depths(L):
+    w = SMALL_PROTEIN.with_(name=f"cg_protein_6x269_L{L}", L=L)
+    pos, types, weights, model = _setup(w, bias_scale=0.1)
+    E, F = _gpu_eval(model, pos, types)
+    ro = w.replica_offsets()
+    Eo, eps_o, Fo = oracle.energy_forces(oracle_model(w, weights), pos.astype(np.float64), types, ro)
+    check_energies(E, Eo, eps_o, ro, label=f"6 x 269, {L} interactions")
+    err = rel_frobenius(F, Fo)
+    print(f"[errors L={L}] forces {err:.3e}")
+    assert err <= FORCE_RTOL
+    # a second evaluation after a few MD steps (the pair sums restart every evaluation)
+    mass = _dev(workloads.masses(w), torch.float32)
+    p, v = _dev(pos, torch.float32), _dev(workloads.velocity_normals(w) * 0.003, torch.float32)
+    t = _dev(types, torch.int32)
+    model.step(p, v, t, mass, 5, n_rebuild=5, seed=9)
+    x = p.cpu().numpy()
+    model.build_neighbors(p)
+    E2, F2 = model.energy_forces(p, t)
+    torch.cuda.synchronize()
+    Eo2, eps_o2, Fo2 = oracle.energy_forces(oracle_model(w, weights), x.astype(np.float64), types, ro)
+    check_energies(E2.cpu().numpy(), Eo2, eps_o2, ro, label=f"6 x 269, {L} interactions, after 5 steps")
+    assert rel_frobenius(F2.cpu().numpy(), Fo2) <= FORCE_RTOL

@@ -152,9 +152,11 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.rev = cv.take<int32_t>(d.cap); w.erow = cv.take<int32_t>(d.cap);
     w.s_edge = cv.take<float>(d.cap);
     w.crow = cv.take<int32_t>(d.cap); w.ccol = cv.take<int32_t>(d.cap); w.cidx = cv.take<int32_t>(d.cap);
+    w.cdist = cv.take<float>(d.cap);
     w.ccount = cv.take<int32_t>(MAX_CTA);
     w.part = cv.take<int32_t>(MAX_CTA + 1);
     w.crow_h = cv.take<int32_t>(d.cap); w.ccol_h = cv.take<int32_t>(d.cap); w.cidx_h = cv.take<int32_t>(d.cap);
+    w.cdist_h = cv.take<float>(d.cap);
     w.ccount_h = cv.take<int32_t>(MAX_CTA);
     w.part_h = cv.take<int32_t>(MAX_CTA + 1);
     w.cell_of = cv.take<int32_t>(N); w.cell_atoms = cv.take<int32_t>(N);

@@ -44,7 +44,7 @@
 namespace schnet {
 
 struct MPArgs {
-    const float4* pos4;
+    const float* cdist;      // distance of each compacted edge (minimum image), from the masking pass
     const int32_t* crow;     // compacted edges (d < r_c) of each CTA's rows: row, column,
     const int32_t* ccol;     //   and index in the full list; CTA c's run starts at
     const int32_t* cidx;     //   row_ptr[part[c]] and holds ccount[c] edges
@@ -168,7 +168,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar)
 // dependent loads (edge -> atom -> position) overlap the previous tile's work.
 struct EdgePre {
     int i, j;
-    float4 pi, pj;
+    float d;       // the edge's distance, computed once per step by the masking pass
     int gidx;      // backward: index of the edge in the full list (where s_e is stored)
     float sold;    // backward: s_e accumulated by the later interactions so far
 };
@@ -179,15 +179,14 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
     EdgePre p;
     p.i = 0;
     p.j = -1;
-    p.pi = p.pj = make_float4(0.f, 0.f, 0.f, 0.f);
+    p.d = 0.f;
     p.gidx = 0;
     p.sold = 0.f;
     const int t = mt & (TE - 1);
     if (t < ne) {
         p.i = __ldg(a.crow + e0 + t);
         p.j = __ldg(a.ccol + e0 + t);
-        p.pi = __ldg(a.pos4 + p.i);
-        p.pj = __ldg(a.pos4 + p.j);
+        p.d = __ldg(a.cdist + e0 + t);
         if (BWD && mt < TE) {
             p.gidx = __ldg(a.cidx + e0 + t);
             if (a.accumulate_s) p.sold = a.s_edge[p.gidx];
@@ -214,9 +213,8 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMet
     float d = 0.f;
     bool valid = false;
     if (e < ne) {
-        float3 v;
-        d = edge_distance(ep.pi, ep.pj, a.box, v);
-        valid = d < a.rc && d > 0.f;
+        d = ep.d;
+        valid = d < a.rc && d > 0.f;   // holds for every compacted edge
     }
     if (kq == 0) {
         float fc = 0.f, dfc = 0.f;
@@ -1049,6 +1047,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 struct CompactList {
     const int32_t* part;
     int32_t *crow, *ccol, *cidx, *ccount;
+    float* cdist;
 };
 
 __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__ row_ptr, int ncta,
@@ -1064,6 +1063,7 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
     int32_t* __restrict__ ccol = L.ccol;
     int32_t* __restrict__ cidx = L.cidx;
     int32_t* __restrict__ ccount = L.ccount;
+    float* __restrict__ cdist = L.cdist;
     const int32_t* __restrict__ part = L.part;
     constexpr int CI = 4;             // consecutive edges per thread and pass
     __shared__ int wcount[32];
@@ -1080,6 +1080,7 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
     for (long long eb = e0; eb < e1; eb += (long long)CI * blockDim.x) {
         const long long ef = eb + (long long)CI * threadIdx.x;
         int ii[CI], jj[CI];
+        float dd[CI];
         unsigned vmask = 0;
 #pragma unroll
         for (int q = 0; q < CI; ++q) {
@@ -1095,6 +1096,7 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
             if (ef + q < e1) {
                 float3 v;
                 const float d = edge_distance(pos4[ii[q]], pos4[jj[q]], box, v);
+                dd[q] = d;
                 if (d < rc && d > 0.f && (!is_half || jj[q] > ii[q])) vmask |= 1u << q;
             }
         }
@@ -1128,6 +1130,7 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
                 crow[k] = ii[q];
                 ccol[k] = jj[q];
                 cidx[k] = (int32_t)(ef + q);
+                cdist[k] = dd[q];
                 ++k;
             }
         }
@@ -1142,8 +1145,8 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
 cudaError_t launch_compact(schnet_ctx* c, bool with_half)
 {
     Workspace& w = c->ws;
-    const CompactList full{w.part, w.crow, w.ccol, w.cidx, w.ccount};
-    const CompactList half{w.part_h, w.crow_h, w.ccol_h, w.cidx_h, w.ccount_h};
+    const CompactList full{w.part, w.crow, w.ccol, w.cidx, w.ccount, w.cdist};
+    const CompactList half{w.part_h, w.crow_h, w.ccol_h, w.cidx_h, w.ccount_h, w.cdist_h};
     c->launches += 1;
     return launch_pdl(k_compact, c->ncta * (with_half ? 2 : 1), 1024, 0, c->s, (const int32_t*)w.row_ptr,
                       (int)c->ncta, (const int32_t*)w.erow, (const int32_t*)w.col, (const float4*)w.pos4, c->box,
@@ -1157,7 +1160,7 @@ static MPArgs make_args(schnet_ctx* c, int layer)
 {
     Workspace& w = c->ws;
     MPArgs a;
-    a.pos4 = w.pos4;
+    a.cdist = w.cdist;
     a.crow = w.crow;
     a.ccol = w.ccol;
     a.cidx = w.cidx;
@@ -1248,6 +1251,7 @@ cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s)
     a.crow = c->ws.crow_h;
     a.ccol = c->ws.ccol_h;
     a.cidx = c->ws.cidx_h;
+    a.cdist = c->ws.cdist_h;
     a.ccount = c->ws.ccount_h;
     a.part = c->ws.part_h;
     a.accumulate_s = accumulate_s;

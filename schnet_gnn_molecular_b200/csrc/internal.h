@@ -71,9 +71,11 @@ struct Workspace {
     int32_t *col, *coltmp, *rev, *erow;  // [cap]
     float* s_edge;                // [cap]
     int32_t *crow, *ccol, *cidx;  // [cap] edges with d < r_c, per CTA row range
+    float* cdist;                 // [cap] their distances
     int32_t* ccount;              // [ncta]
     int32_t* part;                // [ncta+1]
     int32_t *crow_h, *ccol_h, *cidx_h;  // [cap] the half list: edges (i, j), j > i, d < r_c
+    float* cdist_h;               // [cap] their distances
     int32_t* ccount_h;            // [ncta]    its per-CTA edge counts
     int32_t* part_h;              // [ncta+1]  and its own row partition
     // cell list

@@ -53,7 +53,6 @@ struct MPArgs {
     const int32_t* part;
     DevMeta* meta;
     long long cap;
-    Box box;
     float rc, inv_rc;
     float mu0, dmu;       // Gaussian centres mu_k = mu0 + k dmu
     float ngc;            // -log2(e) / (2 sigma^2): e_k = 2^(ngc (d - mu_k)^2)
@@ -61,11 +60,11 @@ struct MPArgs {
     const uint8_t* img;   // this layer's packed W1^T / W2^T images
     const float *s1, *s2, *b1;  // this layer's channel scales and first-layer bias [FP]
     const float* b2;      // this layer's second-layer bias [FP]
-    const float* h;       // [N][FP]
-    const float* u;       // [N][FP]   (backward)
-    float* out;           // m (forward) or dh (backward)   [N][FP]
-    float* s_edge;        // [cap]     (backward)
-    int accumulate_s;
+    const float* h;       // [N][FP]   gathered per edge: h (forward), u = dE/dm (dE/dh launch), h (pairs)
+    const float* u;       // [N][FP]   u = dE/dm (pair kernel)
+    float* out;           // [N][FP]   m, or dE/dh (forward kernel)
+    float* s_edge;        // [cap]     pair derivatives on their owning edges (pair kernel)
+    int accumulate_s;     //           add to the later interactions' values
 };
 
 constexpr int NT = 512;                  // threads per CTA: two math groups of 8 warps
@@ -1169,7 +1168,6 @@ static MPArgs make_args(schnet_ctx* c, int layer)
     a.part = w.part;
     a.meta = w.meta;
     a.cap = c->cap;
-    a.box = c->box;
     a.rc = c->cfg.cutoff;
     a.inv_rc = 1.0f / c->cfg.cutoff;
     a.mu0 = c->mu0;

@@ -147,7 +147,7 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     if (wend) *wend = cv.off;
     w.pos4 = cv.take<float4>(N); w.ref4 = cv.take<float4>(N); w.frc4 = cv.take<float4>(N);
     w.perm = cv.take<int32_t>(N); w.cell_slot = cv.take<int32_t>(N);
-    w.row_ptr = cv.take<int32_t>(N + 1); w.rowcnt = cv.take<int32_t>(N + 1);
+    w.row_ptr = cv.take<int32_t>(N + 1); w.rowcnt = cv.take<int32_t>(N + 1); w.hcnt = cv.take<int32_t>(N + 1);
     w.col = cv.take<int32_t>(d.cap); w.coltmp = cv.take<int32_t>(d.cap);
     w.rev = cv.take<int32_t>(d.cap); w.erow = cv.take<int32_t>(d.cap);
     w.s_edge = cv.take<float>(d.cap);

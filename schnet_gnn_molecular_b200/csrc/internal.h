@@ -68,6 +68,7 @@ struct Workspace {
     float4 *pos4, *ref4, *frc4;   // [N]
     // neighbour list
     int32_t *row_ptr, *rowcnt;    // [N+1]
+    int32_t* hcnt;                // [N+1] per-row half-list counts (scratch of the partition)
     int32_t *col, *coltmp, *rev, *erow;  // [cap]
     float* s_edge;                // [cap]
     int32_t *crow, *ccol, *cidx;  // [cap] edges with d < r_c, per CTA row range

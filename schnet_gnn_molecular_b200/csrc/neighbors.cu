@@ -448,17 +448,14 @@ __global__ void k_rev(const int32_t* __restrict__ row_ptr, const int32_t* __rest
 // within a row, so the unsorted erow is already correct.
 
 // Row partition of the tensor-core kernels: CTA c takes whole rows holding
-// about one share of the edges (at least a few tiles).  row_ptr counts the
-// edges to balance: the whole list (E from the build), or with half = 1 the
-// half list of one edge per unordered pair (E = row_ptr[n]).
+// about one share of the edges (at least a few tiles).  row_ptr is the exclusive
+// prefix sum over the rows of the edges to balance, row_ptr[n] their total.
 __global__ void k_partition(int n, int ncta, const int32_t* __restrict__ row_ptr, long long cap,
-                            const DevMeta* meta, int half, int32_t* __restrict__ part)
+                            const DevMeta* meta, int32_t* __restrict__ part)
 {
     int c = blockIdx.x * blockDim.x + threadIdx.x;
     if (c > ncta) return;
-    long long E = meta->n_edges;
-    if (E > cap) E = 0;
-    else if (half) E = row_ptr[n];
+    const long long E = meta->n_edges > cap ? 0 : row_ptr[n];
     long long share = (E + ncta - 1) / ncta;
     if (share < 2 * TILE_E) share = 2 * TILE_E;
     share = (share + TILE_E - 1) / TILE_E * TILE_E;
@@ -475,21 +472,43 @@ __global__ void k_partition(int n, int ncta, const int32_t* __restrict__ row_ptr
     part[c] = lo;
 }
 
-// Per row, the listed edges (i, j) with j > i: the half list that visits each
-// unordered pair once (rows are sorted, so they are the row's tail).
-__global__ void k_half_counts(int n, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
-                              long long cap, const DevMeta* meta, int32_t* __restrict__ cnt)
+// Per row, the edges the tensor-core kernels will carry at the build's positions:
+// those inside the cutoff (cnt), and of them those with j > i (cnt_half, the half
+// list that visits each unordered pair once).  The distance is the masking pass's
+// own expression, so the counts equal what it keeps at these positions; the row
+// partitions balance them.  One warp per row.
+__global__ void k_cut_counts(int n, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
+                             const float4* __restrict__ pos4, const Box box, float rc, long long cap,
+                             const DevMeta* meta, int32_t* __restrict__ cnt, int32_t* __restrict__ cnt_half)
 {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n) return;
-    if (meta->n_edges > cap) { cnt[i] = 0; return; }
-    int lo = row_ptr[i], hi = row_ptr[i + 1];
-    const int end = hi;
-    while (lo < hi) {                      // first entry with col > i
-        const int mid = (lo + hi) >> 1;
-        if (col[mid] > i) hi = mid; else lo = mid + 1;
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    const bool over = meta->n_edges > cap;
+    for (int i = warp; i < n; i += nwarps) {
+        int c = 0, ch = 0;
+        if (!over) {
+            const float4 pi = pos4[i];
+            for (int e = row_ptr[i] + lane; e < row_ptr[i + 1]; e += 32) {
+                const int j = col[e];
+                float3 v;
+                const float d = edge_distance(pi, pos4[j], box, v);
+                if (d < rc && d > 0.f) {
+                    ++c;
+                    ch += j > i;
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            c += __shfl_xor_sync(0xffffffffu, c, o);
+            ch += __shfl_xor_sync(0xffffffffu, ch, o);
+        }
+        if (lane == 0) {
+            cnt[i] = c;
+            cnt_half[i] = ch;
+        }
     }
-    cnt[i] = end - lo;
 }
 
 __global__ void k_check_capacity(long long cap, DevMeta* meta)
@@ -536,14 +555,17 @@ cudaError_t launch_build_neighbors(schnet_ctx* c, const float* d_pos)
     int nsort = c->nsm * 8;
     k_sort_rows<<<nsort, 256, 0, c->s>>>(N, w.row_ptr, w.coltmp, c->cap, w.meta, w.col);
     k_rev<<<c->nsm * 8, 256, 0, c->s>>>(w.row_ptr, w.col, w.erow, c->cap, w.meta, w.rev);
-    k_partition<<<(c->ncta + 1 + 127) / 128, 128, 0, c->s>>>(N, c->ncta, w.row_ptr, c->cap, w.meta, 0, w.part);
-    // the half list's own partition (rowcnt is free scratch once the list is built)
-    k_half_counts<<<nb, 256, 0, c->s>>>(N, w.row_ptr, w.col, c->cap, w.meta, w.rowcnt);
-    c->launches += 6;
+    // the row partitions of the full and the half list, balanced on the edges inside the
+    // cutoff at the build's positions (rowcnt is free scratch once the list is built)
+    k_cut_counts<<<c->nsm * 8, 256, 0, c->s>>>(N, w.row_ptr, w.col, w.pos4, c->box, c->cfg.cutoff, c->cap, w.meta,
+                                               w.rowcnt, w.hcnt);
+    c->launches += 5;
     if ((err = scan_exclusive(c, w.rowcnt, N, w.rowcnt, nullptr)) != cudaSuccess) return err;   // in place
-    k_partition<<<(c->ncta + 1 + 127) / 128, 128, 0, c->s>>>(N, c->ncta, w.rowcnt, c->cap, w.meta, 1, w.part_h);
+    if ((err = scan_exclusive(c, w.hcnt, N, w.hcnt, nullptr)) != cudaSuccess) return err;
+    k_partition<<<(c->ncta + 1 + 127) / 128, 128, 0, c->s>>>(N, c->ncta, w.rowcnt, c->cap, w.meta, w.part);
+    k_partition<<<(c->ncta + 1 + 127) / 128, 128, 0, c->s>>>(N, c->ncta, w.hcnt, c->cap, w.meta, w.part_h);
     cudaMemcpyAsync(w.ref4, w.pos4, sizeof(float4) * N, cudaMemcpyDeviceToDevice, c->s);
-    c->launches += 1;
+    c->launches += 2;
     return cudaGetLastError();
 }
 

@@ -333,23 +333,30 @@ def run_native(args):
         clk_prof = clocks.window(prof_t0, prof_t1)
         E_list, E_cut = _edge_stats(model, p.cpu().numpy(), w)
         peaks, src = _peaks()
-        # algorithmic work per launch: the forward kernel (interactions' forward and their dE/dh)
-        # contracts the filter MLP once per directed edge inside the cutoff; the pair kernel
-        # forms W and its derivative W' (twice the contraction) per unordered pair (E_cut / 2)
-        flop_launch = 2.0 * (w.K * w.F + w.F * w.F) * E_cut
+        # algorithmic work per step: the forward kernel contracts the filter MLP (45,568 FLOP for
+        # the 64 x 269 model) once per directed edge inside the cutoff in each interaction's
+        # forward, and once per edge of the complementary half list (E_cut / 2) in the dE/dh
+        # launches of interactions 1..L-1; the pair kernel forms W and its derivative W' (twice
+        # the contraction) per unordered pair (E_cut / 2) in every interaction
+        f1 = 2.0 * (w.K * w.F + w.F * w.F)
         mu = mufu_per_edge(w.K, w.F)
-        kern = {"k_cfconv_fwd": {"classes": ("cfconv_fwd", "cfconv_dh"), "mufu": mu["fwd"] * E_cut},
-                "k_cfconv_bwd": {"classes": ("cfconv_bwd",), "mufu": mu["bwd"] * E_cut / 2}}
+        fwd_edges = (w.L + (w.L - 1) * 0.5) * E_cut
+        kern = {"k_cfconv_fwd": {"classes": ("cfconv_fwd", "cfconv_dh"), "flop_step": f1 * fwd_edges,
+                                 "mufu_step": mu["fwd"] * fwd_edges},
+                "k_cfconv_bwd": {"classes": ("cfconv_bwd",), "flop_step": 2.0 * f1 * w.L * E_cut / 2,
+                                 "mufu_step": mu["bwd"] * w.L * E_cut / 2}}
         for k, v in kern.items():
-            v["ms"] = sum(prof[c][0] for c in v["classes"])
+            v["ms"] = sum(prof[c][0] for c in v["classes"])        # over the n_rb profiled steps
             v["launches"] = sum(prof[c][1] for c in v["classes"])
             v["ms_per_launch"] = v["ms"] / max(v["launches"], 1)
+            v["flop_launch"] = v["flop_step"] * n_rb / max(v["launches"], 1)
+            v["mufu"] = v["mufu_step"] * n_rb / max(v["launches"], 1)
         per_launch = {k: x[0] / max(x[1], 1) for k, x in prof.items()}
         per_step = {k: x[0] / n_rb for k, x in prof.items()}
         tot_ms = sum(x[0] for x in prof.values())
         dominant = max(kern, key=lambda k: kern[k]["ms"])
         kms = kern[dominant]["ms_per_launch"]
-        flops = flop_launch
+        flops = kern[dominant]["flop_launch"]
         peak, peak_kind = tensor_peak(peaks, clk_prof)
         achieved = flops / (kms * 1e-3) / 1e12
         traffic = _traffic(dominant)
@@ -359,11 +366,13 @@ def run_native(args):
         mufu_peak = 148 * 16 * f_clk
         hb = hbm_kernel_bytes(w, E_list, E_cut)
         n_aw = 6 * w.L                                    # atom-wise layer applications per step
-        tensor_s = flop_launch / (peak * 1e12)
+        fw, bw = kern["k_cfconv_fwd"], kern["k_cfconv_bwd"]
+        share_dh = (w.L - 1) * 0.5 / (w.L + (w.L - 1) * 0.5)     # the dE/dh launches' part of fw
+        fw_bound = max(fw["flop_step"] / (peak * 1e12), fw["mufu_step"] / mufu_peak)
         bounds = {
-            "cfconv_fwd": w.L * max(tensor_s, kern["k_cfconv_fwd"]["mufu"] / mufu_peak),
-            "cfconv_dh": (w.L - 1) * max(tensor_s, kern["k_cfconv_fwd"]["mufu"] / mufu_peak),
-            "cfconv_bwd": w.L * max(tensor_s, kern["k_cfconv_bwd"]["mufu"] / mufu_peak),
+            "cfconv_fwd": fw_bound * (1.0 - share_dh),
+            "cfconv_dh": fw_bound * share_dh,
+            "cfconv_bwd": max(bw["flop_step"] / (peak * 1e12), bw["mufu_step"] / mufu_peak),
             "atomwise": max(n_aw * 2.0 * w.F * w.F * w.n_atoms / (peak * 1e12),
                             n_aw * 2 * w.n_atoms * w.F * 4 / hbm),
             "forces": hb["forces"] / hbm, "integrate": hb["integrate"] / hbm, "mask": hb["mask"] / hbm,
@@ -383,9 +392,9 @@ def run_native(args):
                  "how": f"one CUDA Graph of {k_interval} trivial kernels (one rebuild interval's count), "
                         f"replayed; per step = replay time / {n_rb}"}
         fused = {k: {"launches_per_step": round(v["launches"] / n_rb, 2), "ms_per_launch": round(v["ms_per_launch"], 4),
-                     "flop_per_launch": flop_launch,
-                     "tflops": round(flop_launch / (v["ms_per_launch"] * 1e-3) / 1e12, 2),
-                     "frac_tensor": round(flop_launch / (v["ms_per_launch"] * 1e-3) / 1e12 / peak, 4),
+                     "flop_per_launch": v["flop_launch"],
+                     "tflops": round(v["flop_launch"] / (v["ms_per_launch"] * 1e-3) / 1e12, 2),
+                     "frac_tensor": round(v["flop_launch"] / (v["ms_per_launch"] * 1e-3) / 1e12 / peak, 4),
                      "mufu_per_launch": v["mufu"],
                      "frac_mufu": round(v["mufu"] / (v["ms_per_launch"] * 1e-3) / mufu_peak, 4)}
                  for k, v in kern.items()}

@@ -147,7 +147,8 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     if (wend) *wend = cv.off;
     w.pos4 = cv.take<float4>(N); w.ref4 = cv.take<float4>(N); w.frc4 = cv.take<float4>(N);
     w.perm = cv.take<int32_t>(N); w.cell_slot = cv.take<int32_t>(N);
-    w.row_ptr = cv.take<int32_t>(N + 1); w.rowcnt = cv.take<int32_t>(N + 1); w.hcnt = cv.take<int32_t>(N + 1);
+    w.row_ptr = cv.take<int32_t>(N + 1); w.rowcnt = cv.take<int32_t>(N + 1);
+    w.hcnt = cv.take<int32_t>(N + 1); w.rcnt = cv.take<int32_t>(N + 1);
     w.col = cv.take<int32_t>(d.cap); w.coltmp = cv.take<int32_t>(d.cap);
     w.rev = cv.take<int32_t>(d.cap); w.erow = cv.take<int32_t>(d.cap);
     w.s_edge = cv.take<float>(d.cap);
@@ -159,6 +160,9 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.cdist_h = cv.take<float>(d.cap);
     w.ccount_h = cv.take<int32_t>(MAX_CTA);
     w.part_h = cv.take<int32_t>(MAX_CTA + 1);
+    w.crow_r = cv.take<int32_t>(d.cap); w.ccol_r = cv.take<int32_t>(d.cap); w.cdist_r = cv.take<float>(d.cap);
+    w.ccount_r = cv.take<int32_t>(MAX_CTA);
+    w.part_r = cv.take<int32_t>(MAX_CTA + 1);
     w.cell_of = cv.take<int32_t>(N); w.cell_atoms = cv.take<int32_t>(N);
     w.cell_cnt = cv.take<int32_t>((size_t)d.ncell + 1); w.cell_start = cv.take<int32_t>((size_t)d.ncell + 1);
     w.cell_fill = cv.take<int32_t>((size_t)d.ncell + 1);
@@ -534,10 +538,11 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
     if (!need_forces) return cudaSuccess;
     SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd_top(c));
     for (int l = c->L - 1; l >= 0; --l) {
-        // pair derivatives over the half list (one edge per unordered pair)
-        SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_pair(c, l, l < c->L - 1 ? 1 : 0));
-        // dE/dh and the atom-wise backward carry the gradient to the earlier interactions;
-        // interaction 0's would only reach the embedding, which forces do not need
+        // pair derivatives over the half list (one edge per unordered pair) and, but for
+        // interaction 0 (whose dE/dh would only reach the embedding, which forces do not
+        // need), the half list's terms of dE/dh; the complementary list adds the rest, and
+        // the atom-wise backward carries the gradient to the earlier interactions
+        SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_pair(c, l, l < c->L - 1 ? 1 : 0, l > 0));
         if (l > 0) {
             SCHNET_TIMED(SCHNET_KERNEL_CFCONV_DH, launch_cfconv_dh(c, l));
             SCHNET_TIMED(SCHNET_KERNEL_ATOMWISE, launch_aw_bwd(c, l));

@@ -374,6 +374,21 @@ struct ChunkSeg {
     float acc, pf;
 };
 
+// A completed row's sum into out (ACC: added to what an earlier launch left there),
+// and the rows between two rows with edges: zero, or left as they are with ACC.
+template <bool ACC>
+__device__ __forceinline__ void put_row(float* __restrict__ out, int row, int f, float v)
+{
+    if (ACC) out[(size_t)row * FP + f] += v;
+    else out[(size_t)row * FP + f] = v;
+}
+template <bool ACC>
+__device__ __forceinline__ void zero_rows(float* __restrict__ out, int from, int to, int f)
+{
+    if (!ACC)
+        for (int rr = from; rr < to; ++rr) out[(size_t)rr * FP + f] = 0.f;
+}
+
 __device__ __forceinline__ void seg_begin(ChunkSeg& c, int rfirst)
 {
     c.rfirst = rfirst;
@@ -382,12 +397,13 @@ __device__ __forceinline__ void seg_begin(ChunkSeg& c, int rfirst)
     c.pf = 0.f;
 }
 
+template <bool ACC>
 __device__ __forceinline__ void seg_row(ChunkSeg& c, int row, float* __restrict__ out, int f)
 {
     if (row != c.lrow) {
         if (c.lrow == c.rfirst) c.pf = c.acc;
-        else out[(size_t)c.lrow * FP + f] = c.acc;
-        for (int rr = c.lrow + 1; rr < row; ++rr) out[(size_t)rr * FP + f] = 0.f;
+        else put_row<ACC>(out, c.lrow, f, c.acc);
+        zero_rows<ACC>(out, c.lrow + 1, row, f);
         c.lrow = row;
         c.acc = 0.f;
     }
@@ -396,7 +412,7 @@ __device__ __forceinline__ void seg_row(ChunkSeg& c, int row, float* __restrict_
 // In-order merge of a tile's chunk partials into the carried row (threads of
 // the group with feature f = group thread index < 128): rows the carry leaves
 // are complete and written out, with zeros for edge-less rows in between.
-template <int NCH>
+template <int NCH, bool ACC>
 __device__ __forceinline__ void merge_chunks(const ChunkInfo* ci, const float* pf, const float* pl, int ne, int f,
                                              float* __restrict__ out, int& cur, float& acc)
 {
@@ -408,13 +424,13 @@ __device__ __forceinline__ void merge_chunks(const ChunkInfo* ci, const float* p
         if (rfirst == cur) {
             acc += v;
         } else {
-            out[(size_t)cur * FP + f] = acc;
-            for (int rr = cur + 1; rr < rfirst; ++rr) out[(size_t)rr * FP + f] = 0.f;
+            put_row<ACC>(out, cur, f, acc);
+            zero_rows<ACC>(out, cur + 1, rfirst, f);
             cur = rfirst;
             acc = v;
         }
         if (rlast != rfirst) {
-            out[(size_t)cur * FP + f] = acc;
+            put_row<ACC>(out, cur, f, acc);
             cur = rlast;
             acc = pl[c * 128 + f];
         }
@@ -423,7 +439,7 @@ __device__ __forceinline__ void merge_chunks(const ChunkInfo* ci, const float* p
 
 // Merge step of tile t by its group: wait for tile t-1's merge, fold this
 // tile's partials into the carry, hand the carry on.  Returns false on timeout.
-template <int NCH>
+template <int NCH, bool ACC>
 __device__ __forceinline__ bool merge_tile(Carry* cy, uint64_t* tok, const ChunkInfo* ci, const float* pf,
                                            const float* pl, int ne, int t, float* __restrict__ out, DevMeta* meta,
                                            int g, int mt)
@@ -432,7 +448,7 @@ __device__ __forceinline__ bool merge_tile(Carry* cy, uint64_t* tok, const Chunk
     if (mt < 128) {
         int cur = cy->cur[(t + 1) & 1];      // written by tile t-1 (or the initial row)
         float acc = cy->acc[mt];
-        merge_chunks<NCH>(ci, pf, pl, ne, mt, out, cur, acc);
+        merge_chunks<NCH, ACC>(ci, pf, pl, ne, mt, out, cur, acc);
         cy->acc[mt] = acc;
         if (mt == 0) cy->cur[t & 1] = cur;
         mbar_arrive(tok);
@@ -460,7 +476,7 @@ __device__ __forceinline__ float tree_sum(float (&v)[N])
 // rows strictly between them are written as zeros).  Three or more rows: the
 // serial segmented sum (rows read from the tile's global row list) writes the
 // inner rows out.
-template <int N>
+template <int N, bool ACC>
 __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_t* __restrict__ rows_g, int eb,
                                                int ne, float (&t)[N], float* __restrict__ out, int f, float& pf,
                                                float& pl)
@@ -479,7 +495,7 @@ __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_
             }
             pf = tree_sum<N>(t);
             pl = tree_sum<N>(u);
-            for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) out[(size_t)rr * FP + f] = 0.f;
+            zero_rows<ACC>(out, ci.rfirst + 1, ci.rlast, f);
         }
         return;
     }
@@ -489,7 +505,7 @@ __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_
     for (int q = 0; q < N; ++q) {
         const int e = eb + q;
         if (e >= ne) break;
-        seg_row(c, __ldg(rows_g + e), out, f);
+        seg_row<ACC>(c, __ldg(rows_g + e), out, f);
         c.acc += t[q];
     }
     if (c.lrow == c.rfirst) { pf = c.acc; pl = 0.f; } else { pf = c.pf; pl = c.acc; }
@@ -559,7 +575,8 @@ __device__ __forceinline__ bool kernel_rows(const MPArgs& a, uint32_t tmem, Carr
 }
 
 // Common epilogue: the carried row is complete; rows after it without edges are zero
-// (nothing to write when the kernel produces no per-row output).
+// (left as they are with ACC; nothing to write when the kernel produces no per-row output).
+template <bool ACC>
 __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r1, float* __restrict__ out, bool ok,
                                               uint64_t* bars, const uint32_t* phases, const uint32_t* pending,
                                               uint32_t tmem, bool write_out = true)
@@ -568,8 +585,9 @@ __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r
     if (ok && write_out) {
         if (threadIdx.x < FP) {
             const int cur = cy->cur[(ntiles + 1) & 1];
-            out[(size_t)cur * FP + threadIdx.x] = cy->acc[threadIdx.x];
-            for (int rr = cur + 1; rr < r1; ++rr) out[(size_t)rr * FP + threadIdx.x] = 0.f;
+            if (ntiles > 0) put_row<ACC>(out, cur, threadIdx.x, cy->acc[threadIdx.x]);
+            else zero_rows<ACC>(out, cur, cur + 1, threadIdx.x);
+            zero_rows<ACC>(out, cur + 1, r1, threadIdx.x);
         }
     } else if ((threadIdx.x & (GT - 1)) == 0) {
         // drain: give the group's in-flight MMAs a bounded chance to retire before freeing TMEM
@@ -611,7 +629,7 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
 }
 
 // forward epilogue 2 for chunk cc: W = f_c (s2 ln2 Q + b2), terms h_j W, chunk partials
-template <int TE>
+template <int TE, bool ACC>
 __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* tm, const int32_t* rows_g, int cc,
                                        int ne, float s2L, float b2, const float (&hv)[32], float* __restrict__ out,
                                        int f, float& pf, float& pl)
@@ -631,7 +649,7 @@ __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* t
         r[q] = v.x;
         r[q + 1] = v.y;
     }
-    chunk_partials<32>(tm->c[cc], rows_g, eb, ne, r, out, f, pf, pl);
+    chunk_partials<32, ACC>(tm->c[cc], rows_g, eb, ne, r, out, f, pf, pl);
 }
 
 // Issue GEMM1 of a tile (group g): D = W1^T [B rows of the group's GEMM1 operand]
@@ -650,7 +668,7 @@ __device__ __forceinline__ void issue_gemm1(uint32_t tmem, uint32_t dacc, uint32
 // t+2 (into the group's own GEMM1 operand and second metadata buffer) and the
 // first gather under GEMM2 -> E2 -> issue GEMM1(t+2) (by warp 4) -> merge under GEMM1(t+2)
 // (warps 0-3).
-template <int FMT, int NW, int NX>
+template <int FMT, int NW, int NX, bool ACC>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {
     constexpr int TE = TE_F;
@@ -744,7 +762,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
             const int cc = ch * 2 + c2;
             if (c2 == 1) gather<32>(h_f, tm->col, cc * 32, hv);
             float pf, pl;
-            fwd_e2<TE>(tA + c2 * 32, tm, rows_g, cc, ne, s2L, b2, hv, a.out, f, pf, pl);
+            fwd_e2<TE, ACC>(tA + c2 * 32, tm, rows_g, cc, ne, s2L, b2, hv, a.out, f, pf, pl);
             pf_s[cc * 128 + f] = pf;
             pl_s[cc * 128 + f] = pl;
         }
@@ -754,7 +772,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         // thread blocks while the tensor core's queue is full)
         if (next && mt == 128) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
-        if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
+        if (!(ok = merge_tile<NCH, ACC>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
         group_sync(g);          // merge done with the partials before E1 of the next tile overwrites them
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
@@ -763,7 +781,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         pend_s[g] = ok ? 0u : pending;
     }
     const bool all_ok = __syncthreads_or(!ok) == 0;
-    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem);
+    kernel_finish<ACC>(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem);
 }
 
 // ---------------------------------------------------------------------------
@@ -814,18 +832,22 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
     }
 }
 
-// Backward of one interaction for the forces: the pair derivative
-// dE/dd_ij = D_ij = sum_f W'_f(d_ij) (u_i,f h_j,f + u_j,f h_i,f), the same for
-// (i, j) and (j, i) because W_ij = W_ji.  The launch runs over one edge per
+// Backward of one interaction.  The pair derivative
+// dE/dd_ij = D_ij = sum_f W'_f(d_ij) (u_i,f h_j,f + u_j,f h_i,f) is the same for
+// (i, j) and (j, i) because W_ij = W_ji: the launch runs over one edge per
 // unordered pair (the half list: edges (i, j) with j > i, in rows balanced by
 // their own partition) and writes (adds, for the later interactions' sums) D_ij
 // to s_e of that edge; the force assembly reads each pair's value from its
-// owning edge, so both atoms receive it.  dE/dh_j = sum_i u_i (.) W_ij is the
-// forward kernel's segment sum with u in place of h, launched separately.
-template <int FMT, int NW, int NX>
+// owning edge, so both atoms receive it.  With DH (every interaction but the
+// first, whose dE/dh would only reach the embedding) the same tiles also form
+// row i's share of dE/dh_i = sum_j W_ij (.) u_j over its half-list edges, a
+// segment sum in registers written to out like the forward's; the other half
+// (j < i) is the forward kernel over the complementary list, adding to out.
+template <int FMT, int NW, int NX, bool DH>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
     constexpr int TE = TE_B;
+    constexpr int NCH = TE / 32;
     using Meta = TileMeta<TE, true>;
     extern __shared__ __align__(1024) uint8_t smem[];
     Carry* cy = reinterpret_cast<Carry*>(smem + sm_carry<TE, true>());
@@ -849,7 +871,9 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     uint8_t* rbf = smem + SM_RBF + g * 2 * RBF_TERM;
     uint8_t* act = smem + SM_ACT + g * 2 * ACT_TERM;
     Meta* tmb = reinterpret_cast<Meta*>(smem + sm_meta<TE, true>() + g * 2 * sizeof(Meta));
-    float* ps_s = reinterpret_cast<float*>(act);    // after GEMM2: [quadrant][edge] partial of D
+    float* pf_s = reinterpret_cast<float*>(act);    // after GEMM2: [chunk][feature] dE/dh partials
+    float* pl_s = pf_s + NCH * 128;
+    float* ps_s = pl_s + NCH * 128;                 // [quadrant][edge] partial of D
     // per-warp [32 edges][36] scratch of the D transpose (behind the partials, inside the
     // group's GEMM2 operand buffer, which is free between GEMM2's completion and the next E1)
     float* s_w = reinterpret_cast<float*>(act + 4096) + (warp & 7) * (32 * 36);
@@ -924,97 +948,128 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         gather<16>(h_f, tm->col, eb, hv);
         if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2(t) done
         pending = 0;
-        // epilogue 2: W' = f_c' z + f_c z' (z = s2 ln2 Q + b2, z' = s2 Q'), and per edge the
-        // pair derivative D = sum_f W'_f (u_i,f h_j,f + u_j,f h_i,f)
-        if (eb < ne) {
-            const ChunkInfo ci = tm->c[ch];
-            // 1: one row in the chunk; 2: two rows (the first a prefix); 3: a third row occurs,
-            // rows read per edge
-            const int kind = ci.other ? 3 : (ci.rfirst == ci.rlast ? 1 : 2);
-            const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
-            const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
-            const float h_first = __ldg(h_f + (size_t)ci.rfirst * FP);
-            const float h_last = __ldg(h_f + (size_t)ci.rlast * FP);
-            int lrow = ci.rfirst;
-            float u_row = u_first, h_row = h_first;
+        // epilogue 2: W = f_c z, W' = f_c' z + f_c z' (z = s2 ln2 Q + b2, z' = s2 Q'); per edge the
+        // pair derivative D = sum_f W'_f (u_i,f h_j,f + u_j,f h_i,f) and, with DH, the row's share
+        // of dE/dh_i = sum_j W_ij (.) u_j as a segment sum (chunk partials, merged in tile order)
+        {
+            float pf = 0.f, pl = 0.f;
+            if (eb < ne) {
+                const ChunkInfo ci = tm->c[ch];
+                // 1: one row in the chunk; 2: two rows (the first a prefix); 3: a third row
+                // occurs, rows read per edge
+                const int kind = ci.other ? 3 : (ci.rfirst == ci.rlast ? 1 : 2);
+                const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
+                const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
+                const float h_first = __ldg(h_f + (size_t)ci.rfirst * FP);
+                const float h_last = __ldg(h_f + (size_t)ci.rlast * FP);
+                float u_row = u_first, h_row = h_first;
+                float sf = 0.f, sl = 0.f;
+                ChunkSeg c;
+                seg_begin(c, ci.rfirst);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                if (hh == 1) {
-                    gather<16>(u_f, tm->col, eb + 16, uv);
-                    gather<16>(h_f, tm->col, eb + 16, hv);
-                }
-                float r[16], rd[16];
-                tmem_ld16(tP + hh * 16, r);          // Q
-                tmem_ld16(tPd + hh * 16, rd);        // Q'
-                tmem_ld_wait();
-                const float* fcp = tm->fc + eb + hh * 16;
-                const float* dfcp = tm->dfc + eb + hh * 16;
-                if (kind == 1) {
-#pragma unroll
-                    for (int gq = 0; gq < 16; gq += 4) {
-                        float fc[4], dfc[4];
-                        load_edges<4>(fcp, gq, fc);
-                        load_edges<4>(dfcp, gq, dfc);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int q = gq + i;
-                            const float z = fmaf(s2L, r[q], b2);
-                            const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
-                            rd[q] = wd * fmaf(uv[q], h_first, u_first * hv[q]);
-                        }
+                for (int hh = 0; hh < 2; ++hh) {
+                    if (hh == 1) {
+                        gather<16>(u_f, tm->col, eb + 16, uv);
+                        gather<16>(h_f, tm->col, eb + 16, hv);
                     }
-                } else if (kind == 2) {
+                    float r[16], rd[16];
+                    tmem_ld16(tP + hh * 16, r);          // Q
+                    tmem_ld16(tPd + hh * 16, rd);        // Q'
+                    tmem_ld_wait();
+                    const float* fcp = tm->fc + eb + hh * 16;
+                    const float* dfcp = tm->dfc + eb + hh * 16;
+                    if (kind == 1) {
 #pragma unroll
-                    for (int gq = 0; gq < 16; gq += 4) {
-                        float fc[4], dfc[4];
-                        load_edges<4>(fcp, gq, fc);
-                        load_edges<4>(dfcp, gq, dfc);
+                        for (int gq = 0; gq < 16; gq += 4) {
+                            float fc[4], dfc[4];
+                            load_edges<4>(fcp, gq, fc);
+                            load_edges<4>(dfcp, gq, dfc);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int q = gq + i;
-                            const float z = fmaf(s2L, r[q], b2);
-                            const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
-                            const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
-                            rd[q] = wd * fmaf(uv[q], first ? h_first : h_last, (first ? u_first : u_last) * hv[q]);
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int e = eb + hh * 16 + q;
-                        float tval = 0.f;
-                        if (e < ne) {
-                            const int row = __ldg(rows_g + e);
-                            if (row != lrow) {
-                                lrow = row;
-                                u_row = __ldg(u_f + (size_t)row * FP);
-                                h_row = __ldg(h_f + (size_t)row * FP);
+                            for (int i = 0; i < 4; ++i) {
+                                const int q = gq + i;
+                                const float z = fmaf(s2L, r[q], b2);
+                                if (DH) sf = fmaf(fc[i] * z, uv[q], sf);
+                                const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
+                                rd[q] = wd * fmaf(uv[q], h_first, u_first * hv[q]);
                             }
-                            const float z = fmaf(s2L, r[q], b2);
-                            const float wd = fmaf(dfcp[q], z, fcp[q] * (s2 * rd[q]));
-                            tval = wd * fmaf(uv[q], h_row, u_row * hv[q]);
                         }
-                        rd[q] = tval;
+                    } else if (kind == 2) {
+#pragma unroll
+                        for (int gq = 0; gq < 16; gq += 4) {
+                            float fc[4], dfc[4];
+                            load_edges<4>(fcp, gq, fc);
+                            load_edges<4>(dfcp, gq, dfc);
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int q = gq + i;
+                                const float z = fmaf(s2L, r[q], b2);
+                                const bool first = (ci.firstmask >> (hh * 16 + q)) & 1u;
+                                if (DH) {
+                                    const float dt = fc[i] * z * uv[q];
+                                    sf += first ? dt : 0.f;
+                                    sl += first ? 0.f : dt;
+                                }
+                                const float wd = fmaf(dfc[i], z, fc[i] * (s2 * rd[q]));
+                                rd[q] = wd * fmaf(uv[q], first ? h_first : h_last, (first ? u_first : u_last) * hv[q]);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 16; ++q) {
+                            const int e = eb + hh * 16 + q;
+                            float tval = 0.f;
+                            if (e < ne) {
+                                const int row = __ldg(rows_g + e);
+                                if (row != c.lrow) {
+                                    if (DH) seg_row<false>(c, row, a.out, f);
+                                    else c.lrow = row;
+                                    u_row = __ldg(u_f + (size_t)row * FP);
+                                    h_row = __ldg(h_f + (size_t)row * FP);
+                                }
+                                const float z = fmaf(s2L, r[q], b2);
+                                if (DH) c.acc = fmaf(fcp[q] * z, uv[q], c.acc);
+                                const float wd = fmaf(dfcp[q], z, fcp[q] * (s2 * rd[q]));
+                                tval = wd * fmaf(uv[q], h_row, u_row * hv[q]);
+                            }
+                            rd[q] = tval;
+                        }
                     }
-                }
-                // stage this half's 16 per-edge values as S[edge][feature lane] (row stride 36:
-                // the stores and the 16-byte row reads below are free of bank conflicts)
+                    // stage this half's 16 per-edge values as S[edge][feature lane] (row stride 36:
+                    // the stores and the 16-byte row reads below are free of bank conflicts)
 #pragma unroll
-                for (int q = 0; q < 16; ++q) s_w[(hh * 16 + q) * 36 + lane] = rd[q];
-            }
-            // lane k sums edge k of the warp's chunk over the warp's 32 features (the same
-            // pairwise tree as a butterfly over the lanes)
-            __syncwarp();
-            {
-                float v[32];
-#pragma unroll
-                for (int c4 = 0; c4 < 8; ++c4) {
-                    const float4 x = *reinterpret_cast<const float4*>(s_w + lane * 36 + c4 * 4);
-                    v[4 * c4] = x.x; v[4 * c4 + 1] = x.y; v[4 * c4 + 2] = x.z; v[4 * c4 + 3] = x.w;
+                    for (int q = 0; q < 16; ++q) s_w[(hh * 16 + q) * 36 + lane] = rd[q];
                 }
-                ps_s[qd * TE + eb + lane] = tree_sum<32>(v);
+                // lane k sums edge k of the warp's chunk over the warp's 32 features (the same
+                // pairwise tree as a butterfly over the lanes)
+                __syncwarp();
+                {
+                    float v[32];
+#pragma unroll
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 x = *reinterpret_cast<const float4*>(s_w + lane * 36 + c4 * 4);
+                        v[4 * c4] = x.x; v[4 * c4 + 1] = x.y; v[4 * c4 + 2] = x.z; v[4 * c4 + 3] = x.w;
+                    }
+                    ps_s[qd * TE + eb + lane] = tree_sum<32>(v);
+                }
+                __syncwarp();
+                if (!DH) {
+                } else if (kind == 1) {
+                    pf = sf;
+                } else if (kind == 2) {
+                    pf = sf;
+                    pl = sl;
+                    for (int rr = ci.rfirst + 1; rr < ci.rlast; ++rr) a.out[(size_t)rr * FP + f] = 0.f;
+                } else if (c.lrow == c.rfirst) {
+                    pf = c.acc;
+                } else {
+                    pf = c.pf;
+                    pl = c.acc;
+                }
             }
-            __syncwarp();
+            if (DH) {
+                pf_s[ch * 128 + f] = pf;
+                pl_s[ch * 128 + f] = pl;
+            }
         }
         tc_fence_before();
         group_sync(g);          // Q, Q' read out; per-edge partials and the next tile's Gaussians in place
@@ -1026,7 +1081,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];
             a.s_edge[my_g] = a.accumulate_s ? my_so + sv : sv;
         }
-        group_sync(g);          // s_e done with the partials before E1 of the next tile overwrites them
+        if (DH && !(ok = merge_tile<NCH, false>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
+        group_sync(g);          // s_e and the merge done with the partials before E1 of the next tile overwrites them
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
     if (mt == 0) {
@@ -1034,30 +1090,33 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         pend_s[g] = ok ? 0u : pending;
     }
     const bool all_ok = __syncthreads_or(!ok) == 0;
-    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, false);
+    kernel_finish<false>(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, DH);
 }
 
 // ---------------------------------------------------------------------------
 // cutoff masking: per CTA row range, the listed edges with d < r_c, in order;
-// list 1 (the half list) keeps only the edges (i, j) with j > i, in the row
-// ranges of its own partition.  One launch builds both lists (CTAs ncta ..
-// 2 ncta - 1 take the half list), so the two passes share the GPU.
+// list 1 (the half list) keeps only the edges (i, j) with j > i and list 2 (its
+// complement) those with j < i, each in the row ranges of its own partition.
+// One launch builds all three (CTAs k ncta .. (k+1) ncta - 1 take list k), so
+// the passes share the GPU.
 // ---------------------------------------------------------------------------
 struct CompactList {
     const int32_t* part;
-    int32_t *crow, *ccol, *cidx, *ccount;
+    int32_t *crow, *ccol, *cidx, *ccount;   // cidx may be null (the list is not used for s_e)
     float* cdist;
 };
 
 __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__ row_ptr, int ncta,
                                                   const int32_t* __restrict__ erow, const int32_t* __restrict__ col,
                                                   const float4* __restrict__ pos4, Box box, float rc, long long cap,
-                                                  const DevMeta* meta, CompactList full, CompactList half)
+                                                  const DevMeta* meta, CompactList full, CompactList half,
+                                                  CompactList rev)
 {
     pdl_trigger();
     pdl_wait();
-    const bool is_half = (int)blockIdx.x >= ncta;
-    const CompactList L = is_half ? half : full;
+    const int list = (int)blockIdx.x / ncta;      // 0: full, 1: half (j > i), 2: complement (j < i)
+    const bool is_half = list == 1, is_rev = list == 2;
+    const CompactList L = list == 0 ? full : (is_half ? half : rev);
     int32_t* __restrict__ crow = L.crow;
     int32_t* __restrict__ ccol = L.ccol;
     int32_t* __restrict__ cidx = L.cidx;
@@ -1067,7 +1126,7 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
     constexpr int CI = 4;             // consecutive edges per thread and pass
     __shared__ int wcount[32];
     __shared__ int total_s;
-    const int c = is_half ? (int)blockIdx.x - ncta : (int)blockIdx.x;
+    const int c = (int)blockIdx.x - list * ncta;
     const int r0 = part[c], r1 = part[c + 1];
     if (meta->n_edges > cap || r0 >= r1) {
         if (threadIdx.x == 0) ccount[c] = 0;
@@ -1096,7 +1155,8 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
                 float3 v;
                 const float d = edge_distance(pos4[ii[q]], pos4[jj[q]], box, v);
                 dd[q] = d;
-                if (d < rc && d > 0.f && (!is_half || jj[q] > ii[q])) vmask |= 1u << q;
+                if (d < rc && d > 0.f && (!is_half || jj[q] > ii[q]) && (!is_rev || jj[q] < ii[q]))
+                    vmask |= 1u << q;
             }
         }
         // block-wide exclusive scan of the per-thread counts, edge order kept
@@ -1128,7 +1188,7 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
             if ((vmask >> q) & 1u) {
                 crow[k] = ii[q];
                 ccol[k] = jj[q];
-                cidx[k] = (int32_t)(ef + q);
+                if (cidx) cidx[k] = (int32_t)(ef + q);
                 cdist[k] = dd[q];
                 ++k;
             }
@@ -1140,16 +1200,17 @@ __global__ void __launch_bounds__(1024, 2) k_compact(const int32_t* __restrict__
 }
 
 // The full list of the step's edges inside the cutoff and, when forces follow, the
-// half list of the pair-derivative launches
+// half list of the pair-derivative launches and its complement (the dE/dh launches)
 cudaError_t launch_compact(schnet_ctx* c, bool with_half)
 {
     Workspace& w = c->ws;
     const CompactList full{w.part, w.crow, w.ccol, w.cidx, w.ccount, w.cdist};
     const CompactList half{w.part_h, w.crow_h, w.ccol_h, w.cidx_h, w.ccount_h, w.cdist_h};
+    const CompactList rev{w.part_r, w.crow_r, w.ccol_r, nullptr, w.ccount_r, w.cdist_r};
     c->launches += 1;
-    return launch_pdl(k_compact, c->ncta * (with_half ? 2 : 1), 1024, 0, c->s, (const int32_t*)w.row_ptr,
+    return launch_pdl(k_compact, c->ncta * (with_half ? 3 : 1), 1024, 0, c->s, (const int32_t*)w.row_ptr,
                       (int)c->ncta, (const int32_t*)w.erow, (const int32_t*)w.col, (const float4*)w.pos4, c->box,
-                      c->cfg.cutoff, (long long)c->cap, (const DevMeta*)w.meta, full, half);
+                      c->cfg.cutoff, (long long)c->cap, (const DevMeta*)w.meta, full, half, rev);
 }
 
 // ---------------------------------------------------------------------------
@@ -1190,11 +1251,15 @@ static MPArgs make_args(schnet_ctx* c, int layer)
 template <int FMT, int NW, int NX>
 static cudaError_t set_attrs()
 {
-    cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<TE_F, false>());
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_bytes<TE_B, true>());
+    const int sf = (int)smem_bytes<TE_F, false>(), sb = (int)smem_bytes<TE_B, true>();
+    cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, sf);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, sf);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, sb);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, sb);
+    return e;
 }
 
 cudaError_t cfconv_init_attributes()
@@ -1208,17 +1273,32 @@ cudaError_t cfconv_init_attributes()
 
 // operand formats: fp32 weights (fp16 hi+lo weights and activations), fp16 or bf16
 // weights (one weight term, hi+lo activations), fp16 weights with fp16 activations
+template <bool ACC>
 static cudaError_t launch_fwd(schnet_ctx* c, const MPArgs& a)
 {
     const size_t sm = smem_bytes<TE_F, false>();
     if (c->n_xterms == 1)
-        return launch_pdl(k_cfconv_fwd<0, 1, 1>, c->ncta, NT, sm, c->s, a);
+        return launch_pdl(k_cfconv_fwd<0, 1, 1, ACC>, c->ncta, NT, sm, c->s, a);
     else if (c->weight_fmt == 0 && c->n_wterms == 2)
-        return launch_pdl(k_cfconv_fwd<0, 2, 2>, c->ncta, NT, sm, c->s, a);
+        return launch_pdl(k_cfconv_fwd<0, 2, 2, ACC>, c->ncta, NT, sm, c->s, a);
     else if (c->weight_fmt == 0)
-        return launch_pdl(k_cfconv_fwd<0, 1, 2>, c->ncta, NT, sm, c->s, a);
+        return launch_pdl(k_cfconv_fwd<0, 1, 2, ACC>, c->ncta, NT, sm, c->s, a);
     else
-        return launch_pdl(k_cfconv_fwd<1, 1, 2>, c->ncta, NT, sm, c->s, a);
+        return launch_pdl(k_cfconv_fwd<1, 1, 2, ACC>, c->ncta, NT, sm, c->s, a);
+}
+
+template <bool DH>
+static cudaError_t launch_bwd(schnet_ctx* c, const MPArgs& a)
+{
+    const size_t sm = smem_bytes<TE_B, true>();
+    if (c->n_xterms == 1)
+        return launch_pdl(k_cfconv_bwd<0, 1, 1, DH>, c->ncta, NT, sm, c->s, a);
+    else if (c->weight_fmt == 0 && c->n_wterms == 2)
+        return launch_pdl(k_cfconv_bwd<0, 2, 2, DH>, c->ncta, NT, sm, c->s, a);
+    else if (c->weight_fmt == 0)
+        return launch_pdl(k_cfconv_bwd<0, 1, 2, DH>, c->ncta, NT, sm, c->s, a);
+    else
+        return launch_pdl(k_cfconv_bwd<1, 1, 2, DH>, c->ncta, NT, sm, c->s, a);
 }
 
 // m = sum_j h_j (.) W_ij of interaction `layer`
@@ -1227,23 +1307,31 @@ cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
     MPArgs a = make_args(c, layer);
     a.out = c->ws.m;
     c->launches += 1;
-    return launch_fwd(c, a);
+    return launch_fwd<false>(c, a);
 }
 
-// dE/dh_j = sum_i u_i (.) W_ij with u = dE/dm of interaction `layer`: the same
-// segment sum over the symmetric list, with u gathered in place of h
+// The rest of dE/dh_i = sum_j u_j (.) W_ij with u = dE/dm of interaction `layer`:
+// the terms j < i, over the complementary half list (the pair launch formed the
+// terms j > i), added to dh by the forward kernel's segment sum with u gathered
+// in place of h
 cudaError_t launch_cfconv_dh(schnet_ctx* c, int layer)
 {
     MPArgs a = make_args(c, layer);
+    a.crow = c->ws.crow_r;
+    a.ccol = c->ws.ccol_r;
+    a.cdist = c->ws.cdist_r;
+    a.ccount = c->ws.ccount_r;
+    a.part = c->ws.part_r;
     a.h = c->ws.m;
     a.out = c->ws.dh;
     c->launches += 1;
-    return launch_fwd(c, a);
+    return launch_fwd<true>(c, a);
 }
 
 // Pair derivatives of interaction `layer` over the half list, written to s_e of
-// each pair's owning edge (added to the later interactions' when accumulate_s)
-cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s)
+// each pair's owning edge (added to the later interactions' when accumulate_s);
+// with_dh: also the half list's share of dE/dh (the terms j > i), written to dh
+cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s, bool with_dh)
 {
     MPArgs a = make_args(c, layer);
     a.crow = c->ws.crow_h;
@@ -1252,19 +1340,10 @@ cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s)
     a.cdist = c->ws.cdist_h;
     a.ccount = c->ws.ccount_h;
     a.part = c->ws.part_h;
+    a.out = c->ws.dh;
     a.accumulate_s = accumulate_s;
-    const size_t sm = smem_bytes<TE_B, true>();
-    cudaError_t e;
-    if (c->n_xterms == 1)
-        e = launch_pdl(k_cfconv_bwd<0, 1, 1>, c->ncta, NT, sm, c->s, a);
-    else if (c->weight_fmt == 0 && c->n_wterms == 2)
-        e = launch_pdl(k_cfconv_bwd<0, 2, 2>, c->ncta, NT, sm, c->s, a);
-    else if (c->weight_fmt == 0)
-        e = launch_pdl(k_cfconv_bwd<0, 1, 2>, c->ncta, NT, sm, c->s, a);
-    else
-        e = launch_pdl(k_cfconv_bwd<1, 1, 2>, c->ncta, NT, sm, c->s, a);
     c->launches += 1;
-    return e;
+    return with_dh ? launch_bwd<true>(c, a) : launch_bwd<false>(c, a);
 }
 
 }  // namespace schnet

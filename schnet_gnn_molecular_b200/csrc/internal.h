@@ -68,7 +68,7 @@ struct Workspace {
     float4 *pos4, *ref4, *frc4;   // [N]
     // neighbour list
     int32_t *row_ptr, *rowcnt;    // [N+1]
-    int32_t* hcnt;                // [N+1] per-row half-list counts (scratch of the partition)
+    int32_t *hcnt, *rcnt;         // [N+1] per-row counts of the half list and its complement (scratch)
     int32_t *col, *coltmp, *rev, *erow;  // [cap]
     float* s_edge;                // [cap]
     int32_t *crow, *ccol, *cidx;  // [cap] edges with d < r_c, per CTA row range
@@ -79,6 +79,10 @@ struct Workspace {
     float* cdist_h;               // [cap] their distances
     int32_t* ccount_h;            // [ncta]    its per-CTA edge counts
     int32_t* part_h;              // [ncta+1]  and its own row partition
+    int32_t *crow_r, *ccol_r;     // [cap] the complement: edges (i, j), j < i, d < r_c (dE/dh launches)
+    float* cdist_r;               // [cap] their distances
+    int32_t* ccount_r;            // [ncta]
+    int32_t* part_r;              // [ncta+1]
     // cell list
     int32_t *cell_of, *cell_atoms;       // [N]  caller order
     int32_t* cell_slot;                  // [N]  cell of each slot
@@ -198,7 +202,7 @@ cudaError_t launch_aw_bwd(schnet_ctx* c, int layer);
 cudaError_t launch_compact(schnet_ctx* c, bool with_half);
 cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer);
 cudaError_t launch_cfconv_dh(schnet_ctx* c, int layer);
-cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s);
+cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s, bool with_dh);
 cudaError_t cfconv_init_attributes();
 cudaError_t atomwise_init_attributes();
 

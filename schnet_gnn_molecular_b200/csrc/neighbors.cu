@@ -474,12 +474,14 @@ __global__ void k_partition(int n, int ncta, const int32_t* __restrict__ row_ptr
 
 // Per row, the edges the tensor-core kernels will carry at the build's positions:
 // those inside the cutoff (cnt), and of them those with j > i (cnt_half, the half
-// list that visits each unordered pair once).  The distance is the masking pass's
-// own expression, so the counts equal what it keeps at these positions; the row
-// partitions balance them.  One warp per row.
+// list that visits each unordered pair once) and those with j < i (cnt_rev, its
+// complement).  The distance is the masking pass's own expression, so the counts
+// equal what it keeps at these positions; the row partitions balance them.  One
+// warp per row.
 __global__ void k_cut_counts(int n, const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
                              const float4* __restrict__ pos4, const Box box, float rc, long long cap,
-                             const DevMeta* meta, int32_t* __restrict__ cnt, int32_t* __restrict__ cnt_half)
+                             const DevMeta* meta, int32_t* __restrict__ cnt, int32_t* __restrict__ cnt_half,
+                             int32_t* __restrict__ cnt_rev)
 {
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -507,6 +509,7 @@ __global__ void k_cut_counts(int n, const int32_t* __restrict__ row_ptr, const i
         if (lane == 0) {
             cnt[i] = c;
             cnt_half[i] = ch;
+            cnt_rev[i] = c - ch;
         }
     }
 }
@@ -558,14 +561,17 @@ cudaError_t launch_build_neighbors(schnet_ctx* c, const float* d_pos)
     // the row partitions of the full and the half list, balanced on the edges inside the
     // cutoff at the build's positions (rowcnt is free scratch once the list is built)
     k_cut_counts<<<c->nsm * 8, 256, 0, c->s>>>(N, w.row_ptr, w.col, w.pos4, c->box, c->cfg.cutoff, c->cap, w.meta,
-                                               w.rowcnt, w.hcnt);
+                                               w.rowcnt, w.hcnt, w.rcnt);
     c->launches += 5;
     if ((err = scan_exclusive(c, w.rowcnt, N, w.rowcnt, nullptr)) != cudaSuccess) return err;   // in place
     if ((err = scan_exclusive(c, w.hcnt, N, w.hcnt, nullptr)) != cudaSuccess) return err;
-    k_partition<<<(c->ncta + 1 + 127) / 128, 128, 0, c->s>>>(N, c->ncta, w.rowcnt, c->cap, w.meta, w.part);
-    k_partition<<<(c->ncta + 1 + 127) / 128, 128, 0, c->s>>>(N, c->ncta, w.hcnt, c->cap, w.meta, w.part_h);
+    if ((err = scan_exclusive(c, w.rcnt, N, w.rcnt, nullptr)) != cudaSuccess) return err;
+    const int npb = (c->ncta + 1 + 127) / 128;
+    k_partition<<<npb, 128, 0, c->s>>>(N, c->ncta, w.rowcnt, c->cap, w.meta, w.part);
+    k_partition<<<npb, 128, 0, c->s>>>(N, c->ncta, w.hcnt, c->cap, w.meta, w.part_h);
+    k_partition<<<npb, 128, 0, c->s>>>(N, c->ncta, w.rcnt, c->cap, w.meta, w.part_r);
     cudaMemcpyAsync(w.ref4, w.pos4, sizeof(float4) * N, cudaMemcpyDeviceToDevice, c->s);
-    c->launches += 2;
+    c->launches += 3;
     return cudaGetLastError();
 }
 

@@ -551,27 +551,18 @@ __device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslo
     return tmem;
 }
 
-// After pdl_wait: this CTA's row range [r0, r1) (empty when the list overflowed
-// its capacity); a CTA without rows releases its tensor memory and returns false.
-__device__ __forceinline__ bool kernel_rows(const MPArgs& a, uint32_t tmem, Carry* cy, int& r0, int& r1)
+// This CTA's row range [r0, r1), empty when the list overflowed its capacity.
+// Read before pdl_wait: the partitions and the edge count are written only by the
+// neighbour build, whose kernels are launched without programmatic serialization,
+// so they have completed before any kernel of a step or evaluation starts.  A CTA
+// without rows returns at once, before it allocates tensor memory.
+__device__ __forceinline__ void kernel_rows(const MPArgs& a, int& r0, int& r1)
 {
     r0 = r1 = 0;
     if (a.meta->n_edges <= a.cap) {
         r0 = a.part[blockIdx.x];
         r1 = a.part[blockIdx.x + 1];
     }
-    if (r0 >= r1) {
-        tc_fence_before();
-        __syncthreads();
-        if ((threadIdx.x >> 5) == 0) {
-            tc_fence_after();
-            tmem_dealloc(tmem, 512);
-        }
-        return false;
-    }
-    if (threadIdx.x == 0) cy->cur[1] = r0;   // tile 0 reads the carry of "tile -1"
-    __syncthreads();
-    return true;
 }
 
 // Common epilogue: the carried row is complete; rows after it without edges are zero
@@ -688,10 +679,13 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     const int f = qd * 32 + lane;                   // this thread's output feature
 
     pdl_trigger();
-    const uint32_t tmem = kernel_setup(a, tslot, bars, cy);
-    pdl_wait();                                     // the previous kernel's results from here on
     int r0, r1;
-    if (!kernel_rows(a, tmem, cy, r0, r1)) return;
+    kernel_rows(a, r0, r1);
+    if (r0 >= r1) return;
+    const uint32_t tmem = kernel_setup(a, tslot, bars, cy);
+    if (threadIdx.x == 0) cy->cur[1] = r0;         // tile 0 reads the carry of "tile -1"
+    pdl_wait();                                     // the previous kernel's results from here on
+    __syncthreads();
     const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     uint8_t* rbf = smem + SM_RBF + g * 2 * RBF_TERM;
     uint8_t* act = smem + SM_ACT + g * 2 * ACT_TERM;
@@ -863,10 +857,13 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     const int f = qd * 32 + lane;
 
     pdl_trigger();
-    const uint32_t tmem = kernel_setup(a, tslot, bars, cy);
-    pdl_wait();                                     // the previous kernel's results from here on
     int r0, r1;
-    if (!kernel_rows(a, tmem, cy, r0, r1)) return;
+    kernel_rows(a, r0, r1);
+    if (r0 >= r1) return;
+    const uint32_t tmem = kernel_setup(a, tslot, bars, cy);
+    if (threadIdx.x == 0) cy->cur[1] = r0;         // tile 0 reads the carry of "tile -1"
+    pdl_wait();                                     // the previous kernel's results from here on
+    __syncthreads();
     const long long e0 = a.row_ptr[r0], e1 = e0 + a.ccount[blockIdx.x];
     uint8_t* rbf = smem + SM_RBF + g * 2 * RBF_TERM;
     uint8_t* act = smem + SM_ACT + g * 2 * ACT_TERM;

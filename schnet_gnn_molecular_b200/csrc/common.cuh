@@ -35,9 +35,10 @@ __device__ __forceinline__ void set_flag(DevMeta* meta, unsigned int bit)
 // Programmatic dependent launch (kernels launched with launch_pdl): the next
 // kernel on the stream may be scheduled once every CTA of this one has called
 // pdl_trigger; pdl_wait blocks until the previous kernel has completed and its
-// writes are visible.  Before pdl_wait a kernel touches only constant data
-// (weights, its own shared and tensor memory).  Both are no-ops in a kernel
-// launched without the attribute.
+// writes are visible.  Before pdl_wait a kernel touches only data no kernel of
+// the step writes (weights, the neighbour build's partitions and edge count, its
+// own shared and tensor memory).  Both are no-ops in a kernel launched without
+// the attribute.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 

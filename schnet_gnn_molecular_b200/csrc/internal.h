@@ -118,9 +118,11 @@ struct GraphKey {
 
 // Launch on `s` with programmatic stream serialization: the kernel's CTAs may be
 // scheduled while the previous kernel on the stream is still finishing, run
-// their prologue on constant data, and wait in pdl_wait for its results.  Every
-// kernel launched this way calls pdl_wait before reading anything an earlier
-// kernel wrote and before writing anything an earlier kernel reads.
+// their prologue on data no kernel of the step writes, and wait in pdl_wait for
+// its results.  Every kernel launched this way calls pdl_wait before reading
+// anything an earlier kernel of the step wrote and before writing anything an
+// earlier kernel reads.  The neighbour build's kernels are launched without it,
+// so they have completed before the next kernel starts.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
                               Args... args)

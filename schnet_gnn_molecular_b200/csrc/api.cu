@@ -171,7 +171,7 @@ size_t carve(const Derived& d, uint8_t* base, Workspace& w, size_t* wbegin = nul
     w.x = cv.take<float>(N * FP);
     w.h = cv.take<float>(L * N * FP);
     w.q = cv.take<float>(L * N * FP);
-    w.m = cv.take<float>(N * FP); w.g = cv.take<float>(N * FP); w.dh = cv.take<float>(N * FP);
+    w.m = cv.take<float>(N * FP); w.g = cv.take<float>(N * FP); w.dh = cv.take<float>(N * FP); w.dh2 = cv.take<float>(N * FP);
     w.pr = cv.take<float>(N * HP); w.eps = cv.take<float>(N); w.ke = cv.take<float>(N);
     w.partial = cv.take<double>(d.nchunk);
     w.epot = cv.take<double>(R); w.ekin = cv.take<double>(R);
@@ -540,8 +540,9 @@ cudaError_t schnet::launch_energy_forces(schnet_ctx* c, const int32_t* types, do
     for (int l = c->L - 1; l >= 0; --l) {
         // pair derivatives over the half list (one edge per unordered pair) and, but for
         // interaction 0 (whose dE/dh would only reach the embedding, which forces do not
-        // need), the half list's terms of dE/dh; the complementary list adds the rest, and
-        // the atom-wise backward carries the gradient to the earlier interactions
+        // need), the half list's terms of dE/dh; the complementary list's launch forms the
+        // rest, and the atom-wise backward adds the two and carries the gradient to the
+        // earlier interactions
         SCHNET_TIMED(SCHNET_KERNEL_CFCONV_BWD, launch_cfconv_pair(c, l, l < c->L - 1 ? 1 : 0, l > 0));
         if (l > 0) {
             SCHNET_TIMED(SCHNET_KERNEL_CFCONV_DH, launch_cfconv_dh(c, l));

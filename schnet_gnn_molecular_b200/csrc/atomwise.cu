@@ -41,7 +41,8 @@ struct AWArgs {
     const uint8_t* img[3];        // the layers' packed A images (hi term, then lo term)
     const float* sc[3];           // their per-row scales [FP]
     const float *bo1, *bo2, *c1, *R2, *c2;
-    float *x, *h_out, *q, *m, *g, *dh, *pr, *eps;
+    float *x, *h_out, *q, *m, *g, *pr, *eps;
+    const float *dh, *dh2;        // backward: dE/dh as two parts (half list, complement) that add up
     const float* q_in;            // backward: q of the layer whose u is formed
     DevMeta* meta;
 };
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
             for (int q = 0; q < 32; ++q) v[q] = (f < HP && row_ok(q)) ? sigmoidf(__ldg(a.pr + at(q, HP))) * r2 : 0.f;
         } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) v[q] = row_ok(q) ? __ldg(a.dh + at(q, FP)) : 0.f;
+            for (int q = 0; q < 32; ++q) v[q] = row_ok(q) ? __ldg(a.dh + at(q, FP)) + __ldg(a.dh2 + at(q, FP)) : 0.f;
         }
         s = tile_scale(v, wmax, inv);
         stage_b(B, v, s, c, f);
@@ -325,7 +326,7 @@ static AWArgs aw_args(schnet_ctx* c, int mode, int layer)
     a.ntiles = (c->N + ATILE - 1) / ATILE;
     a.bo1 = w.bo1 + layer * FP; a.bo2 = w.bo2 + layer * FP;
     a.c1 = w.c1; a.R2 = w.R2; a.c2 = w.c2;
-    a.x = w.x; a.q = w.q + (size_t)layer * c->N * FP; a.m = w.m; a.g = w.g; a.dh = w.dh; a.pr = w.pr;
+    a.x = w.x; a.q = w.q + (size_t)layer * c->N * FP; a.m = w.m; a.g = w.g; a.dh = w.dh; a.dh2 = w.dh2; a.pr = w.pr;
     a.eps = w.eps; a.meta = w.meta;
     int ids[3] = {0, 0, 0};
     if (mode == AW_FWD) {

@@ -13,12 +13,11 @@
 //   flash message passing + flash aggregation (How): cutoff masking, gather of
 //     h_j, filter product and the CSR segment sum m_i = sum_j h_j (.) W_ij,
 //     accumulated in registers, no atomics, no edge tensor in HBM.
-// The backward kernel recomputes W and its distance derivative W' by forward-
-// mode tangents and produces dE/dh_j (segment sum over the symmetric list) and
-// the per-edge scalar s_e = sum_f W'_f u_i,f h_j,f (the edge's share of dE/dd);
-// for the first interaction, whose dE/dh only feeds the embedding's gradient,
-// it visits each unordered pair once (the half list, exploiting W_ij = W_ji)
-// and produces the pair's whole derivative sum_f W'_f (u_i h_j + u_j h_i).
+// The backward kernel visits each unordered pair once (the half list, exploiting
+// W_ij = W_ji), recomputes W and its distance derivative W' by forward-mode
+// tangents, and produces the pair's derivative sum_f W'_f (u_i h_j + u_j h_i)
+// and the half list's terms of dE/dh_i = sum_j W_ij (.) u_j; the forward kernel
+// over the complementary list adds the other terms.
 //
 // Tile orientation: the GEMMs are computed transposed, D[f][e] = W^T[f][k] B[e][k],
 // so TMEM lane = output feature and TMEM column = edge.  Each epilogue thread
@@ -374,19 +373,15 @@ struct ChunkSeg {
     float acc, pf;
 };
 
-// A completed row's sum into out (ACC: added to what an earlier launch left there),
-// and the rows between two rows with edges: zero, or left as they are with ACC.
-template <bool ACC>
+// A completed row's sum into out, and zeros for the rows without edges between two
+// rows with edges (every row of the CTA's range is written).
 __device__ __forceinline__ void put_row(float* __restrict__ out, int row, int f, float v)
 {
-    if (ACC) out[(size_t)row * FP + f] += v;
-    else out[(size_t)row * FP + f] = v;
+    out[(size_t)row * FP + f] = v;
 }
-template <bool ACC>
 __device__ __forceinline__ void zero_rows(float* __restrict__ out, int from, int to, int f)
 {
-    if (!ACC)
-        for (int rr = from; rr < to; ++rr) out[(size_t)rr * FP + f] = 0.f;
+    for (int rr = from; rr < to; ++rr) out[(size_t)rr * FP + f] = 0.f;
 }
 
 __device__ __forceinline__ void seg_begin(ChunkSeg& c, int rfirst)
@@ -397,13 +392,12 @@ __device__ __forceinline__ void seg_begin(ChunkSeg& c, int rfirst)
     c.pf = 0.f;
 }
 
-template <bool ACC>
 __device__ __forceinline__ void seg_row(ChunkSeg& c, int row, float* __restrict__ out, int f)
 {
     if (row != c.lrow) {
         if (c.lrow == c.rfirst) c.pf = c.acc;
-        else put_row<ACC>(out, c.lrow, f, c.acc);
-        zero_rows<ACC>(out, c.lrow + 1, row, f);
+        else put_row(out, c.lrow, f, c.acc);
+        zero_rows(out, c.lrow + 1, row, f);
         c.lrow = row;
         c.acc = 0.f;
     }
@@ -412,7 +406,7 @@ __device__ __forceinline__ void seg_row(ChunkSeg& c, int row, float* __restrict_
 // In-order merge of a tile's chunk partials into the carried row (threads of
 // the group with feature f = group thread index < 128): rows the carry leaves
 // are complete and written out, with zeros for edge-less rows in between.
-template <int NCH, bool ACC>
+template <int NCH>
 __device__ __forceinline__ void merge_chunks(const ChunkInfo* ci, const float* pf, const float* pl, int ne, int f,
                                              float* __restrict__ out, int& cur, float& acc)
 {
@@ -424,13 +418,13 @@ __device__ __forceinline__ void merge_chunks(const ChunkInfo* ci, const float* p
         if (rfirst == cur) {
             acc += v;
         } else {
-            put_row<ACC>(out, cur, f, acc);
-            zero_rows<ACC>(out, cur + 1, rfirst, f);
+            put_row(out, cur, f, acc);
+            zero_rows(out, cur + 1, rfirst, f);
             cur = rfirst;
             acc = v;
         }
         if (rlast != rfirst) {
-            put_row<ACC>(out, cur, f, acc);
+            put_row(out, cur, f, acc);
             cur = rlast;
             acc = pl[c * 128 + f];
         }
@@ -439,7 +433,7 @@ __device__ __forceinline__ void merge_chunks(const ChunkInfo* ci, const float* p
 
 // Merge step of tile t by its group: wait for tile t-1's merge, fold this
 // tile's partials into the carry, hand the carry on.  Returns false on timeout.
-template <int NCH, bool ACC>
+template <int NCH>
 __device__ __forceinline__ bool merge_tile(Carry* cy, uint64_t* tok, const ChunkInfo* ci, const float* pf,
                                            const float* pl, int ne, int t, float* __restrict__ out, DevMeta* meta,
                                            int g, int mt)
@@ -448,7 +442,7 @@ __device__ __forceinline__ bool merge_tile(Carry* cy, uint64_t* tok, const Chunk
     if (mt < 128) {
         int cur = cy->cur[(t + 1) & 1];      // written by tile t-1 (or the initial row)
         float acc = cy->acc[mt];
-        merge_chunks<NCH, ACC>(ci, pf, pl, ne, mt, out, cur, acc);
+        merge_chunks<NCH>(ci, pf, pl, ne, mt, out, cur, acc);
         cy->acc[mt] = acc;
         if (mt == 0) cy->cur[t & 1] = cur;
         mbar_arrive(tok);
@@ -476,7 +470,7 @@ __device__ __forceinline__ float tree_sum(float (&v)[N])
 // rows strictly between them are written as zeros).  Three or more rows: the
 // serial segmented sum (rows read from the tile's global row list) writes the
 // inner rows out.
-template <int N, bool ACC>
+template <int N>
 __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_t* __restrict__ rows_g, int eb,
                                                int ne, float (&t)[N], float* __restrict__ out, int f, float& pf,
                                                float& pl)
@@ -495,7 +489,7 @@ __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_
             }
             pf = tree_sum<N>(t);
             pl = tree_sum<N>(u);
-            zero_rows<ACC>(out, ci.rfirst + 1, ci.rlast, f);
+            zero_rows(out, ci.rfirst + 1, ci.rlast, f);
         }
         return;
     }
@@ -505,16 +499,16 @@ __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_
     for (int q = 0; q < N; ++q) {
         const int e = eb + q;
         if (e >= ne) break;
-        seg_row<ACC>(c, __ldg(rows_g + e), out, f);
+        seg_row(c, __ldg(rows_g + e), out, f);
         c.acc += t[q];
     }
     if (c.lrow == c.rfirst) { pf = c.acc; pl = 0.f; } else { pf = c.pf; pl = c.acc; }
 }
 
 // Common prologue of both kernels, on constant data only (it runs before
-// pdl_wait): TMEM allocation, mbarriers, the filter weights into TMEM (warps
-// 0-3, one output channel per lane), the zero carry.  Returns the TMEM base
-// address.
+// pdl_wait): TMEM allocation, mbarriers, the filter weights into TMEM (one output
+// channel per lane; the six 32-column row loads of each lane quadrant spread over
+// the quadrant's four warps), the zero carry.  Returns the TMEM base address.
 __device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslot, uint64_t* bars, Carry* cy)
 {
     const int warp = threadIdx.x >> 5;
@@ -534,15 +528,15 @@ __device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslo
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot;
-    if (warp < 4) {
-        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-        const int f = threadIdx.x;
-        weights_to_tmem(tl, TM_W1H, a.img, f, 0);
-        weights_to_tmem(tl, TM_W1L, a.img + W1_IMG, f, 0);
-        weights_to_tmem(tl, TM_W2H, a.img + 2 * W1_IMG, f, 0);
-        weights_to_tmem(tl, TM_W2H, a.img + 2 * W1_IMG, f, 1);
-        weights_to_tmem(tl, TM_W2L, a.img + 2 * W1_IMG + W2_IMG, f, 0);
-        weights_to_tmem(tl, TM_W2L, a.img + 2 * W1_IMG + W2_IMG, f, 1);
+    {
+        const int qd = warp & 3;                      // the lane quadrant this warp may access
+        const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+        const int f = qd * 32 + (threadIdx.x & 31);
+        for (int job = warp >> 2; job < 6; job += NT / 128) {
+            const uint32_t col = job == 0 ? TM_W1H : job == 1 ? TM_W1L : job < 4 ? TM_W2H : TM_W2L;
+            const uint8_t* term = a.img + (job == 0 ? 0 : job == 1 ? W1_IMG : job < 4 ? 2 * W1_IMG : 2 * W1_IMG + W2_IMG);
+            weights_to_tmem(tl, col, term, f, job < 2 ? 0 : job & 1);
+        }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
@@ -566,8 +560,7 @@ __device__ __forceinline__ void kernel_rows(const MPArgs& a, int& r0, int& r1)
 }
 
 // Common epilogue: the carried row is complete; rows after it without edges are zero
-// (left as they are with ACC; nothing to write when the kernel produces no per-row output).
-template <bool ACC>
+// (nothing to write when the kernel produces no per-row output).
 __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r1, float* __restrict__ out, bool ok,
                                               uint64_t* bars, const uint32_t* phases, const uint32_t* pending,
                                               uint32_t tmem, bool write_out = true)
@@ -576,9 +569,9 @@ __device__ __forceinline__ void kernel_finish(const Carry* cy, int ntiles, int r
     if (ok && write_out) {
         if (threadIdx.x < FP) {
             const int cur = cy->cur[(ntiles + 1) & 1];
-            if (ntiles > 0) put_row<ACC>(out, cur, threadIdx.x, cy->acc[threadIdx.x]);
-            else zero_rows<ACC>(out, cur, cur + 1, threadIdx.x);
-            zero_rows<ACC>(out, cur + 1, r1, threadIdx.x);
+            if (ntiles > 0) put_row(out, cur, threadIdx.x, cy->acc[threadIdx.x]);
+            else zero_rows(out, cur, cur + 1, threadIdx.x);
+            zero_rows(out, cur + 1, r1, threadIdx.x);
         }
     } else if ((threadIdx.x & (GT - 1)) == 0) {
         // drain: give the group's in-flight MMAs a bounded chance to retire before freeing TMEM
@@ -620,7 +613,7 @@ __device__ __forceinline__ void fwd_e1(uint32_t tP, float s1L, float b1L, uint8_
 }
 
 // forward epilogue 2 for chunk cc: W = f_c (s2 ln2 Q + b2), terms h_j W, chunk partials
-template <int TE, bool ACC>
+template <int TE>
 __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* tm, const int32_t* rows_g, int cc,
                                        int ne, float s2L, float b2, const float (&hv)[32], float* __restrict__ out,
                                        int f, float& pf, float& pl)
@@ -640,7 +633,7 @@ __device__ __forceinline__ void fwd_e2(uint32_t tQ, const TileMeta<TE, false>* t
         r[q] = v.x;
         r[q + 1] = v.y;
     }
-    chunk_partials<32, ACC>(tm->c[cc], rows_g, eb, ne, r, out, f, pf, pl);
+    chunk_partials<32>(tm->c[cc], rows_g, eb, ne, r, out, f, pf, pl);
 }
 
 // Issue GEMM1 of a tile (group g): D = W1^T [B rows of the group's GEMM1 operand]
@@ -659,7 +652,7 @@ __device__ __forceinline__ void issue_gemm1(uint32_t tmem, uint32_t dacc, uint32
 // t+2 (into the group's own GEMM1 operand and second metadata buffer) and the
 // first gather under GEMM2 -> E2 -> issue GEMM1(t+2) (by warp 4) -> merge under GEMM1(t+2)
 // (warps 0-3).
-template <int FMT, int NW, int NX, bool ACC>
+template <int FMT, int NW, int NX>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {
     constexpr int TE = TE_F;
@@ -756,7 +749,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
             const int cc = ch * 2 + c2;
             if (c2 == 1) gather<32>(h_f, tm->col, cc * 32, hv);
             float pf, pl;
-            fwd_e2<TE, ACC>(tA + c2 * 32, tm, rows_g, cc, ne, s2L, b2, hv, a.out, f, pf, pl);
+            fwd_e2<TE>(tA + c2 * 32, tm, rows_g, cc, ne, s2L, b2, hv, a.out, f, pf, pl);
             pf_s[cc * 128 + f] = pf;
             pl_s[cc * 128 + f] = pl;
         }
@@ -766,7 +759,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         // thread blocks while the tensor core's queue is full)
         if (next && mt == 128) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
-        if (!(ok = merge_tile<NCH, ACC>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
+        if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
         group_sync(g);          // merge done with the partials before E1 of the next tile overwrites them
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
@@ -775,7 +768,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         pend_s[g] = ok ? 0u : pending;
     }
     const bool all_ok = __syncthreads_or(!ok) == 0;
-    kernel_finish<ACC>(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem);
+    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem);
 }
 
 // ---------------------------------------------------------------------------
@@ -829,14 +822,15 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
 // Backward of one interaction.  The pair derivative
 // dE/dd_ij = D_ij = sum_f W'_f(d_ij) (u_i,f h_j,f + u_j,f h_i,f) is the same for
 // (i, j) and (j, i) because W_ij = W_ji: the launch runs over one edge per
-// unordered pair (the half list: edges (i, j) with j > i, in rows balanced by
-// their own partition) and writes (adds, for the later interactions' sums) D_ij
-// to s_e of that edge; the force assembly reads each pair's value from its
-// owning edge, so both atoms receive it.  With DH (every interaction but the
+// unordered pair (the half list: the edges (i, j) that own their pair, in rows
+// balanced by their own partition) and writes (adds, for the later interactions'
+// sums) D_ij to s_e of that edge; the force assembly reads each pair's value from
+// its owning edge, so both atoms receive it.  With DH (every interaction but the
 // first, whose dE/dh would only reach the embedding) the same tiles also form
 // row i's share of dE/dh_i = sum_j W_ij (.) u_j over its half-list edges, a
-// segment sum in registers written to out like the forward's; the other half
-// (j < i) is the forward kernel over the complementary list, adding to out.
+// segment sum in registers written to out like the forward's; the other terms
+// (the complement's edges) come from the forward kernel over the complementary
+// list, in a second buffer.
 template <int FMT, int NW, int NX, bool DH>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
 {
@@ -943,6 +937,15 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         float uv[16], hv[16];
         gather<16>(u_f, tm->col, eb, uv);
         gather<16>(h_f, tm->col, eb, hv);
+        // u and h of the chunk's first and last rows, shared by all its edges
+        float u_first = 0.f, u_last = 0.f, h_first = 0.f, h_last = 0.f;
+        if (eb < ne) {
+            const int rf = tm->c[ch].rfirst, rl = tm->c[ch].rlast;
+            u_first = __ldg(u_f + (size_t)rf * FP);
+            u_last = __ldg(u_f + (size_t)rl * FP);
+            h_first = __ldg(h_f + (size_t)rf * FP);
+            h_last = __ldg(h_f + (size_t)rl * FP);
+        }
         if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM2(t) done
         pending = 0;
         // epilogue 2: W = f_c z, W' = f_c' z + f_c z' (z = s2 ln2 Q + b2, z' = s2 Q'); per edge the
@@ -955,10 +958,6 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                 // 1: one row in the chunk; 2: two rows (the first a prefix); 3: a third row
                 // occurs, rows read per edge
                 const int kind = ci.other ? 3 : (ci.rfirst == ci.rlast ? 1 : 2);
-                const float u_first = __ldg(u_f + (size_t)ci.rfirst * FP);
-                const float u_last = __ldg(u_f + (size_t)ci.rlast * FP);
-                const float h_first = __ldg(h_f + (size_t)ci.rfirst * FP);
-                const float h_last = __ldg(h_f + (size_t)ci.rlast * FP);
                 float u_row = u_first, h_row = h_first;
                 float sf = 0.f, sl = 0.f;
                 ChunkSeg c;
@@ -1018,7 +1017,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
                             if (e < ne) {
                                 const int row = __ldg(rows_g + e);
                                 if (row != c.lrow) {
-                                    if (DH) seg_row<false>(c, row, a.out, f);
+                                    if (DH) seg_row(c, row, a.out, f);
                                     else c.lrow = row;
                                     u_row = __ldg(u_f + (size_t)row * FP);
                                     h_row = __ldg(h_f + (size_t)row * FP);
@@ -1078,7 +1077,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];
             a.s_edge[my_g] = a.accumulate_s ? my_so + sv : sv;
         }
-        if (DH && !(ok = merge_tile<NCH, false>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
+        if (DH && !(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
         group_sync(g);          // s_e and the merge done with the partials before E1 of the next tile overwrites them
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
@@ -1087,13 +1086,13 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         pend_s[g] = ok ? 0u : pending;
     }
     const bool all_ok = __syncthreads_or(!ok) == 0;
-    kernel_finish<false>(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, DH);
+    kernel_finish(cy, ntiles, r1, a.out, all_ok, bars, phases_s, pend_s, tmem, DH);
 }
 
 // ---------------------------------------------------------------------------
 // cutoff masking: per CTA row range, the listed edges with d < r_c, in order;
-// list 1 (the half list) keeps only the edges (i, j) with j > i and list 2 (its
-// complement) those with j < i, each in the row ranges of its own partition.
+// list 1 (the half list) keeps only the edges that own their pair and list 2 (its
+// complement) the others, each in the row ranges of its own partition.
 // One launch builds all three (CTAs k ncta .. (k+1) ncta - 1 take list k), so
 // the passes share the GPU.
 // ---------------------------------------------------------------------------
@@ -1111,7 +1110,7 @@ __global__ void __launch_bounds__(512, 4) k_compact(const int32_t* __restrict__ 
 {
     pdl_trigger();
     pdl_wait();
-    const int list = (int)blockIdx.x / ncta;      // 0: full, 1: half (j > i), 2: complement (j < i)
+    const int list = (int)blockIdx.x / ncta;      // 0: full, 1: half (owning edges), 2: complement
     const bool is_half = list == 1, is_rev = list == 2;
     const CompactList L = list == 0 ? full : (is_half ? half : rev);
     int32_t* __restrict__ crow = L.crow;
@@ -1152,7 +1151,7 @@ __global__ void __launch_bounds__(512, 4) k_compact(const int32_t* __restrict__ 
                 float3 v;
                 const float d = edge_distance(pos4[ii[q]], pos4[jj[q]], box, v);
                 dd[q] = d;
-                if (d < rc && d > 0.f && (!is_half || jj[q] > ii[q]) && (!is_rev || jj[q] < ii[q]))
+                if (d < rc && d > 0.f && (!is_half || owns_pair(ii[q], jj[q])) && (!is_rev || !owns_pair(ii[q], jj[q])))
                     vmask |= 1u << q;
             }
         }
@@ -1250,9 +1249,7 @@ template <int FMT, int NW, int NX>
 static cudaError_t set_attrs()
 {
     const int sf = (int)smem_bytes<TE_F, false>(), sb = (int)smem_bytes<TE_B, true>();
-    cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, sf);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, sf);
+    cudaError_t e = cudaFuncSetAttribute(k_cfconv_fwd<FMT, NW, NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, sf);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(k_cfconv_bwd<FMT, NW, NX, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, sb);
     if (e == cudaSuccess)
@@ -1271,18 +1268,17 @@ cudaError_t cfconv_init_attributes()
 
 // operand formats: fp32 weights (fp16 hi+lo weights and activations), fp16 or bf16
 // weights (one weight term, hi+lo activations), fp16 weights with fp16 activations
-template <bool ACC>
 static cudaError_t launch_fwd(schnet_ctx* c, const MPArgs& a)
 {
     const size_t sm = smem_bytes<TE_F, false>();
     if (c->n_xterms == 1)
-        return launch_pdl(k_cfconv_fwd<0, 1, 1, ACC>, c->ncta, NT, sm, c->s, a);
+        return launch_pdl(k_cfconv_fwd<0, 1, 1>, c->ncta, NT, sm, c->s, a);
     else if (c->weight_fmt == 0 && c->n_wterms == 2)
-        return launch_pdl(k_cfconv_fwd<0, 2, 2, ACC>, c->ncta, NT, sm, c->s, a);
+        return launch_pdl(k_cfconv_fwd<0, 2, 2>, c->ncta, NT, sm, c->s, a);
     else if (c->weight_fmt == 0)
-        return launch_pdl(k_cfconv_fwd<0, 1, 2, ACC>, c->ncta, NT, sm, c->s, a);
+        return launch_pdl(k_cfconv_fwd<0, 1, 2>, c->ncta, NT, sm, c->s, a);
     else
-        return launch_pdl(k_cfconv_fwd<1, 1, 2, ACC>, c->ncta, NT, sm, c->s, a);
+        return launch_pdl(k_cfconv_fwd<1, 1, 2>, c->ncta, NT, sm, c->s, a);
 }
 
 template <bool DH>
@@ -1305,13 +1301,14 @@ cudaError_t launch_cfconv_fwd(schnet_ctx* c, int layer)
     MPArgs a = make_args(c, layer);
     a.out = c->ws.m;
     c->launches += 1;
-    return launch_fwd<false>(c, a);
+    return launch_fwd(c, a);
 }
 
 // The rest of dE/dh_i = sum_j u_j (.) W_ij with u = dE/dm of interaction `layer`:
-// the terms j < i, over the complementary half list (the pair launch formed the
-// terms j > i), added to dh by the forward kernel's segment sum with u gathered
-// in place of h
+// the terms over the complementary list, the edges that do not own their pair
+// (the pair launch formed the half list's terms in dh), written to dh2 by the
+// forward kernel's segment sum with u gathered in place of h; the atom-wise
+// backward adds the two
 cudaError_t launch_cfconv_dh(schnet_ctx* c, int layer)
 {
     MPArgs a = make_args(c, layer);
@@ -1321,14 +1318,14 @@ cudaError_t launch_cfconv_dh(schnet_ctx* c, int layer)
     a.ccount = c->ws.ccount_r;
     a.part = c->ws.part_r;
     a.h = c->ws.m;
-    a.out = c->ws.dh;
+    a.out = c->ws.dh2;
     c->launches += 1;
-    return launch_fwd<true>(c, a);
+    return launch_fwd(c, a);
 }
 
 // Pair derivatives of interaction `layer` over the half list, written to s_e of
 // each pair's owning edge (added to the later interactions' when accumulate_s);
-// with_dh: also the half list's share of dE/dh (the terms j > i), written to dh
+// with_dh: also the half list's share of dE/dh (its edges' terms), written to dh
 cudaError_t launch_cfconv_pair(schnet_ctx* c, int layer, int accumulate_s, bool with_dh)
 {
     MPArgs a = make_args(c, layer);

@@ -161,6 +161,18 @@ __device__ __forceinline__ float edge_distance(float4 pi, float4 pj, const Box& 
     return sqrtf(v.x * v.x + v.y * v.y + v.z * v.z);
 }
 
+// Which of the two edges (i, j) and (j, i) of an unordered pair owns it (carries
+// the pair in the half list and its derivative in s_e): (i, j) when i and j differ
+// in parity and j > i, or share it and j < i.  Exactly one of the two edges
+// qualifies, and each row owns about half of its neighbours wherever it sits in
+// the atom order (owning the pairs with j > i would give the early rows nearly all
+// of theirs and the late rows almost none), so the rows of the half list and of
+// its complement are evenly long.
+__device__ __forceinline__ bool owns_pair(int i, int j)
+{
+    return ((i ^ j) & 1) ? j > i : j < i;
+}
+
 // ---------------------------------------------------------------------------
 // shared-memory / mbarrier / tcgen05 wrappers (sm_100a)
 // ---------------------------------------------------------------------------

@@ -1,7 +1,7 @@
 // Forces from the per-edge scalars of the backward pass, and the Langevin /
 // velocity-Verlet update of many replicas at once.
 //
-// Forces: the backward kernels leave, on the owning edge e = (i, j), j > i, of
+// Forces: the backward kernels leave, on the owning edge e = (i, j) (owns_pair), of
 // every pair within the cutoff, its derivative dE/dd_ij summed over the
 // interactions (the half list visits each pair once); and
 // F_i = sum_{e in row i} dE/dd_ij (r_j - r_i) / d_ij, with the value read from
@@ -42,9 +42,9 @@ __global__ void k_forces(int n, const int32_t* __restrict__ row_ptr, const int32
             float3 v;
             const float d = edge_distance(pi, pos4[j], box, v);
             if (d < rc && d > 0.f) {
-                // the pair's derivative sits on its owning edge (i, j) with j > i
+                // the pair's derivative sits on its owning edge
                 const int re = rev[e];
-                const float D = j > i ? s_edge[e] : (re >= 0 ? s_edge[re] : 0.f);
+                const float D = owns_pair(i, j) ? s_edge[e] : (re >= 0 ? s_edge[re] : 0.f);
                 float k = D / d;
                 fx = fmaf(k, v.x, fx);
                 fy = fmaf(k, v.y, fy);

@@ -75,11 +75,11 @@ struct Workspace {
     float* cdist;                 // [cap] their distances
     int32_t* ccount;              // [ncta]
     int32_t* part;                // [ncta+1]
-    int32_t *crow_h, *ccol_h, *cidx_h;  // [cap] the half list: edges (i, j), j > i, d < r_c
+    int32_t *crow_h, *ccol_h, *cidx_h;  // [cap] the half list: edges (i, j) that own their pair, d < r_c
     float* cdist_h;               // [cap] their distances
     int32_t* ccount_h;            // [ncta]    its per-CTA edge counts
     int32_t* part_h;              // [ncta+1]  and its own row partition
-    int32_t *crow_r, *ccol_r;     // [cap] the complement: edges (i, j), j < i, d < r_c (dE/dh launches)
+    int32_t *crow_r, *ccol_r;     // [cap] the complement: the other edges with d < r_c (dE/dh launches)
     float* cdist_r;               // [cap] their distances
     int32_t* ccount_r;            // [ncta]
     int32_t* part_r;              // [ncta+1]
@@ -92,7 +92,8 @@ struct Workspace {
     GridGeom* rgrid_geom;         // [R]   grid origin and inverse cell sizes (float64)
     long long* scan_tmp;          // [SCAN_TILE] tile sums
     // activations
-    float *x, *h, *q, *m, *g, *dh, *pr, *eps, *ke;
+    float *x, *h, *q, *m, *g, *pr, *eps, *ke;
+    float *dh, *dh2;              // [N*FP] dE/dh: the half list's terms and the complement's
     // reductions
     double* partial;              // [nchunk]
     int32_t *chunk_rep, *chunk_lo, *chunk_hi;  // [nchunk]

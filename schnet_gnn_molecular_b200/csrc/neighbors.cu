@@ -473,8 +473,8 @@ __global__ void k_partition(int n, int ncta, const int32_t* __restrict__ row_ptr
 }
 
 // Per row, the edges the tensor-core kernels will carry at the build's positions:
-// those inside the cutoff (cnt), and of them those with j > i (cnt_half, the half
-// list that visits each unordered pair once) and those with j < i (cnt_rev, its
+// those inside the cutoff (cnt), and of them those that own their pair (cnt_half,
+// the half list that visits each unordered pair once) and the others (cnt_rev, its
 // complement).  The distance is the masking pass's own expression, so the counts
 // equal what it keeps at these positions; the row partitions balance them.  One
 // warp per row.
@@ -497,7 +497,7 @@ __global__ void k_cut_counts(int n, const int32_t* __restrict__ row_ptr, const i
                 const float d = edge_distance(pi, pos4[j], box, v);
                 if (d < rc && d > 0.f) {
                     ++c;
-                    ch += j > i;
+                    ch += owns_pair(i, j);
                 }
             }
         }

@@ -108,6 +108,7 @@ struct TileMeta {
     int32_t col[TE];
     float fc[TE];
     float dfc[BWD ? TE : 4];
+    float d[TE];                 // distance (stage R's Gaussian units read it)
     ChunkInfo c[TE / 32];
 };
 
@@ -142,8 +143,9 @@ __device__ __forceinline__ void group_sync(int g)
     asm volatile("bar.sync %0, %1;" ::"r"(1 + g), "n"(GT) : "memory");
 }
 
-// OR of a predicate over math group g (a barrier of the group's 256 threads)
-__device__ __forceinline__ bool group_or(int g, bool v)
+// OR of a predicate over the NTH threads that meet at named barrier id
+template <int NTH>
+__device__ __forceinline__ bool bar_or(int id, bool v)
 {
     uint32_t r;
     asm volatile(
@@ -152,10 +154,18 @@ __device__ __forceinline__ bool group_or(int g, bool v)
         "bar.red.or.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)v), "r"(1 + g), "n"(GT)
+        : "r"((uint32_t)v), "r"(id), "n"(NTH)
         : "memory");
     return r != 0;
 }
+
+// OR of a predicate over math group g (a barrier of the group's 256 threads, ids 1, 2)
+__device__ __forceinline__ bool group_or(int g, bool v) { return bar_or<GT>(1 + g, v); }
+
+// OR of a predicate over the merging warps 0-3 of math group g (ids 3, 4): the
+// merge waits for no other warp of its group, in particular not for the one
+// issuing the next tile's GEMM1
+__device__ __forceinline__ bool merge_or(int g, bool v) { return bar_or<128>(3 + g, v); }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar)
 {
@@ -172,7 +182,7 @@ struct EdgePre {
 };
 
 template <int TE, bool BWD>
-__device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, int ne, int mt)
+__device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, int ne, int t)
 {
     EdgePre p;
     p.i = 0;
@@ -180,12 +190,11 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
     p.d = 0.f;
     p.gidx = 0;
     p.sold = 0.f;
-    const int t = mt & (TE - 1);
-    if (t < ne) {
+    if (t >= 0 && t < ne) {
         p.i = __ldg(a.crow + e0 + t);
         p.j = __ldg(a.ccol + e0 + t);
         p.d = __ldg(a.cdist + e0 + t);
-        if (BWD && mt < TE) {
+        if (BWD) {
             p.gidx = __ldg(a.cidx + e0 + t);
             if (a.accumulate_s) p.sold = a.s_edge[p.gidx];
         }
@@ -193,75 +202,84 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
     return p;
 }
 
-// Stage R: GT / TE threads per edge, each for KP / (GT / TE) Gaussians: distance
-// (minimum image), cutoff mask, Gaussian expansion written as hi/lo 16-bit
-// K-major B rows; in the backward tile row TE + e holds the d-derivative of
-// edge e's Gaussians, scaled by 1 / (2 ln 2) (the epilogue folds the factor
-// back in).  Gaussian columns K .. KP-1 meet zero weight rows and are stored
-// as zeros without evaluating them; masked or padding edges have
-// f_c = f_c' = 0, so their Gaussians need no mask (they stay finite).
+// Stage R, by the group's warps 1-7 (worker w = group thread - 32): warp 0 issues
+// GEMM2 meanwhile, and an issuing thread blocks while the tensor core's queue is
+// full, so warp 0 does no stage-R work.  Workers w < TE take edge w (its endpoints
+// and distance prefetched a tile ahead): cutoff envelope f_c (and f_c'), column
+// and distance into the tile's record, and a row summary of each 32-edge chunk by
+// warp votes.  After a barrier of the 224 workers, work unit u = w, w + 224, ...
+// writes the Gaussians 8 (u / TE) .. 8 (u / TE) + 7 of edge u % TE as hi/lo 16-bit
+// K-major B rows; in the backward tile row TE + e holds the d-derivative of edge
+// e's Gaussians, scaled by 1 / (2 ln 2) (the epilogue folds the factor back in).
+// Gaussian columns K .. KP-1 meet zero weight rows and are stored as zeros without
+// evaluating them; masked or padding edges have f_c = f_c' = 0, so their Gaussians
+// need no mask (they stay finite).
+constexpr int NWK = GT - 32;              // stage-R workers per group
+
+// named barrier of the stage-R workers of group g (ids 5 and 6)
+__device__ __forceinline__ void workers_sync(int g)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(5 + g), "n"(NWK) : "memory");
+}
+
 template <int FMT, int NX, bool BWD, int TE>
 __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMeta<TE, BWD>* tmeta, const EdgePre& ep,
-                                          int ne, int mt)
+                                          int ne, int w, int g)
 {
-    constexpr int TPE = GT / TE;         // threads per edge
-    constexpr int KPT = KP / TPE;        // Gaussians per thread
-    const int e = mt & (TE - 1);
-    const int kq = mt / TE;              // warp-uniform
-    float d = 0.f;
-    bool valid = false;
-    if (e < ne) {
-        d = ep.d;
-        valid = d < a.rc && d > 0.f;   // holds for every compacted edge
-    }
-    if (kq == 0) {
-        float fc = 0.f, dfc = 0.f;
-        if (valid) {
-            float sn, cs;
-            sincospif(d * a.inv_rc, &sn, &cs);
-            fc = 0.5f * (cs + 1.0f);
-            dfc = -0.5f * 3.14159265358979f * a.inv_rc * sn;
+    if (w < TE) {
+        const int e = w;
+        float d = 0.f, fc = 0.f, dfc = 0.f;
+        if (e < ne) {
+            d = ep.d;
+            if (d < a.rc && d > 0.f) {   // holds for every compacted edge
+                float sn, cs;
+                sincospif(d * a.inv_rc, &sn, &cs);
+                fc = 0.5f * (cs + 1.0f);
+                dfc = -0.5f * 3.14159265358979f * a.inv_rc * sn;
+            }
         }
         const int row = e < ne ? ep.i : 0x7fffffff;
         tmeta->col[e] = e < ne ? ep.j : 0;
         tmeta->fc[e] = fc;
+        tmeta->d[e] = d;
         if (BWD) tmeta->dfc[e] = dfc;
-        // warp w of this quarter holds edges 32w .. 32w+31: summarise the chunk's rows
-        const int lane = mt & 31, w = e >> 5;
-        const int nv = min(max(ne - 32 * w, 0), 32);
+        // the worker's warp holds edges 32c .. 32c+31: summarise the chunk's rows
+        const int lane = w & 31, c = e >> 5;
+        const int nv = min(max(ne - 32 * c, 0), 32);
         const int rfirst = __shfl_sync(0xffffffffu, row, 0);
         const int rlast = __shfl_sync(0xffffffffu, row, nv > 0 ? nv - 1 : 0);
         const unsigned fm = __ballot_sync(0xffffffffu, e < ne && row == rfirst);
         const int oth = __any_sync(0xffffffffu, e < ne && row != rfirst && row != rlast);
-        if (lane == 0) tmeta->c[w] = ChunkInfo{rfirst, rlast, fm, oth};
+        if (lane == 0) tmeta->c[c] = ChunkInfo{rfirst, rlast, fm, oth};
     }
+    workers_sync(g);
     uint8_t* b_hi = rbf;
     uint8_t* b_lo = rbf + RBF_TERM;
-    const float dm = d - fmaf((float)(kq * KPT), a.dmu, a.mu0);   // d - mu of this thread's first Gaussian
-#pragma unroll
-    for (int g = 0; g < KPT / 8; ++g) {
-        const int kg = kq * (KPT / 8) + g;
+#pragma unroll 1
+    for (int u = w; u < TE * (KP / 8); u += NWK) {
+        const int e = u & (TE - 1), kg = u / TE;
         const uint32_t off = kmajor_off(e, kg * 8, MN);
         const uint32_t offd = kmajor_off(TE + e, kg * 8, MN);
-        if (kg * 8 >= a.K) {                 // padding columns (warp-uniform)
+        if (kg * 8 >= a.K) {                 // padding columns
             store8_zero(b_hi, b_lo, off);
             if (BWD) store8_zero(b_hi, b_lo, offd);
             continue;
         }
+        const float dm = tmeta->d[e] - fmaf((float)(kg * 8), a.dmu, a.mu0);   // d - mu of the unit's first Gaussian
         float gv[8], dv[8];
         if (!BWD) {
 #pragma unroll
             for (int q = 0; q < 8; q += 2) {
-                const float2 x = fma2(make_float2(-(float)(g * 8 + q), -(float)(g * 8 + q + 1)), dup2(a.dmu), dup2(dm));
+                const float2 x = fma2(make_float2(-(float)q, -(float)(q + 1)), dup2(a.dmu), dup2(dm));
                 const float2 t = mul2(x, dup2(a.ngc));
-                const float2 e = mul2(t, x);
-                gv[q] = ex2_mufu(e.x);
-                gv[q + 1] = ex2_mufu(e.y);
+                const float2 ee = mul2(t, x);
+                gv[q] = ex2_mufu(ee.x);
+                gv[q + 1] = ex2_mufu(ee.y);
             }
         } else {
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                const float x = fmaf(-(float)(g * 8 + q), a.dmu, dm);
+                const float x = fmaf(-(float)q, a.dmu, dm);
                 const float t = x * a.ngc;
                 const float gg = ex2_mufu(t * x);
                 gv[q] = gg;
@@ -431,22 +449,32 @@ __device__ __forceinline__ void merge_chunks(const ChunkInfo* ci, const float* p
     }
 }
 
-// Merge step of tile t by its group: wait for tile t-1's merge, fold this
-// tile's partials into the carry, hand the carry on.  Returns false on timeout.
+// Merge step of tile t by its group's warps 0-3 (thread mt = feature): wait for
+// tile t-1's merge (warp 0 polls the token, a barrier of the 128 merging threads
+// shares the outcome, and warps 1-3 repeat the test for their own acquire), fold
+// this tile's partials into the carry, hand the carry on.  Returns false (uniformly
+// over the 128 threads) on timeout.
 template <int NCH>
 __device__ __forceinline__ bool merge_tile(Carry* cy, uint64_t* tok, const ChunkInfo* ci, const float* pf,
                                            const float* pl, int ne, int t, float* __restrict__ out, DevMeta* meta,
                                            int g, int mt)
 {
-    if (!wait_group(tok, (uint32_t)((t - 1) & 1), t > 0, mt < 128, meta, g, mt)) return false;
-    if (mt < 128) {
-        int cur = cy->cur[(t + 1) & 1];      // written by tile t-1 (or the initial row)
-        float acc = cy->acc[mt];
-        merge_chunks<NCH>(ci, pf, pl, ne, mt, out, cur, acc);
-        cy->acc[mt] = acc;
-        if (mt == 0) cy->cur[t & 1] = cur;
-        mbar_arrive(tok);
+    if (t > 0) {
+        const uint32_t parity = (uint32_t)((t - 1) & 1);
+        bool ok = true;
+        if ((mt >> 5) == 0) ok = mbar_wait_bounded(tok, parity, WAIT_POLLS);
+        if (merge_or(g, !ok)) {
+            if (mt == 0) set_flag(meta, SCHNET_FLAG_TIMEOUT);
+            return false;
+        }
+        if ((mt >> 5) != 0) (void)mbar_try_wait(tok, parity);
     }
+    int cur = cy->cur[(t + 1) & 1];      // written by tile t-1 (or the initial row)
+    float acc = cy->acc[mt];
+    merge_chunks<NCH>(ci, pf, pl, ne, mt, out, cur, acc);
+    cy->acc[mt] = acc;
+    if (mt == 0) cy->cur[t & 1] = cur;
+    mbar_arrive(tok);
     return true;
 }
 
@@ -699,12 +727,13 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     const int ntiles = (int)((e1 - e0 + TE - 1) / TE);
     auto tile_ne = [&](int t) { return (int)min((long long)TE, e1 - e0 - (long long)t * TE); };
 
+    const int w = mt - 32;                          // stage-R worker (warps 1-7 of the group)
     EdgePre ep;
     if (g < ntiles) {
         if (g == 1) ok = wait_group(&bars[3], 0u, true, false, a.meta, g, mt);   // start half a tile behind
-        ep = prefetch_edge<TE, false>(a, e0 + (long long)g * TE, tile_ne(g), mt);
-        stage_rbf<FMT, NX, false, TE>(a, rbf, tmb, ep, tile_ne(g), mt);
-        if (g + 2 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(g + 2) * TE, tile_ne(g + 2), mt);
+        ep = prefetch_edge<TE, false>(a, e0 + (long long)g * TE, tile_ne(g), w);
+        if (w >= 0) stage_rbf<FMT, NX, false, TE>(a, rbf, tmb, ep, tile_ne(g), w, g);
+        if (g + 2 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(g + 2) * TE, tile_ne(g + 2), w);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
@@ -734,10 +763,10 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
             mma_commit(&bars[g]);
         }
         pending = 1;
-        // under GEMM2: stage R of tile t+2 and the first gather of this tile
+        // under GEMM2: stage R of tile t+2 (warps 1-7) and the first gather of this tile
         if (next) {
-            stage_rbf<FMT, NX, false, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), mt);
-            if (t + 4 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(t + 4) * TE, tile_ne(t + 4), mt);
+            if (w >= 0) stage_rbf<FMT, NX, false, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), w, g);
+            if (t + 4 < ntiles) ep = prefetch_edge<TE, false>(a, e0 + (long long)(t + 4) * TE, tile_ne(t + 4), w);
             fence_proxy_async_smem();
         }
         float hv[32];
@@ -759,8 +788,11 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         // thread blocks while the tensor core's queue is full)
         if (next && mt == 128) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
-        if (!(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
-        group_sync(g);          // merge done with the partials before E1 of the next tile overwrites them
+        bool merged = true;
+        if (mt < 128) merged = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt);
+        // the merge done with the partials before E1 of the next tile overwrites them (and its
+        // outcome known to the whole group)
+        if (!(ok = !group_or(g, !merged))) break;
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
     if (mt == 0) {
@@ -885,16 +917,17 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     const int ntiles = (int)((e1 - e0 + TE - 1) / TE);
     auto tile_ne = [&](int t) { return (int)min((long long)TE, e1 - e0 - (long long)t * TE); };
 
+    const int w = mt - 32;         // stage-R worker (warps 1-7 of the group)
     EdgePre ep;
-    int my_g = 0, nx_g = 0;        // group threads < TE: s_e slot of edge mt (this tile / tile t+2)
+    int my_g = 0, nx_g = 0;        // workers w < TE: s_e slot of edge w (this tile / tile t+2)
     float my_so = 0.f, nx_so = 0.f;
     if (g < ntiles) {
         if (g == 1) ok = wait_group(&bars[3], 0u, true, false, a.meta, g, mt);   // start half a tile behind
-        ep = prefetch_edge<TE, true>(a, e0 + (long long)g * TE, tile_ne(g), mt);
-        stage_rbf<FMT, NX, true, TE>(a, rbf, tmb, ep, tile_ne(g), mt);
+        ep = prefetch_edge<TE, true>(a, e0 + (long long)g * TE, tile_ne(g), w);
+        if (w >= 0) stage_rbf<FMT, NX, true, TE>(a, rbf, tmb, ep, tile_ne(g), w, g);
         nx_g = ep.gidx;
         nx_so = ep.sold;
-        if (g + 2 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(g + 2) * TE, tile_ne(g + 2), mt);
+        if (g + 2 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(g + 2) * TE, tile_ne(g + 2), w);
         fence_proxy_async_smem();
         tc_fence_before();
         group_sync(g);
@@ -925,12 +958,12 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
             mma_commit(&bars[g]);
         }
         pending = 1;
-        // under GEMM2: stage R of tile t+2 and the first gathers of this tile
+        // under GEMM2: stage R of tile t+2 (warps 1-7) and the first gathers of this tile
         if (next) {
-            stage_rbf<FMT, NX, true, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), mt);
+            if (w >= 0) stage_rbf<FMT, NX, true, TE>(a, rbf, tmb + (buf ^ 1), ep, tile_ne(t + 2), w, g);
             nx_g = ep.gidx;
             nx_so = ep.sold;
-            if (t + 4 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(t + 4) * TE, tile_ne(t + 4), mt);
+            if (t + 4 < ntiles) ep = prefetch_edge<TE, true>(a, e0 + (long long)(t + 4) * TE, tile_ne(t + 4), w);
             fence_proxy_async_smem();
         }
         const int eb = col0;
@@ -1069,16 +1102,22 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         }
         tc_fence_before();
         group_sync(g);          // Q, Q' read out; per-edge partials and the next tile's Gaussians in place
-        // GEMM1(t+2) is issued by warp 4, which does not write s_e below (an issuing thread
-        // blocks while the tensor core's queue is full)
+        // GEMM1(t+2) is issued by warp 4, which does not write s_e below (warps 1 and 2 do; an
+        // issuing thread blocks while the tensor core's queue is full)
         if (next && mt == 128) issue_gemm1<NW, NX>(tmem, dacc, srbf, id, &bars[g]);
         if (next) pending = 1;
-        if (mt < ne) {
-            const float sv = ps_s[mt] + ps_s[TE + mt] + ps_s[2 * TE + mt] + ps_s[3 * TE + mt];
+        if (w >= 0 && w < ne) {
+            const float sv = ps_s[w] + ps_s[TE + w] + ps_s[2 * TE + w] + ps_s[3 * TE + w];
             a.s_edge[my_g] = a.accumulate_s ? my_so + sv : sv;
         }
-        if (DH && !(ok = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt))) break;
-        group_sync(g);          // s_e and the merge done with the partials before E1 of the next tile overwrites them
+        if (DH) {
+            bool merged = true;
+            if (mt < 128) merged = merge_tile<NCH>(cy, &bars[2], tm->c, pf_s, pl_s, ne, t, a.out, a.meta, g, mt);
+            // s_e and the merge done with the partials before E1 of the next tile overwrites them
+            if (!(ok = !group_or(g, !merged))) break;
+        } else {
+            group_sync(g);      // s_e done with the partials before E1 of the next tile overwrites them
+        }
     }
     if (g == 0 && !go_sent && mt == 0) mbar_arrive(&bars[3]);
     if (mt == 0) {

@@ -114,10 +114,11 @@ def tensor_peak(peaks, clk):
 # MUFU (special-function unit) operations counted from the kernel source: forward kernel, per
 # directed edge -- one ex2 per evaluated Gaussian (K), and per feature one ex2 and one lg2 for the
 # base-2 softplus, except that one feature pair in four takes its ex2 on the FMA pipe; pair
-# kernel, per unordered pair -- K Gaussian ex2, per feature ex2 and lg2 for the softplus and one
-# more ex2 for the logistic.  148 SMs x 16 MUFU results per clock.
+# kernel, per unordered pair -- K Gaussian ex2, per feature ex2 and lg2 for the softplus (one
+# feature pair in four with its ex2 on the FMA pipe) and one more ex2 for the logistic.  148 SMs
+# x 16 MUFU results per clock.
 def mufu_per_edge(K, F):
-    return {"fwd": K + 2 * F - F // 4, "bwd": K + 3 * F}
+    return {"fwd": K + 2 * F - F // 4, "bwd": K + 3 * F - F // 4}
 
 
 def hbm_kernel_bytes(w, E_list, E_cut):

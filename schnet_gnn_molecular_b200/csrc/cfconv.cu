@@ -119,8 +119,9 @@ template <int TE, bool BWD> constexpr uint32_t sm_carry() { return sm_meta<TE, B
 template <int TE, bool BWD> constexpr uint32_t sm_bar() { return sm_carry<TE, BWD>() + CARRY_BYTES; }
 template <int TE, bool BWD> constexpr uint32_t smem_bytes() { return sm_bar<TE, BWD>() + BAR_BYTES; }
 // barrier block: [0] group 0 MMA commits, [1] group 1 MMA commits, [2] merge token,
-// [3] group 1 start (u64 each); then the TMEM base (u32), each group's MMA phase to
-// drain on an error exit (u32 x2) and each group's "commit outstanding" flag (u32 x2)
+// [3] group 1 start, [4] epilogue-1 token (u64 each); then the TMEM base (u32), each
+// group's MMA phase to drain on an error exit (u32 x2) and each group's "commit
+// outstanding" flag (u32 x2)
 static_assert(smem_bytes<TE_F, false>() <= 232448, "forward shared memory exceeds the per-block limit");
 static_assert(smem_bytes<TE_B, true>() <= 232448, "backward shared memory exceeds the per-block limit");
 static_assert(sizeof(TileMeta<TE_F, false>) % 16 == 0 && sizeof(TileMeta<TE_B, true>) % 16 == 0, "meta alignment");
@@ -328,6 +329,28 @@ __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, DevMeta
 {
     bool ok = true;
     if ((mt >> 5) == 0) ok = mbar_wait_bounded(bar, phase, WAIT_POLLS);
+    if (group_or(g, !ok)) {
+        if (mt == 0) set_flag(meta, SCHNET_FLAG_TIMEOUT);
+        return false;
+    }
+    phase ^= 1u;
+    tc_fence_after();
+    return true;
+}
+
+// Wait for group g's tensor-core commit and, for every tile but the first, for the
+// epilogue-1 token of the previous tile (phase `tparity`: the other group has
+// finished its epilogue 1, which keeps the two groups' MUFU-bound epilogues 1 from
+// overlapping and the groups from falling into step); false (uniformly over the
+// group) on timeout.  The token orders work only, it guards no data.
+__device__ __forceinline__ bool wait_mma_e1(uint64_t* bar, uint32_t& phase, uint64_t* tok, uint32_t tparity,
+                                            bool need_tok, DevMeta* meta, int g, int mt)
+{
+    bool ok = true;
+    if ((mt >> 5) == 0) {
+        ok = mbar_wait_bounded(bar, phase, WAIT_POLLS);
+        if (ok && need_tok) ok = mbar_wait_bounded(tok, tparity, WAIT_POLLS);
+    }
     if (group_or(g, !ok)) {
         if (mt == 0) set_flag(meta, SCHNET_FLAG_TIMEOUT);
         return false;
@@ -549,6 +572,7 @@ __device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslo
         mbar_init(&bars[1], 1);      // group 1 MMA commits
         mbar_init(&bars[2], 128);    // merge token: the 128 merging threads of a tile
         mbar_init(&bars[3], 1);      // group 1 start
+        mbar_init(&bars[4], 1);      // epilogue-1 token: one arrival per tile, in tile order
         fence_mbar_init();
     }
     if (threadIdx.x < FP) cy->acc[threadIdx.x] = 0.f;
@@ -689,7 +713,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     extern __shared__ __align__(1024) uint8_t smem[];
     Carry* cy = reinterpret_cast<Carry*>(smem + sm_carry<TE, false>());
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sm_bar<TE, false>());
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 5);
     uint32_t* phases_s = tslot + 1;
     uint32_t* pend_s = tslot + 3;
 
@@ -746,7 +770,9 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
         const bool next = t + 2 < ntiles;
         Meta* tm = tmb + buf;
         const int32_t* rows_g = a.crow + e0 + (long long)t * TE;
-        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM1(t) done
+        // GEMM1(t) done (the epilogue-1 token is not used here: with it the forward settles
+        // a quarter tile apart, as without, and runs 0.5 % slower)
+        if (!(ok = wait_mma_e1(&bars[g], phase, &bars[4], 0u, false, a.meta, g, mt))) break;
         pending = 0;
         if (g == 0 && !go_sent) {
             if (mt == 0) mbar_arrive(&bars[3]);
@@ -829,7 +855,10 @@ __device__ __forceinline__ void bwd_e1(uint32_t tP, uint32_t tPd, float s1L, flo
 #pragma unroll
         for (int q = 0; q < 16; q += 2) {
             const float2 p = fma2(dup2(s1L), make_float2(r[q], r[q + 1]), dup2(b1L));
-            const float2 t = make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y)));
+            // one pair in four takes 2^-|p| from the FMA pipe (the MUFU carries three operations
+            // per element here)
+            const float2 t = ((q >> 1) & 3) == 3 ? ex2_fma2(make_float2(-fabsf(p.x), -fabsf(p.y)))
+                                                 : make_float2(ex2_mufu(-fabsf(p.x)), ex2_mufu(-fabsf(p.y)));
             constexpr float c = NX == 2 ? 0.5f : 1.0f;
             const float2 y = fma2(dup2(c), t, dup2(c));                     // c (1 + t)
             const float2 l = make_float2(lg2_mufu(y.x), lg2_mufu(y.y));
@@ -872,7 +901,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     extern __shared__ __align__(1024) uint8_t smem[];
     Carry* cy = reinterpret_cast<Carry*>(smem + sm_carry<TE, true>());
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sm_bar<TE, true>());
-    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 4);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 5);
     uint32_t* phases_s = tslot + 1;
     uint32_t* pend_s = tslot + 3;
 
@@ -942,7 +971,8 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         const int32_t* rows_g = a.crow + e0 + (long long)t * TE;
         my_g = nx_g;
         my_so = nx_so;
-        if (!(ok = wait_mma(&bars[g], phase, a.meta, g, mt))) break;     // GEMM1(t) done
+        // GEMM1(t) done, and epilogue 1 of tile t-1 (the other group's)
+        if (!(ok = wait_mma_e1(&bars[g], phase, &bars[4], (uint32_t)((t - 1) & 1), t > 0, a.meta, g, mt))) break;
         pending = 0;
         if (g == 0 && !go_sent) {
             if (mt == 0) mbar_arrive(&bars[3]);
@@ -953,6 +983,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
         tc_fence_before();
         group_sync(g);
         if (mt == 0) {
+            mbar_arrive(&bars[4]);  // epilogue 1 of tile t done: the other group's tile t+1 may start its own
             tc_fence_after();
             issue_gemm<NW, NX, FP / 16>(dacc, tmem + TM_W2H, tmem + TM_W2L, sact, ACT_TERM, id_mn);
             mma_commit(&bars[g]);

@@ -212,9 +212,10 @@ __device__ __forceinline__ EdgePre prefetch_edge(const MPArgs& a, long long e0, 
 // writes the Gaussians 8 (u / TE) .. 8 (u / TE) + 7 of edge u % TE as hi/lo 16-bit
 // K-major B rows; in the backward tile row TE + e holds the d-derivative of edge
 // e's Gaussians, scaled by 1 / (2 ln 2) (the epilogue folds the factor back in).
-// Gaussian columns K .. KP-1 meet zero weight rows and are stored as zeros without
-// evaluating them; masked or padding edges have f_c = f_c' = 0, so their Gaussians
-// need no mask (they stay finite).
+// Gaussian columns K .. KP-1 meet zero weight rows: the K-groups of 8 wholly past K
+// are zeroed once at kernel start and never written here, and the last partial
+// group's extra columns take finite Gaussian values.  Masked or padding edges have
+// f_c = f_c' = 0, so their Gaussians need no mask (they stay finite).
 constexpr int NWK = GT - 32;              // stage-R workers per group
 
 // named barrier of the stage-R workers of group g (ids 5 and 6)
@@ -256,16 +257,12 @@ __device__ __forceinline__ void stage_rbf(const MPArgs& a, uint8_t* rbf, TileMet
     workers_sync(g);
     uint8_t* b_hi = rbf;
     uint8_t* b_lo = rbf + RBF_TERM;
+    const int nu = TE * ((a.K + 7) >> 3);  // units that hold a Gaussian below K
 #pragma unroll 1
-    for (int u = w; u < TE * (KP / 8); u += NWK) {
+    for (int u = w; u < nu; u += NWK) {
         const int e = u & (TE - 1), kg = u / TE;
         const uint32_t off = kmajor_off(e, kg * 8, MN);
         const uint32_t offd = kmajor_off(TE + e, kg * 8, MN);
-        if (kg * 8 >= a.K) {                 // padding columns
-            store8_zero(b_hi, b_lo, off);
-            if (BWD) store8_zero(b_hi, b_lo, offd);
-            continue;
-        }
         const float dm = tmeta->d[e] - fmaf((float)(kg * 8), a.dmu, a.mu0);   // d - mu of the unit's first Gaussian
         float gv[8], dv[8];
         if (!BWD) {
@@ -560,9 +557,22 @@ __device__ __forceinline__ void chunk_partials(const ChunkInfo& ci, const int32_
 // pdl_wait): TMEM allocation, mbarriers, the filter weights into TMEM (one output
 // channel per lane; the six 32-column row loads of each lane quadrant spread over
 // the quadrant's four warps), the zero carry.  Returns the TMEM base address.
-__device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint32_t* tslot, uint64_t* bars, Carry* cy)
+__device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint8_t* smem, uint32_t* tslot, uint64_t* bars,
+                                                 Carry* cy)
 {
     const int warp = threadIdx.x >> 5;
+    {
+        // the K-groups of both groups' GEMM1 B operands (hi and lo terms) wholly past K: zero
+        // for every tile, so stage R does not write them
+        const int nkg = (a.K + 7) >> 3;
+        const uint32_t pad = (uint32_t)(KP / 8 - nkg) * (MN * 16);   // bytes per term
+        for (uint32_t o = threadIdx.x * 16; o < 4 * pad; o += NT * 16) {
+            const uint32_t term = o / pad, r = o % pad;                // term = 2 group + (hi, lo)
+            *reinterpret_cast<uint4*>(smem + SM_RBF + term * RBF_TERM + (uint32_t)nkg * (MN * 16) + r) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+    }
     if (warp == 0) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
@@ -727,7 +737,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
     int r0, r1;
     kernel_rows(a, r0, r1);
     if (r0 >= r1) return;
-    const uint32_t tmem = kernel_setup(a, tslot, bars, cy);
+    const uint32_t tmem = kernel_setup(a, smem, tslot, bars, cy);
     if (threadIdx.x == 0) cy->cur[1] = r0;         // tile 0 reads the carry of "tile -1"
     pdl_wait();                                     // the previous kernel's results from here on
     __syncthreads();
@@ -915,7 +925,7 @@ __global__ void __launch_bounds__(NT, 1) k_cfconv_bwd(MPArgs a)
     int r0, r1;
     kernel_rows(a, r0, r1);
     if (r0 >= r1) return;
-    const uint32_t tmem = kernel_setup(a, tslot, bars, cy);
+    const uint32_t tmem = kernel_setup(a, smem, tslot, bars, cy);
     if (threadIdx.x == 0) cy->cur[1] = r0;         // tile 0 reads the carry of "tile -1"
     pdl_wait();                                     // the previous kernel's results from here on
     __syncthreads();

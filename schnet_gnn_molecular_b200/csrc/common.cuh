@@ -411,11 +411,6 @@ __device__ __forceinline__ void store8_act(uint8_t* hi_base, uint8_t* lo_base, u
     else store8_hi<FMT>(hi_base, off, v);
 }
 
-__device__ __forceinline__ void store8_zero(uint8_t* hi_base, uint8_t* lo_base, uint32_t off)
-{
-    *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(0u, 0u, 0u, 0u);
-    *reinterpret_cast<uint4*>(lo_base + off) = make_uint4(0u, 0u, 0u, 0u);
-}
 
 // 32 lanes x 16 columns of TMEM -> 16 registers per thread
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16])

@@ -227,6 +227,23 @@ def test_protein64_sampled_replicas():
 
 
 # ---------------------------------------------------------------------------
+# Gaussian counts: K = 13 (the last group of 8 partly past K, the groups after it
+# zero), K = 64 (no padding at all) and K = 8 (one group)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("K", [8, 13, 64])
+def test_energy_forces_gaussian_counts(K):
+    w = SMALL_PROTEIN.with_(name=f"cg_protein_6x269_K{K}", K=K)
+    pos, types, weights, model = _setup(w, bias_scale=0.1)
+    E, F = _gpu_eval(model, pos, types)
+    ro = w.replica_offsets()
+    Eo, eps_o, Fo = oracle.energy_forces(oracle_model(w, weights), pos.astype(np.float64), types, ro)
+    check_energies(E, Eo, eps_o, ro, label=f"6 x 269, K = {K}")
+    err = rel_frobenius(F, Fo)
+    print(f"[errors K={K}] forces {err:.3e}")
+    assert err <= FORCE_RTOL
+
+
+# ---------------------------------------------------------------------------
 # depth: one interaction (its single pair-derivative launch over the half list
 # starts the per-edge sums afresh) and four (three launches add to them)
 # ---------------------------------------------------------------------------

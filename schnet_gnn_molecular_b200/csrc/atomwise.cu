@@ -148,9 +148,21 @@ __global__ void __launch_bounds__(AWT, 1) k_atomwise(AWArgs a)
     tc_fence_after();
     const uint32_t tmem = *tslot;
     const uint32_t lane_base = tmem + ((uint32_t)(qd * 32) << 16);
-    // weights: warp c of quadrant qd loads (term c >> 1, half c & 1) of every slot
-    for (int s = 0; s < a.ngemm; ++s)
-        weights_to_tmem(lane_base, AW_SLOT + 128 * s + (c >> 1) * 64, a.img[s] + (c >> 1) * AW_BTERM, f, c & 1);
+    // weights: warp c of quadrant qd loads (term c >> 1, half c & 1) of every slot, all slots'
+    // rows first (one trip to L2), then the TMEM stores
+    {
+        uint32_t x[3][32];
+#pragma unroll
+        for (int s = 0; s < 3; ++s) {
+            if (s >= a.ngemm) break;
+            weight_row(a.img[s] + (c >> 1) * AW_BTERM, f, c & 1, x[s]);
+        }
+#pragma unroll
+        for (int s = 0; s < 3; ++s) {
+            if (s >= a.ngemm) break;
+            tmem_st32(lane_base + AW_SLOT + 128 * s + (c >> 1) * 64 + (c & 1) * 32, x[s]);
+        }
+    }
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     const uint32_t sB = smem_u32(B);
     const uint32_t tD = lane_base + AW_ACC + c * 32;

@@ -3,9 +3,10 @@
 // One kernel per interaction and direction does, for tiles of a CTA's contiguous
 // CSR rows (forward: 128 edges; backward: 64 edges, whose derivative rows fill
 // the other half of the GEMM's N = 128):
-//   flash radial basis  (FlashSchNet paper-curation summary, How): distance,
-//     Gaussian expansion and cosine envelope computed once per edge into
-//     shared memory, never to HBM;
+//   flash radial basis  (FlashSchNet paper-curation summary, How): Gaussian
+//     expansion and cosine envelope of the edge's distance (stored by the
+//     cutoff-masking pass) computed once per edge into shared memory, never to
+//     HBM;
 //   filter network      (How, quantization item; contraction on tensor cores):
 //     W(d) = f_c(d) (ssp(e W1 + b1) W2 + b2) as two chained tcgen05 GEMMs with
 //     TMEM accumulators; channel-wise scaled 16-bit operands, hi/lo split of
@@ -36,8 +37,14 @@
 // group waits for its GEMMs or its gathers, the other issues.  The CSR segment
 // sums cross tile boundaries through a carry (current row, partial sum per
 // feature) handed from tile to tile in order by an mbarrier token.  Group 1
-// starts once group 0's first GEMM1 has completed, so that the groups settle
-// half a tile apart rather than in step.
+// starts once group 0's first GEMM1 has completed.
+//
+// Warp roles inside a group: warp 0 issues GEMM2 (an issuing thread blocks while
+// the tensor core's queue is full) and so takes no part in stage R (the
+// Gaussians of tile t+2, run by warps 1-7 under GEMM2); warp 4 issues the next
+// GEMM1 while warps 0-3 merge the segment sums.  In the backward kernel an
+// mbarrier token also orders the two groups' epilogues 1 in tile order, which
+// keeps their MUFU-bound phases from overlapping and the groups out of step.
 #include "internal.h"
 
 namespace schnet {
@@ -594,11 +601,19 @@ __device__ __forceinline__ uint32_t kernel_setup(const MPArgs& a, uint8_t* smem,
         const int qd = warp & 3;                      // the lane quadrant this warp may access
         const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
         const int f = qd * 32 + (threadIdx.x & 31);
-        for (int job = warp >> 2; job < 6; job += NT / 128) {
-            const uint32_t col = job == 0 ? TM_W1H : job == 1 ? TM_W1L : job < 4 ? TM_W2H : TM_W2L;
-            const uint8_t* term = a.img + (job == 0 ? 0 : job == 1 ? W1_IMG : job < 4 ? 2 * W1_IMG : 2 * W1_IMG + W2_IMG);
-            weights_to_tmem(tl, col, term, f, job < 2 ? 0 : job & 1);
-        }
+        // job j: 0 W1 hi, 1 W1 lo, 2-3 W2 hi (K halves), 4-5 W2 lo; warp takes jobs warp/4 and
+        // warp/4 + 4, both rows loaded before either store (one trip to L2)
+        auto col_of = [](int j) { return j == 0 ? TM_W1H : j == 1 ? TM_W1L : j < 4 ? TM_W2H : TM_W2L; };
+        auto term_of = [&](int j) {
+            return a.img + (j == 0 ? 0 : j == 1 ? W1_IMG : j < 4 ? 2 * W1_IMG : 2 * W1_IMG + W2_IMG);
+        };
+        auto half_of = [](int j) { return j < 2 ? 0 : j & 1; };
+        const int j0 = warp >> 2, j1 = j0 + NT / 128;
+        uint32_t v0[32], v1[32];
+        weight_row(term_of(j0), f, half_of(j0), v0);
+        if (j1 < 6) weight_row(term_of(j1), f, half_of(j1), v1);
+        tmem_st32(tl + col_of(j0) + half_of(j0) * 32, v0);
+        if (j1 < 6) tmem_st32(tl + col_of(j1) + half_of(j1) * 32, v1);
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
@@ -710,10 +725,10 @@ __device__ __forceinline__ void issue_gemm1(uint32_t tmem, uint32_t dacc, uint32
 // ---------------------------------------------------------------------------
 // forward: m_i = sum_j h_j (.) W(d_ij)
 // ---------------------------------------------------------------------------
-// Per group and tile t: [GEMM1(t) in flight] E1 -> issue GEMM2 -> stage R of
-// t+2 (into the group's own GEMM1 operand and second metadata buffer) and the
-// first gather under GEMM2 -> E2 -> issue GEMM1(t+2) (by warp 4) -> merge under GEMM1(t+2)
-// (warps 0-3).
+// Per group and tile t: [GEMM1(t) in flight] E1 -> issue GEMM2 (warp 0) -> stage R
+// of t+2 (warps 1-7, into the group's own GEMM1 operand and second metadata
+// buffer) and the first gather under GEMM2 -> E2 -> issue GEMM1(t+2) (warp 4) ->
+// merge under GEMM1(t+2) (warps 0-3).
 template <int FMT, int NW, int NX>
 __global__ void __launch_bounds__(NT, 1) k_cfconv_fwd(MPArgs a)
 {

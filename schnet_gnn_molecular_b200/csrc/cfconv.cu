@@ -317,7 +317,8 @@ __device__ __forceinline__ void issue_gemm(uint32_t d_tmem, uint32_t a_hi_t, uin
     for (int ks = 0; ks < KSTEPS; ++ks) {
         const uint64_t step = (uint64_t)((ks * 2 * MN * 16) >> 4);   // 2 core matrices of 8 along K
         if (NW == 2) mma_f16_ts(d_tmem, a_lo_t + ks * 8, bh0 + step, idesc, ks > 0 ? 1u : 0u);
-        if (NX == 2) mma_f16_ts(d_tmem, a_hi_t + ks * 8, bl0 + step, idesc, (NW == 2 || ks > 0) ? 1u : 0u);
+        // the activation residual term is stored negated: its MMA negates B
+        if (NX == 2) mma_f16_ts(d_tmem, a_hi_t + ks * 8, bl0 + step, idesc | IDESC_NEG_B, (NW == 2 || ks > 0) ? 1u : 0u);
     }
 #pragma unroll
     for (int ks = 0; ks < KSTEPS; ++ks) {

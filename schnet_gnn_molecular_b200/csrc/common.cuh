@@ -400,12 +400,55 @@ __device__ __forceinline__ void store8_hi(uint8_t* hi_base, uint32_t off, const 
     *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(h[0], h[1], h[2], h[3]);
 }
 
-// activation operand: hi/lo pair (NX = 2) or the 16-bit rounding alone (NX = 1)
+// two fp32 values -> packed 16-bit hi pair and the NEGATED residual pair: hi - x
+// (exact in fp32, since it is the rounding error of hi) by the mixed-precision
+// subtract of the 16-bit hi and the fp32 x, then rounded once to 16 bits -- the
+// same bits as -RN16(x - hi), without converting hi back to fp32.  The MMAs that
+// read this term negate their B operand (instruction-descriptor bit 14).
+template <int FMT>
+__device__ __forceinline__ void split2_neg(float x0, float x1, uint32_t& hi, uint32_t& nlo);
+template <>
+__device__ __forceinline__ void split2_neg<0>(float x0, float x1, uint32_t& hi, uint32_t& nlo)
+{
+    asm("{\n\t.reg .b16 l, u;\n\t.reg .f32 d0, d1;\n\t"
+        "cvt.rn.f16x2.f32 %0, %3, %2;\n\t"
+        "mov.b32 {l, u}, %0;\n\t"
+        "sub.rn.f32.f16 d0, l, %2;\n\t"
+        "sub.rn.f32.f16 d1, u, %3;\n\t"
+        "cvt.rn.f16x2.f32 %1, d1, d0;\n\t}"
+        : "=r"(hi), "=r"(nlo)
+        : "f"(x0), "f"(x1));
+}
+template <>
+__device__ __forceinline__ void split2_neg<1>(float x0, float x1, uint32_t& hi, uint32_t& nlo)
+{
+    asm("{\n\t.reg .b16 l, u;\n\t.reg .f32 d0, d1;\n\t"
+        "cvt.rn.bf16x2.f32 %0, %3, %2;\n\t"
+        "mov.b32 {l, u}, %0;\n\t"
+        "sub.rn.f32.bf16 d0, l, %2;\n\t"
+        "sub.rn.f32.bf16 d1, u, %3;\n\t"
+        "cvt.rn.bf16x2.f32 %1, d1, d0;\n\t}"
+        : "=r"(hi), "=r"(nlo)
+        : "f"(x0), "f"(x1));
+}
+
+// instruction-descriptor bit of a negated B operand (the negated-residual terms)
+constexpr uint32_t IDESC_NEG_B = 1u << 14;
+
+// activation operand: hi and negated-residual pair (NX = 2), or the 16-bit rounding
+// alone (NX = 1)
 template <int FMT, int NX>
 __device__ __forceinline__ void store8_act(uint8_t* hi_base, uint8_t* lo_base, uint32_t off, const float* v)
 {
-    if (NX == 2) store8<FMT>(hi_base, lo_base, off, v);
-    else store8_hi<FMT>(hi_base, off, v);
+    if (NX == 2) {
+        uint32_t h[4], l[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) split2_neg<FMT>(v[2 * q], v[2 * q + 1], h[q], l[q]);
+        *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(lo_base + off) = make_uint4(l[0], l[1], l[2], l[3]);
+    } else {
+        store8_hi<FMT>(hi_base, off, v);
+    }
 }
 
 

@@ -121,6 +121,22 @@ def mufu_per_edge(K, F):
     return {"fwd": K + 2 * F - F // 4, "bwd": K + 3 * F - F // 4}
 
 
+def fused_work_per_step(K, F, L, E_cut):
+    """Algorithmic FLOP and MUFU operations per MD step of the two fused kernels.  The filter
+    network K -> F -> F costs 2 (K F + F^2) FLOP per evaluation.  k_cfconv_fwd evaluates it once
+    per directed edge inside the cutoff in each interaction's forward (E_cut) and once per edge of
+    the complementary list (E_cut / 2) in the dE/dh launches of interactions 1..L-1; k_cfconv_bwd
+    forms W and its derivative W' (twice the contraction) per unordered pair (E_cut / 2) in every
+    interaction."""
+    f1 = 2.0 * (K * F + F * F)
+    mu = mufu_per_edge(K, F)
+    fwd_edges = (L + (L - 1) * 0.5) * E_cut
+    return {"k_cfconv_fwd": {"classes": ("cfconv_fwd", "cfconv_dh"), "flop_step": f1 * fwd_edges,
+                             "mufu_step": mu["fwd"] * fwd_edges},
+            "k_cfconv_bwd": {"classes": ("cfconv_bwd",), "flop_step": 2.0 * f1 * L * E_cut / 2,
+                             "mufu_step": mu["bwd"] * L * E_cut / 2}}
+
+
 def hbm_kernel_bytes(w, E_list, E_cut):
     """Algorithmic HBM bytes of the memory-bound kernels (per launch; the neighbour build per
     build).  forces: per listed edge col, rev and s_e (4 B each), per atom the position (16 B),
@@ -334,18 +350,8 @@ def run_native(args):
         clk_prof = clocks.window(prof_t0, prof_t1)
         E_list, E_cut = _edge_stats(model, p.cpu().numpy(), w)
         peaks, src = _peaks()
-        # algorithmic work per step: the forward kernel contracts the filter MLP (45,568 FLOP for
-        # the 64 x 269 model) once per directed edge inside the cutoff in each interaction's
-        # forward, and once per edge of the complementary half list (E_cut / 2) in the dE/dh
-        # launches of interactions 1..L-1; the pair kernel forms W and its derivative W' (twice
-        # the contraction) per unordered pair (E_cut / 2) in every interaction
-        f1 = 2.0 * (w.K * w.F + w.F * w.F)
-        mu = mufu_per_edge(w.K, w.F)
-        fwd_edges = (w.L + (w.L - 1) * 0.5) * E_cut
-        kern = {"k_cfconv_fwd": {"classes": ("cfconv_fwd", "cfconv_dh"), "flop_step": f1 * fwd_edges,
-                                 "mufu_step": mu["fwd"] * fwd_edges},
-                "k_cfconv_bwd": {"classes": ("cfconv_bwd",), "flop_step": 2.0 * f1 * w.L * E_cut / 2,
-                                 "mufu_step": mu["bwd"] * w.L * E_cut / 2}}
+        # algorithmic work per step (45,568 FLOP per filter evaluation for the 64 x 269 model)
+        kern = fused_work_per_step(w.K, w.F, w.L, E_cut)
         for k, v in kern.items():
             v["ms"] = sum(prof[c][0] for c in v["classes"])        # over the n_rb profiled steps
             v["launches"] = sum(prof[c][1] for c in v["classes"])
@@ -411,7 +417,7 @@ def run_native(args):
                     "e2e_how": "sum over kernel classes of max(tensor FLOP / tensor peak, MUFU ops / MUFU peak, "
                                "algorithmic HBM bytes / HBM peak), divided by the measured ms_per_step",
                     "fused_kernels": fused,
-                    "mufu_per_edge_interaction": mu, "mufu_peak_per_s": mufu_peak,
+                    "mufu_per_edge_interaction": mufu_per_edge(w.K, w.F), "mufu_peak_per_s": mufu_peak,
                     "hbm_peak_GBs": peaks["hbm_gbs"], "hbm_kernels": hbm_kernels}
         cfg = dict(_workload_config(w, n_rb, ws))
         cfg.update({"edges_listed": E_list, "edges_within_cutoff": E_cut,

@@ -62,3 +62,28 @@ def test_traffic_figure_is_keyed_to_the_kernel_sources(tmp_path, monkeypatch):
         h.update(open(os.path.join(ROOT, src), "rb").read())
     current = h.hexdigest()[:16] == d["sources_sha256_16"]
     assert (bench._traffic("k_cfconv_bwd") is not None) == current
+
+
+def test_fused_work_model_from_the_filter_shape():
+    """The roofline's algorithmic work: the filter network K -> F -> F costs 2 (K F + F^2)
+    FLOP per evaluation (45,568 for K = 50, F = 128); per step the forward kernel evaluates it
+    L E_cut times in the forwards and (L - 1) E_cut / 2 times in the dE/dh launches over the
+    complementary list, and the pair kernel forms value and derivative once per unordered pair
+    (2 L E_cut / 2 evaluations).  MUFU operations: K Gaussian exponentials per evaluation, per
+    feature an exponential and a logarithm for the softplus (a quarter of the exponentials on the
+    FMA pipe), and in the pair kernel one more exponential per feature for the logistic."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    K, F, L, E = 50, 128, 3, 1_000_000
+    assert b.mufu_per_edge(K, F) == {"fwd": 50 + 256 - 32, "bwd": 50 + 384 - 32}
+    work = b.fused_work_per_step(K, F, L, E)
+    per_eval = 2 * (50 * 128 + 128 * 128)
+    assert per_eval == 45_568
+    assert work["k_cfconv_fwd"]["flop_step"] == per_eval * (3 * E + 2 * E / 2)
+    assert work["k_cfconv_bwd"]["flop_step"] == per_eval * 2 * 3 * E / 2
+    assert work["k_cfconv_fwd"]["mufu_step"] == 274 * (3 * E + 2 * E / 2)
+    assert work["k_cfconv_bwd"]["mufu_step"] == 402 * 3 * E / 2
+    # one interaction: no dE/dh launch at all
+    assert b.fused_work_per_step(K, F, 1, E)["k_cfconv_fwd"]["flop_step"] == per_eval * E
